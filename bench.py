@@ -1,0 +1,382 @@
+"""Benchmark: exact causal attention forward + backward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl lca|reference]
+
+A step is one pass of the whole path over one batch: lca_attn_fwd over the
+key/value chunks in ring order (with the (O, lse) merge) followed by
+lca_attn_bwd.  The default workload is the Llama-2-7B attention layer:
+B=1, H=32, d=128, S=32768, bf16, causal, 8 KV chunks of 4096, RoPE inputs.
+
+Under torchrun (N > 1) every rank runs an independent replica of the
+workload on its own GPU (the path has no exchange step to shard over);
+timing is the maximum over ranks.  Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same
+workload on this host's cores (the oracle is the only other implementation
+there is).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "causal attention TFLOP/s fwd+bwd (bf16, 1×B200) & fraction of dense BF16 peak"
+NOMINAL_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="llama2_7b_s32k")
+    ap.add_argument("--impl", default="lca", choices=["lca", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "long_context_exact_attention_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_record(kernel):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    rec = d.get(kernel)
+    if not rec or rec.get("source_sha") != source_sha():
+        return None
+    return rec
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.rows = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([x.strip() for x in line.split(",")])
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = [r for r in self.rows if len(r) >= 9]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def oracle_sample(w, seconds_target=12.0, max_rows=None):
+    """Time the fp64 oracle (as it stands) on the last R query rows of head 0
+    of workload w: forward and backward of those rows.  R doubles until one
+    run takes >= seconds_target / 4, then the timed run is repeated to about
+    seconds_target.  Returns (tflops, rows, seconds, cores)."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from long_context_exact_attention_b200.inputs import make_tensor
+
+    S = w.S
+    tok = (0, S)
+    q = make_tensor(w, "q", "cpu", tok)[:, :, :w.Hq // w.Hkv]
+    k = make_tensor(w, "k", "cpu", tok)[:, :, :1]
+    v = make_tensor(w, "v", "cpu", tok)[:, :, :1]
+    do = make_tensor(w, "dout", "cpu", tok)[:, :, :w.Hq // w.Hkv]
+    q, k, v, do = (t.contiguous() for t in (q, k, v, do))
+
+    def flops(rows):
+        vis = np.asarray(rows) + 1 if w.causal else np.full(len(rows), S)
+        return 3.5 * 4.0 * w.d * float(vis.sum()) * (w.Hq // w.Hkv)
+
+    R = 64
+    while True:
+        rows = np.arange(S - R, S)
+        t0 = time.perf_counter()
+        oracle.attention_backward_rows(q, k, v, do, w.causal, 0, 0, rows)
+        dt = time.perf_counter() - t0
+        if dt >= seconds_target / 4 or R >= S or (max_rows and R >= max_rows):
+            break
+        R *= 2
+    reps = max(1, int(round(seconds_target / max(dt, 1e-3))))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle.attention_backward_rows(q, k, v, do, w.causal, 0, 0, rows)
+    dt = (time.perf_counter() - t0) / reps
+    cores = len(os.sched_getaffinity(0))
+    return flops(rows) / dt / 1e12, R, dt, cores, reps
+
+
+# ---------------------------------------------------------------- main
+
+def main():
+    args = parse()
+    from long_context_exact_attention_b200.inputs import WORKLOADS
+    w = WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    flops_step = w.fwd_flops() + (w.bwd_flops() if w.backward else 0.0)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        for _ in range(args.warmup):
+            oracle_sample(w, seconds_target=2.0, max_rows=512)
+        vals = []
+        info = None
+        for _ in range(args.steps):
+            info = oracle_sample(w, seconds_target=5.0, max_rows=4096)
+            vals.append(info[0])
+        tf, R, dt, cores, reps = info
+        val = statistics.median(vals)
+        line = {
+            "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "S": w.S,
+                       "d": w.d, "causal": w.causal},
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": f"fp64 oracle fwd+bwd of the last {R} query rows of "
+                                       f"the {w.Hq // w.Hkv} query head(s) of key/value head 0"},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from long_context_exact_attention_b200 import lca
+    from long_context_exact_attention_b200.inputs import make_inputs
+
+    if world > 1:
+        dist.init_process_group("nccl", init_method="env://",
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.Stream(dev)
+    x = make_inputs(w, dev)
+    torch.cuda.synchronize()
+    q, k, v = x["q"], x["k"], x["v"]
+    dout = x.get("dout")
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.S), device=dev, dtype=torch.float32)
+    if w.backward:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(lca.workspace_size(q, k), device=dev, dtype=torch.uint8)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        lca.attn_fwd(q, k, v, causal=w.causal, kv_chunk=w.kv_chunk, order=w.order,
+                     q_block=w.q_block, out=out, lse=lse, stream=stream)
+        if ev:
+            ev[1].record(stream)
+        if w.backward:
+            lca.attn_bwd(q, k, v, out, lse, dout, causal=w.causal, dq=dq, dk=dk, dv=dv,
+                         workspace=ws, stream=stream)
+        if ev:
+            ev[2].record(stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    stream.synchronize()
+    lca.check(stream)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    cvd = os.environ.get("CUDA_VISIBLE_DEVICES")
+    clocks = ClockSampler(cvd.split(",")[local] if cvd else str(local))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    stop.record(stream)
+    stop.synchronize()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    lca.check(stream)
+    total_ms = start.elapsed_time(stop)
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    bwd_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_step = total_ms / args.steps
+    value = flops_step * world * args.steps / (total_ms * 1e-3) / 1e12
+
+    # ---- end to end through the C ABI with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+        hdo = dout.cpu().pin_memory() if w.backward else None
+        res = [torch.empty_like(t, device="cpu").pin_memory()
+               for t in ([out, lse] + ([dq, dk, dv] if w.backward else []))]
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv) + ((hdo,) if hdo is not None else ()))
+        d2h = sum(t.numel() * t.element_size() for t in res)
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            if hdo is not None:
+                dout.copy_(hdo, non_blocking=True)
+            step()
+            for r, d in zip(res, [out, lse] + ([dq, dk, dv] if w.backward else [])):
+                r.copy_(d, non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            e2e_step()
+            stream.synchronize()
+            n_e2e = max(2, min(args.steps, 5))
+            if world > 1:
+                dist.barrier()
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            for _ in range(n_e2e):
+                e2e_step()
+            s1.record(stream)
+            s1.synchronize()
+        e_ms = s0.elapsed_time(s1)
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": flops_step * world * n_e2e / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e_ms / n_e2e}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    pk, pk_kind = peaks()
+    sustained = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    fwd_t = statistics.median(fwd_ms)
+    bwd_t = statistics.median(bwd_ms) if w.backward else 0.0
+    if w.backward:
+        kname = "attn_bwd_bf16_sm100"
+        ach = w.bwd_flops() / (bwd_t * 1e-3) / 1e12
+    else:
+        kname = "attn_fwd_bf16_sm100"
+        ach = w.fwd_flops() / (fwd_t * 1e-3) / 1e12
+    tr = traffic_record(kname)
+    roof = {"bound": "tensor", "kernel": kname, "achieved": ach, "peak": sustained,
+            "unit": "TFLOP/s", "frac": ach / sustained, "peak_kind": f"{pk_kind} sustained bf16",
+            "traffic": tr["dram_bytes_per_launch"] if tr else None,
+            "frac_of_nominal_2250": ach / NOMINAL_BF16_TFLOPS,
+            "timing": "CUDA events around the whole lca_attn_bwd call (row-dot, main and "
+                      "dq-finalize launches), median over timed steps"
+                      if w.backward else "CUDA events around lca_attn_fwd"}
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "impl": "lca",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "S": w.S, "d": w.d,
+                   "causal": w.causal, "kv_chunk": w.kv_chunk, "order": w.order,
+                   "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (q, k, v, dout 256 MiB each); no flush"},
+        "fwd_tflops": w.fwd_flops() / (fwd_t * 1e-3) / 1e12, "fwd_ms": fwd_t,
+        "bwd_tflops": (w.bwd_flops() / (bwd_t * 1e-3) / 1e12) if w.backward else None,
+        "bwd_ms": bwd_t if w.backward else None,
+        "frac_of_peak": {"measured_burst": value / world / pk.get("bf16_tflops", 1590.0),
+                         "measured_sustained": value / world / sustained,
+                         "nominal_2250": value / world / NOMINAL_BF16_TFLOPS},
+        "roofline": roof,
+        "clocks": clk,
+        "gpu_launches": args.steps * (1 + (3 if w.backward else 0)),
+        "e2e": e2e,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        tf, R, dt, cores, reps = oracle_sample(w)
+        line["cpu_baseline"] = {
+            "value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"fp64 oracle fwd+bwd of the last {R} query rows of the "
+                      f"{w.Hq // w.Hkv} query head(s) of key/value head 0, {reps} runs, "
+                      f"{dt:.2f} s each"}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

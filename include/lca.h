@@ -1,0 +1,205 @@
+/*
+ * lca.h -- exact long-context attention on NVIDIA B200 (sm_100a): C ABI.
+ *
+ * What it computes
+ *   Exact softmax attention, softmax(Q K^T * scale + mask) V, together with
+ *   the per-row log-sum-exp (lse) and the gradients that recompute the
+ *   attention matrix from that lse.  "Attention stays exact" while it is
+ *   computed block by block, and the per-block partial results combine to
+ *   the same answer whatever order the key/value blocks arrive in (Ring
+ *   Attention with Blockwise Transformers for Near-Infinite Context,
+ *   Summary).  Full attention with no approximation is what the 700K/1M
+ *   token recipes train with (sourcepulse project card of the 1M-context
+ *   training recipe, How It Works).  LongLoRA's shifted sparse attention
+ *   (LongLoRA: Efficient Fine-tuning of Long-Context Large Language Models,
+ *   Summary) is the same computation restricted to groups, with half the
+ *   heads shifted by half a group.
+ *
+ * Layouts (all tensors dense, row-major, no padding)
+ *   q, out, dout, dq : [B, S, Hq,  d]   (token-major, head dim contiguous)
+ *   k, v, dk, dv     : [B, S, Hkv, d]
+ *   lse              : [B, Hq, S] float32, natural log of sum_j exp(scale*s_ij)
+ *   Grouped-query heads: query head h reads key/value head h / (Hq / Hkv).
+ *   Causal: key j is visible to query i iff j <= i (one position axis).
+ *
+ * Element types
+ *   LCA_BF16: q, k, v, out, dout, dq, dk, dv are bfloat16; accumulation in
+ *             float32 on the tensor cores; requires d == 128 and S a multiple
+ *             of 128.
+ *   LCA_FP32: every tensor float32, exact float32 arithmetic on CUDA cores;
+ *             d in {64, 128}, S a multiple of 64.
+ *
+ * Ownership and memory
+ *   The caller allocates every device buffer (inputs, outputs, workspace)
+ *   and keeps it alive until the stream work completes.  Pointers are device
+ *   pointers aligned to 16 bytes.  The library allocates no device memory;
+ *   it keeps no state between calls except one device error word per device.
+ *
+ * Errors
+ *   Argument errors are returned synchronously, before anything is launched.
+ *   A failed launch returns LCA_ERR_CUDA.  Every kernel bounds each of its
+ *   waits; a wait that runs out sets the device error word and the kernel
+ *   returns early (its outputs are then undefined).  lca_check() reports it.
+ *   Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *   default stream) and thread-safe.
+ */
+#ifndef LCA_H
+#define LCA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LCA_API __attribute__((visibility("default")))
+#else
+#define LCA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LCA_OK = 0,
+  LCA_ERR_INVALID_ARG = 1,  /* bad shape, pointer, alignment or option     */
+  LCA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. bf16 d=64)  */
+  LCA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed           */
+  LCA_ERR_TIMEOUT = 4,      /* a kernel wait ran out (see lca_check)       */
+  LCA_ERR_WORKSPACE = 5     /* workspace missing or smaller than required  */
+} lca_status;
+
+typedef enum { LCA_BF16 = 0, LCA_FP32 = 1 } lca_dtype;
+
+/* Order in which a query tile visits the key/value chunks.  The result does
+ * not depend on it beyond float32 rounding (Ring Attention, Summary). */
+typedef enum {
+  LCA_ORDER_INORDER = 0, /* chunks 0, 1, ..., n-1                              */
+  LCA_ORDER_RING = 1,    /* query block i visits chunks i, i-1, ..., i+1 (mod n),
+                            the order in which a ring delivers them            */
+  LCA_ORDER_CUSTOM = 2   /* opts->chunk_perm[0..n-1], a permutation of 0..n-1  */
+} lca_order;
+
+typedef struct {
+  int64_t B, Hq, Hkv, S, d;
+  int32_t dtype;  /* lca_dtype */
+  float scale;    /* softmax scale; 0 selects 1/sqrt(d) */
+} lca_shape;
+
+typedef struct {
+  int32_t order;              /* lca_order                                   */
+  const int32_t* chunk_perm;  /* HOST array of n_chunks entries (CUSTOM only) */
+  int64_t q_block;            /* RING: query-block length, 0 = kv_chunk; must
+                                 be a multiple of the tile (128 bf16, 64 fp32) */
+  uint64_t timeout_cycles;    /* per-wait budget in SM clocks; 0 = default
+                                 (2^31, about one second)                    */
+} lca_opts;
+
+#define LCA_MAX_CHUNKS 1024
+
+/* ---------------------------------------------------------------------------
+ * lca_attn_fwd -- exact attention forward over key/value chunks.
+ *   The keys are split into S / kv_chunk chunks (kv_chunk == 0: one chunk).
+ *   Each query tile attends to the chunks in the order opts selects; the
+ *   partial (O, lse) of every chunk is folded into the running result in
+ *   unnormalised form (running max m, running sum l, running O*l), which is
+ *   the log-sum-exp merge of the Ring Attention summary carried out chunk by
+ *   chunk.  Causal chunks/tiles that hold no visible key are skipped.
+ *   q, k, v: inputs (layouts above).  out: [B,S,Hq,d] output, same dtype.
+ *   lse: [B,Hq,S] float32 output.  opts may be NULL (in-order).
+ *   Errors: LCA_ERR_INVALID_ARG when a pointer is NULL or misaligned, a
+ *   dimension is <= 0, Hq % Hkv != 0, kv_chunk is not a multiple of the tile
+ *   or does not divide S, the chunk count exceeds LCA_MAX_CHUNKS, or the
+ *   permutation is invalid; LCA_ERR_UNSUPPORTED for shapes outside the
+ *   element-type limits above.
+ * ------------------------------------------------------------------------- */
+LCA_API lca_status lca_attn_fwd(const lca_shape* shape, const void* q, const void* k,
+                        const void* v, int causal, int64_t kv_chunk,
+                        const lca_opts* opts, void* out, float* lse,
+                        void* stream);
+
+/* Bytes of device workspace lca_attn_bwd / lca_s2attn_bwd need: float32
+ * rows D_i = dout_i . out_i ([B,Hq,S]) and, for bf16, a float32 dq
+ * accumulator ([B,S,Hq,d]).  Returns 0 for an invalid shape. */
+LCA_API size_t lca_attn_bwd_workspace_size(const lca_shape* shape);
+
+/* ---------------------------------------------------------------------------
+ * lca_attn_bwd -- gradients of sum(dout * out) with respect to q, k, v.
+ *   P is recomputed from q, k and the saved lse (no attention matrix is
+ *   stored): P_ij = exp(scale*s_ij - lse_i), dV = P^T dO, dP = dO V^T,
+ *   dS = P o (dP - D), dQ = scale dS K, dK = scale dS^T Q, D_i = dO_i . O_i.
+ *   With grouped-query heads dk/dv sum over the query heads of a group.
+ *   out and lse must come from lca_attn_fwd on the same inputs and `causal`.
+ *   dq, dk, dv: outputs, input dtype, fully overwritten.  workspace: device
+ *   buffer of ws_bytes >= lca_attn_bwd_workspace_size(shape) bytes, owned
+ *   by the caller, contents need not be initialised.
+ *   Errors: as lca_attn_fwd; LCA_ERR_WORKSPACE when the workspace is NULL
+ *   or too small.
+ * ------------------------------------------------------------------------- */
+LCA_API lca_status lca_attn_bwd(const lca_shape* shape, const void* q, const void* k,
+                        const void* v, const void* out, const float* lse,
+                        const void* dout, int causal, void* dq, void* dk,
+                        void* dv, void* workspace, size_t ws_bytes,
+                        void* stream);
+
+/* ---------------------------------------------------------------------------
+ * lca_s2attn_fwd -- LongLoRA shifted sparse attention (S2-Attn), forward.
+ *   Positions are split into S/group groups of `group`; attention runs
+ *   inside each group (causal by position within the group when `causal`).
+ *   The trailing `shift_heads` query heads (and the key/value heads they
+ *   read) are shifted by group/2: shifted position p holds original token
+ *   (p + group/2) mod S, so the last group wraps around.  Outputs and lse
+ *   are in ORIGINAL token order; the shift is applied to tile coordinates
+ *   inside the kernel, no tensor is rolled.  shift_heads == 0 gives the
+ *   unshifted short attention; group == S with shift_heads == 0 is full
+ *   attention.
+ *   Errors: as lca_attn_fwd, plus LCA_ERR_INVALID_ARG when group does not
+ *   divide S, group/2 is not a multiple of the tile, shift_heads is outside
+ *   [0, Hq], or the shifted heads do not cover whole grouped-query groups.
+ * ------------------------------------------------------------------------- */
+LCA_API lca_status lca_s2attn_fwd(const lca_shape* shape, const void* q, const void* k,
+                          const void* v, int causal, int64_t group,
+                          int64_t shift_heads, void* out, float* lse,
+                          void* stream);
+
+/* lca_s2attn_bwd -- gradients of S2-Attn; arguments as lca_attn_bwd plus
+ * group/shift_heads as lca_s2attn_fwd. */
+LCA_API lca_status lca_s2attn_bwd(const lca_shape* shape, const void* q, const void* k,
+                          const void* v, const void* out, const float* lse,
+                          const void* dout, int causal, int64_t group,
+                          int64_t shift_heads, void* dq, void* dk, void* dv,
+                          void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * lca_lse_merge -- combine two partial attention results over disjoint key
+ * sets (Ring Attention, Summary: per-block results combine independently of
+ * order):  lse = M + ln(e^(lse_a-M) + e^(lse_b-M)), M = max(lse_a, lse_b);
+ * o = e^(lse_a-lse) o_a + e^(lse_b-lse) o_b.  A row with lse = -inf is an
+ * empty partial (identity).  o_*: [rows, d] float32, lse_*: [rows] float32,
+ * all device pointers; o_out/lse_out may alias o_a/lse_a.
+ * Errors: LCA_ERR_INVALID_ARG for rows/d <= 0 or NULL pointers.
+ * ------------------------------------------------------------------------- */
+LCA_API lca_status lca_lse_merge(int64_t rows, int64_t d, const float* o_a,
+                         const float* lse_a, const float* o_b,
+                         const float* lse_b, float* o_out, float* lse_out,
+                         void* stream);
+
+/* Synchronises `stream`, then reports and clears the device error word of
+ * the current device: LCA_ERR_TIMEOUT if a kernel wait ran out since the
+ * last check, LCA_ERR_CUDA if the stream holds a CUDA error, else LCA_OK. */
+LCA_API lca_status lca_check(void* stream);
+
+/* Static description of a status code. */
+LCA_API const char* lca_status_string(lca_status s);
+
+/* Human-readable detail of the last non-OK status returned on this host
+ * thread (which argument, which CUDA error).  Never NULL. */
+LCA_API const char* lca_last_error(void);
+
+/* Library version, (major << 16) | minor. */
+LCA_API int lca_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LCA_H */

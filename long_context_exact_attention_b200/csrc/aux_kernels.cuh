@@ -1,0 +1,94 @@
+// aux_kernels.cuh -- small memory-bound kernels around the attention passes.
+//
+//   bwd_rowdot   D_i = sum_c dout_ic * out_ic (float32), the row term of
+//                dS = P o (dP - D) in the backward pass
+//   dq_finalize  dq = scale * dq_acc, float32 accumulator -> bf16
+//   lse_merge    combine two partial (O, lse) results over disjoint key
+//                sets (Ring Attention with Blockwise Transformers, Summary:
+//                per-block results combine independently of order)
+#pragma once
+
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace lca {
+
+// One warp per (token, head) row; rows ordered [B, S, H]; D written [B, H, S].
+template <typename T, int D>
+__global__ void bwd_rowdot(const T* __restrict__ out, const T* __restrict__ dout,
+                           float* __restrict__ Dst, int B, int S, int H) {
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t nrows = static_cast<int64_t>(B) * S * H;
+  if (row >= nrows) return;
+  const T* o = out + row * D;
+  const T* g = dout + row * D;
+  float acc = 0.f;
+#pragma unroll
+  for (int c = lane; c < D; c += 32) {
+    float ov, gv;
+    if constexpr (sizeof(T) == 2) {
+      ov = __bfloat162float(o[c]);
+      gv = __bfloat162float(g[c]);
+    } else {
+      ov = o[c];
+      gv = g[c];
+    }
+    acc = fmaf(ov, gv, acc);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) {
+    const int h = static_cast<int>(row % H);
+    const int64_t bs = row / H;
+    const int s = static_cast<int>(bs % S);
+    const int b = static_cast<int>(bs / S);
+    Dst[(static_cast<int64_t>(b) * H + h) * S + s] = acc;
+  }
+}
+
+// dq(bf16) = scale * acc, 8 elements per thread.
+__global__ void dq_finalize(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq,
+                            int64_t n8, float scale) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
+    const float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+    __nv_bfloat162 r[4];
+    r[0] = __floats2bfloat162_rn(a.x * scale, a.y * scale);
+    r[1] = __floats2bfloat162_rn(a.z * scale, a.w * scale);
+    r[2] = __floats2bfloat162_rn(b.x * scale, b.y * scale);
+    r[3] = __floats2bfloat162_rn(b.z * scale, b.w * scale);
+    reinterpret_cast<uint4*>(dq)[i] = *reinterpret_cast<uint4*>(r);
+  }
+}
+
+// (O, lse) merge, one warp per row.  Every lane reads the row's two lse
+// values before lane 0 overwrites lse_out, so lse_out may alias lse_a/lse_b;
+// each element of o is read and written by one thread, so o_out may alias
+// o_a/o_b.
+__global__ void lse_merge_kernel(int64_t rows, int d, const float* o_a, const float* lse_a,
+                                 const float* o_b, const float* lse_b, float* o_out,
+                                 float* lse_out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < rows;
+       r += warps) {
+    const float la = lse_a[r], lb = lse_b[r];
+    const float M = fmaxf(la, lb);
+    float wa = 0.f, wb = 0.f, l = -INFINITY;
+    if (M != -INFINITY) {
+      l = M + logf(expf(la - M) + expf(lb - M));
+      wa = expf(la - l);
+      wb = expf(lb - l);
+    }
+    __syncwarp();
+    for (int c = lane; c < d; c += 32) {
+      const int64_t i = r * d + c;
+      o_out[i] = (M == -INFINITY) ? 0.f : wa * o_a[i] + wb * o_b[i];
+    }
+    if (lane == 0) lse_out[r] = l;
+  }
+}
+
+}  // namespace lca

@@ -1,0 +1,368 @@
+// bwd_sm100.cuh -- exact attention backward, bf16, head dim 128, sm_100a.
+//
+// Gradients of sum(dO * O), recomputing the attention matrix from the saved
+// log-sum-exp instead of storing it (the attention-level form of activation
+// checkpointing the long-context recipes rely on: sourcepulse project card
+// of the 1M-context recipe, How It Works).  With D_i = dO_i . O_i:
+//   S^T  = K Q^T                  P^T = exp2(S^T * c - lse_i * log2 e)
+//   dP^T = V dO^T                 dS^T = P^T o (dP^T - D_i)
+//   dV  += P^T dO                 dK  += dS^T Q          (TMEM accumulators)
+//   dQ_i = dS K  -> fp32 atomics into the dq accumulator (scale applied later)
+//
+// One CTA per (key tile of 128, key/value head, batch); it loops over the
+// query heads of its grouped-query group and over the query tiles that can
+// see the key tile, so dK/dV of a key tile finish inside one CTA.
+// Roles (10 warps):
+//   warp 0      TMA producer: K, V once; Q, dO tiles plus lse/D rows per step
+//   warp 1      TMEM owner; lane 0 issues the five MMAs of every step
+//   warps 2..5  P/dS warpgroup: one key row per thread
+//   warps 6..9  dQ warpgroup: one query row per thread, drains dQ from TMEM
+//               and adds it to global memory; writes dV at the end
+// TMEM: S^T [0,128) | dP^T and then dQ [128,256) | dV [256,384) | dK [384,512)
+// Shared memory (128-byte swizzle): K | V | Q | dO | P^T | dS^T | lse | D.
+#pragma once
+
+#include "ptx.cuh"
+#include "sched.cuh"
+
+namespace lca {
+
+namespace bwd {
+
+constexpr int kTile = 128;
+constexpr int kD = 128;
+constexpr uint32_t kHalf = kTile * 64 * 2;
+constexpr uint32_t kTileB = 2 * kHalf;
+constexpr int kThreads = 320;
+
+constexpr uint32_t kOffK = 0;
+constexpr uint32_t kOffV = kOffK + kTileB;
+constexpr uint32_t kOffQ = kOffV + kTileB;
+constexpr uint32_t kOffO = kOffQ + kTileB;    // dO
+constexpr uint32_t kOffP = kOffO + kTileB;    // P^T
+constexpr uint32_t kOffS = kOffP + kTileB;    // dS^T
+constexpr uint32_t kOffL = kOffS + kTileB;    // lse[128]
+constexpr uint32_t kOffD = kOffL + 512;       // D[128]
+constexpr uint32_t kOffBar = kOffD + 512;
+constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
+
+enum {
+  B_KV = 0,
+  B_QFULL,
+  B_QEMPTY,
+  B_SFULL,
+  B_SFREE,   // 128 arrivals
+  B_PFULL,   // 128 arrivals
+  B_PFREE,
+  B_DQFULL,
+  B_DQFREE,  // 128 arrivals
+  B_DONE,
+  B_DRAIN,
+  NUM_BARS
+};
+
+constexpr uint32_t kIdescKK = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T
+constexpr uint32_t kIdescKM = idesc_bf16_f32(128, 128, false, true);   // dV, dK
+constexpr uint32_t kIdescMM = idesc_bf16_f32(128, 128, true, true);    // dQ
+
+struct Args {
+  int B, Hq, Hkv, S;
+  float scale;
+  float scale_log2;
+  unsigned long long budget;
+  const float* lse;      // [B,Hq,S]
+  const float* Drow;     // [B,Hq,S]
+  float* dq_acc;         // [B,S,Hq,d] fp32, zeroed
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  AttnSched sched;
+};
+
+}  // namespace bwd
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+__global__ void __launch_bounds__(bwd::kThreads, 1)
+    attn_bwd_bf16_sm100(const __grid_constant__ CUtensorMap tmQ,
+                        const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV,
+                        const __grid_constant__ CUtensorMap tmDO,
+                        const __grid_constant__ bwd::Args a) {
+  using namespace bwd;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t sK = base + kOffK, sV = base + kOffV, sQ = base + kOffQ, sO = base + kOffO;
+  const uint32_t sP = base + kOffP, sS = base + kOffS, sL = base + kOffL, sD = base + kOffD;
+  const float* lse_s = reinterpret_cast<const float*>(gbase + kOffL);
+  const float* d_s = reinterpret_cast<const float*>(gbase + kOffD);
+  const uint32_t bars = base + kOffBar;
+  auto bar = [&](int i) { return bars + 8u * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kOffBar + 8 * NUM_BARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + kOffBar + 8 * NUM_BARS + 8);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const AttnSched& sc = a.sched;
+  const int rep = a.Hq / a.Hkv;
+  const int BG = a.B * a.Hkv;
+  // Longest causal work first: key tile 0 sees every query tile.
+  const int kt = static_cast<int>(blockIdx.x) / BG;
+  const int bg = static_cast<int>(blockIdx.x) % BG;
+  const int g = bg % a.Hkv;
+  const int b = bg / a.Hkv;
+  const bool shifted = head_shifted(sc, g * rep);
+  const int ktok0 = token_tile(sc, kt, shifted) * kTile;
+  QWalk qw;
+  qw.init(&sc, kt);
+  const int nq = qw.count();
+  const int nsteps = rep * nq;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NUM_BARS; ++i) {
+      const uint32_t cnt = (i == B_SFREE || i == B_PFULL || i == B_DQFREE) ? 128u : 1u;
+      mbar_init(bar(i), cnt);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  WaitCtl wc{abort_flag, a.budget};
+  const int row0 = b * a.S;
+
+  if (warp == 0) {
+    // =================================================== TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmDO);
+      mbar_expect_tx(bar(B_KV), 2 * kTileB);
+      tma_load_3d(sK, &tmK, bar(B_KV), 0, g, row0 + ktok0);
+      tma_load_3d(sK + kHalf, &tmK, bar(B_KV), 64, g, row0 + ktok0);
+      tma_load_3d(sV, &tmV, bar(B_KV), 0, g, row0 + ktok0);
+      tma_load_3d(sV + kHalf, &tmV, bar(B_KV), 64, g, row0 + ktok0);
+      bool ok = true;
+      int issued = 0;
+      for (int i = 0; i < nsteps && ok; ++i) {
+        const int h = g * rep + i / nq;
+        const int qt = qw.t + i % nq;
+        const int qtok0 = token_tile(sc, qt, shifted) * kTile;
+        if (i >= 1) ok = wait_bar(bar(B_QEMPTY), (i - 1) & 1, wc, 111);
+        if (!ok) break;
+        mbar_expect_tx(bar(B_QFULL), 2 * kTileB + 1024);
+        tma_load_3d(sQ, &tmQ, bar(B_QFULL), 0, h, row0 + qtok0);
+        tma_load_3d(sQ + kHalf, &tmQ, bar(B_QFULL), 64, h, row0 + qtok0);
+        tma_load_3d(sO, &tmDO, bar(B_QFULL), 0, h, row0 + qtok0);
+        tma_load_3d(sO + kHalf, &tmDO, bar(B_QFULL), 64, h, row0 + qtok0);
+        const size_t ro = (static_cast<size_t>(b) * a.Hq + h) * a.S + qtok0;
+        bulk_load(sL, a.lse + ro, 512, bar(B_QFULL));
+        bulk_load(sD, a.Drow + ro, 512, bar(B_QFULL));
+        ++issued;
+      }
+      if (!ok) {
+        drain_bar(bar(B_KV), 0, a.budget);
+        if (issued) drain_bar(bar(B_QFULL), (issued - 1) & 1, a.budget);
+      }
+    }
+  } else if (warp == 1) {
+    // =================================================== MMA issuer
+    if (lane == 0) {
+      const uint32_t tSt = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 384;
+      bool ok = wait_bar(bar(B_KV), 0, wc, 211);
+      for (int i = 0; i < nsteps && ok; ++i) {
+        ok = wait_bar(bar(B_QFULL), i & 1, wc, 212);
+        if (ok && i >= 1) ok = wait_bar(bar(B_SFREE), (i - 1) & 1, wc, 213);
+        if (ok && i >= 1) ok = wait_bar(bar(B_DQFREE), (i - 1) & 1, wc, 214);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t off = (k >> 2) * kHalf + (k & 3) * 32;
+          mma_bf16_ss(tSt, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024),
+                      kIdescKK, k > 0);
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t off = (k >> 2) * kHalf + (k & 3) * 32;
+          mma_bf16_ss(tdP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sO + off, 16, 1024),
+                      kIdescKK, k > 0);
+        }
+        tc_commit(bar(B_SFULL));
+        ok = wait_bar(bar(B_PFULL), i & 1, wc, 215);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t offa = (k >> 2) * kHalf + (k & 3) * 32;
+          mma_bf16_ss(tdV, sdesc_sw128(sP + offa, 16, 1024),
+                      sdesc_sw128(sO + k * 2048, kHalf, 1024), kIdescKM, (i > 0 || k > 0));
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t offa = (k >> 2) * kHalf + (k & 3) * 32;
+          mma_bf16_ss(tdK, sdesc_sw128(sS + offa, 16, 1024),
+                      sdesc_sw128(sQ + k * 2048, kHalf, 1024), kIdescKM, (i > 0 || k > 0));
+        }
+        tc_commit(bar(B_QEMPTY));
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          mma_bf16_ss(tdP, sdesc_sw128(sS + k * 2048, kHalf, 1024),
+                      sdesc_sw128(sK + k * 2048, kHalf, 1024), kIdescMM, k > 0);
+        }
+        tc_commit(bar(B_DQFULL));
+        tc_commit(bar(B_PFREE));
+      }
+      tc_commit(bar(B_DONE));
+      tc_commit(bar(B_DRAIN));
+      drain_bar(bar(B_DRAIN), 0, a.budget);
+    }
+  } else if (warp < 6) {
+    // =================================================== P / dS warpgroup
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;  // key row
+    const uint32_t lad = static_cast<uint32_t>(wq * 32) << 16;
+    const float c = a.scale_log2;
+    const float L2E = 1.4426950408889634f;
+    bool ok = true;
+    for (int i = 0; i < nsteps && ok; ++i) {
+      const int qt = qw.t + i % nq;
+      ok = wait_bar(bar(B_SFULL), i & 1, wc, 311);
+      if (ok) ok = wait_bar(bar(B_QFULL), i & 1, wc, 312);
+      if (ok && i >= 1) ok = wait_bar(bar(B_PFREE), (i - 1) & 1, wc, 313);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const bool diag = sc.causal && qt == kt;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        float s[32], dp[32];
+        tmem_ld32(tmem + lad + cc * 32, s);
+        tmem_ld32(tmem + lad + 128 + cc * 32, dp);
+        uint32_t pp[16], dd[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int q0 = cc * 32 + e;
+          float p0 = ex2_approx(fmaf(s[e], c, -lse_s[q0] * L2E));
+          float p1 = ex2_approx(fmaf(s[e + 1], c, -lse_s[q0 + 1] * L2E));
+          if (diag && r > q0) p0 = 0.f;
+          if (diag && r > q0 + 1) p1 = 0.f;
+          const float d0 = p0 * (dp[e] - d_s[q0]);
+          const float d1 = p1 * (dp[e + 1] - d_s[q0 + 1]);
+          pp[e >> 1] = pack_bf16x2(p0, p1);
+          dd[e >> 1] = pack_bf16x2(d0, d1);
+        }
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const int ch = cc * 4 + v;
+          const int half = ch >> 3, cw = ch & 7;
+          const uint32_t off = half * kHalf + r * 128 + ((cw ^ (r & 7)) << 4);
+          st_shared_v4(sP + off, pp[4 * v], pp[4 * v + 1], pp[4 * v + 2], pp[4 * v + 3]);
+          st_shared_v4(sS + off, dd[4 * v], dd[4 * v + 1], dd[4 * v + 2], dd[4 * v + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(B_SFREE));
+      fence_async_smem();
+      mbar_arrive(bar(B_PFULL));
+    }
+    // ---- dK = scale * acc -> bf16
+    if (ok) ok = wait_bar(bar(B_DONE), 0, wc, 314);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      tc_fence_after();
+      __nv_bfloat16* row = a.dk + ((static_cast<size_t>(b) * a.S + ktok0 + r) * a.Hkv + g) * kD;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        float o[32];
+        tmem_ld32(tmem + lad + 384 + cc * 32, o);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          uint4 pk;
+          pk.x = pack_bf16x2(o[v * 8 + 0] * a.scale, o[v * 8 + 1] * a.scale);
+          pk.y = pack_bf16x2(o[v * 8 + 2] * a.scale, o[v * 8 + 3] * a.scale);
+          pk.z = pack_bf16x2(o[v * 8 + 4] * a.scale, o[v * 8 + 5] * a.scale);
+          pk.w = pack_bf16x2(o[v * 8 + 6] * a.scale, o[v * 8 + 7] * a.scale);
+          *reinterpret_cast<uint4*>(row + cc * 32 + v * 8) = pk;
+        }
+      }
+    }
+  } else {
+    // =================================================== dQ warpgroup
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;  // query row (dQ) / key row (dV)
+    const uint32_t lad = static_cast<uint32_t>(wq * 32) << 16;
+    bool ok = true;
+    for (int i = 0; i < nsteps && ok; ++i) {
+      const int h = g * rep + i / nq;
+      const int qt = qw.t + i % nq;
+      const int qtok0 = token_tile(sc, qt, shifted) * kTile;
+      ok = __all_sync(0xffffffffu, wait_bar(bar(B_DQFULL), i & 1, wc, 411));
+      if (!ok) break;
+      tc_fence_after();
+      float dq[128];
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        float tmp[32];
+        tmem_ld32(tmem + lad + 128 + cc * 32, tmp);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) dq[cc * 32 + e] = tmp[e];
+      }
+      tc_fence_before();
+      mbar_arrive(bar(B_DQFREE));
+      float4* dst = reinterpret_cast<float4*>(
+          a.dq_acc + ((static_cast<size_t>(b) * a.S + qtok0 + r) * a.Hq + h) * kD);
+#pragma unroll
+      for (int v = 0; v < 32; ++v) {
+        atomicAdd(dst + v, make_float4(dq[4 * v], dq[4 * v + 1], dq[4 * v + 2], dq[4 * v + 3]));
+      }
+    }
+    // ---- dV -> bf16
+    if (ok) ok = wait_bar(bar(B_DONE), 0, wc, 412);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      tc_fence_after();
+      __nv_bfloat16* row = a.dv + ((static_cast<size_t>(b) * a.S + ktok0 + r) * a.Hkv + g) * kD;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        float o[32];
+        tmem_ld32(tmem + lad + 256 + cc * 32, o);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          uint4 pk;
+          pk.x = pack_bf16x2(o[v * 8 + 0], o[v * 8 + 1]);
+          pk.y = pack_bf16x2(o[v * 8 + 2], o[v * 8 + 3]);
+          pk.z = pack_bf16x2(o[v * 8 + 4], o[v * 8 + 5]);
+          pk.w = pack_bf16x2(o[v * 8 + 6], o[v * 8 + 7]);
+          *reinterpret_cast<uint4*>(row + cc * 32 + v * 8) = pk;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace lca

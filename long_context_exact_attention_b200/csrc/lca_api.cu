@@ -1,0 +1,477 @@
+// lca_api.cu -- the C ABI of liblca (declared in include/lca.h): argument
+// validation, TMA descriptor encoding, launch configuration.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/lca.h"
+#include "aux_kernels.cuh"
+#include "bwd_sm100.cuh"
+#include "fwd_sm100.cuh"
+#include "ptx.cuh"
+#include "sched.cuh"
+#include "simt_f32.cuh"
+
+using namespace lca;
+
+namespace {
+
+thread_local std::string t_last_error = "no error";
+
+lca_status fail(lca_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  t_last_error = std::string(lca_status_string(s)) + ": " + buf;
+  return s;
+}
+
+lca_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(LCA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr unsigned long long kDefaultBudget = 1ull << 31;
+
+struct Common {
+  int B, Hq, Hkv, S, d;
+  int dtype;
+  float scale;
+  int tile;
+};
+
+lca_status check_shape(const lca_shape* sh, Common* c) {
+  if (!sh) return fail(LCA_ERR_INVALID_ARG, "shape is NULL");
+  if (sh->B <= 0 || sh->Hq <= 0 || sh->Hkv <= 0 || sh->S <= 0 || sh->d <= 0)
+    return fail(LCA_ERR_INVALID_ARG, "dimensions must be positive");
+  if (sh->Hq % sh->Hkv) return fail(LCA_ERR_INVALID_ARG, "Hq %% Hkv != 0");
+  if (sh->B > (1 << 20) || sh->Hq > 4096 || sh->S > (1ll << 26))
+    return fail(LCA_ERR_INVALID_ARG, "dimension too large");
+  if (sh->B * sh->S > (1ll << 31) - 1)
+    return fail(LCA_ERR_INVALID_ARG, "B*S must fit in 31 bits");
+  if (sh->dtype != LCA_BF16 && sh->dtype != LCA_FP32)
+    return fail(LCA_ERR_INVALID_ARG, "unknown dtype %d", sh->dtype);
+  if (!(sh->scale >= 0.f) || std::isinf(sh->scale))
+    return fail(LCA_ERR_INVALID_ARG, "scale must be finite and >= 0");
+  c->B = static_cast<int>(sh->B);
+  c->Hq = static_cast<int>(sh->Hq);
+  c->Hkv = static_cast<int>(sh->Hkv);
+  c->S = static_cast<int>(sh->S);
+  c->d = static_cast<int>(sh->d);
+  c->dtype = sh->dtype;
+  c->scale = sh->scale > 0.f ? sh->scale : 1.0f / std::sqrt(static_cast<float>(sh->d));
+  if (sh->dtype == LCA_BF16) {
+    if (sh->d != 128) return fail(LCA_ERR_UNSUPPORTED, "bf16 path needs d == 128 (got %lld)",
+                                  static_cast<long long>(sh->d));
+    c->tile = 128;
+  } else {
+    if (sh->d != 64 && sh->d != 128)
+      return fail(LCA_ERR_UNSUPPORTED, "fp32 path needs d in {64, 128}");
+    c->tile = 64;
+  }
+  if (sh->S % c->tile)
+    return fail(LCA_ERR_UNSUPPORTED, "S must be a multiple of %d", c->tile);
+  return LCA_OK;
+}
+
+lca_status check_ptrs(std::initializer_list<const void*> ps) {
+  int i = 0;
+  for (const void* p : ps) {
+    if (!p) return fail(LCA_ERR_INVALID_ARG, "pointer argument %d is NULL", i);
+    if (!aligned16(p)) return fail(LCA_ERR_INVALID_ARG, "pointer argument %d not 16-byte aligned", i);
+    ++i;
+  }
+  return LCA_OK;
+}
+
+// Chunked (ring-simulating) schedule.
+lca_status make_chunk_sched(const Common& c, int causal, int64_t kv_chunk, const lca_opts* o,
+                            AttnSched* s) {
+  std::memset(s, 0, sizeof *s);
+  s->n_tiles = c.S / c.tile;
+  s->causal = causal ? 1 : 0;
+  const int64_t chunk = kv_chunk == 0 ? c.S : kv_chunk;
+  if (chunk < 0 || chunk % c.tile || c.S % chunk)
+    return fail(LCA_ERR_INVALID_ARG, "kv_chunk must be a multiple of %d dividing S", c.tile);
+  s->tiles_per_chunk = static_cast<int>(chunk / c.tile);
+  s->n_chunks = static_cast<int>(c.S / chunk);
+  if (s->n_chunks > LCA_MAX_CHUNKS)
+    return fail(LCA_ERR_INVALID_ARG, "%d chunks exceed LCA_MAX_CHUNKS", s->n_chunks);
+  s->order = o ? o->order : LCA_ORDER_INORDER;
+  if (s->order < 0 || s->order > 2) return fail(LCA_ERR_INVALID_ARG, "unknown chunk order");
+  int64_t qb = (o && o->q_block) ? o->q_block : chunk;
+  if (qb <= 0 || qb % c.tile)
+    return fail(LCA_ERR_INVALID_ARG, "q_block must be a positive multiple of %d", c.tile);
+  s->q_block_tiles = static_cast<int>(qb / c.tile);
+  if (s->order == LCA_ORDER_CUSTOM) {
+    if (!o->chunk_perm) return fail(LCA_ERR_INVALID_ARG, "CUSTOM order needs chunk_perm");
+    bool seen[LCA_MAX_CHUNKS] = {};
+    for (int i = 0; i < s->n_chunks; ++i) {
+      const int v = o->chunk_perm[i];
+      if (v < 0 || v >= s->n_chunks || seen[v])
+        return fail(LCA_ERR_INVALID_ARG, "chunk_perm is not a permutation of 0..%d",
+                    s->n_chunks - 1);
+      seen[v] = true;
+      s->perm[i] = static_cast<uint16_t>(v);
+    }
+  }
+  return LCA_OK;
+}
+
+lca_status make_s2_sched(const Common& c, int causal, int64_t group, int64_t shift_heads,
+                         AttnSched* s) {
+  std::memset(s, 0, sizeof *s);
+  if (group <= 0 || c.S % group || group % 2 || (group / 2) % c.tile)
+    return fail(LCA_ERR_INVALID_ARG,
+                "group must divide S and group/2 must be a multiple of %d", c.tile);
+  if (shift_heads < 0 || shift_heads > c.Hq)
+    return fail(LCA_ERR_INVALID_ARG, "shift_heads outside [0, Hq]");
+  const int rep = c.Hq / c.Hkv;
+  if ((c.Hq - shift_heads) % rep)
+    return fail(LCA_ERR_INVALID_ARG, "shifted heads must cover whole grouped-query groups");
+  s->n_tiles = c.S / c.tile;
+  s->causal = causal ? 1 : 0;
+  s->s2 = 1;
+  s->n_chunks = 1;
+  s->tiles_per_chunk = s->n_tiles;
+  s->q_block_tiles = s->n_tiles;
+  s->group_tiles = static_cast<int>(group / c.tile);
+  s->shift_tiles = static_cast<int>(group / 2 / c.tile);
+  s->first_shifted_head = static_cast<int>(c.Hq - shift_heads);
+  return LCA_OK;
+}
+
+// ---------------------------------------------------------------- TMA maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [tokens][heads][128] bf16 viewed 3-D; box = 64 head dims x 1 head x 128 tokens.
+lca_status make_map(CUtensorMap* m, const void* ptr, int64_t tokens, int64_t heads) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(LCA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(heads),
+                              static_cast<cuuint64_t>(tokens)};
+  const cuuint64_t strides[2] = {128 * 2, static_cast<cuuint64_t>(heads) * 128 * 2};
+  const cuuint32_t box[3] = {64, 1, 128};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(LCA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return LCA_OK;
+}
+
+// Raise the dynamic shared-memory limit of a kernel once per device.
+template <typename K>
+lca_status ensure_smem(K kernel, size_t bytes, int slot) {
+  static std::mutex mu;
+  static bool done[64][8] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lk(mu);
+  if (dev < 64 && done[dev][slot]) return LCA_OK;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(bytes));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  if (dev < 64) done[dev][slot] = true;
+  return LCA_OK;
+}
+
+lca_status launched(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return LCA_OK;
+}
+
+unsigned long long budget_of(const lca_opts* o) {
+  return (o && o->timeout_cycles) ? o->timeout_cycles : kDefaultBudget;
+}
+
+// ---------------------------------------------------------------- forward
+lca_status run_fwd(const Common& c, const AttnSched& s, const void* q, const void* k,
+                   const void* v, void* out, float* lse, unsigned long long budget,
+                   cudaStream_t st) {
+  const int64_t tokens = static_cast<int64_t>(c.B) * c.S;
+  const unsigned grid = static_cast<unsigned>(s.n_tiles) * c.B * c.Hq;
+  if (c.dtype == LCA_BF16) {
+    CUtensorMap mq, mk, mv;
+    lca_status r;
+    if ((r = make_map(&mq, q, tokens, c.Hq)) != LCA_OK) return r;
+    if ((r = make_map(&mk, k, tokens, c.Hkv)) != LCA_OK) return r;
+    if ((r = make_map(&mv, v, tokens, c.Hkv)) != LCA_OK) return r;
+    if ((r = ensure_smem(attn_fwd_bf16_sm100, fwd::kSmemBytes, 0)) != LCA_OK) return r;
+    fwd::Args a;
+    a.B = c.B;
+    a.Hq = c.Hq;
+    a.Hkv = c.Hkv;
+    a.S = c.S;
+    a.scale_log2 = c.scale * 1.4426950408889634f;
+    a.budget = budget;
+    a.out = static_cast<__nv_bfloat16*>(out);
+    a.lse = lse;
+    a.sched = s;
+    attn_fwd_bf16_sm100<<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(mq, mk, mv, a);
+    return launched("attn_fwd_bf16_sm100");
+  }
+  f32::Args a{};
+  a.q = static_cast<const float*>(q);
+  a.k = static_cast<const float*>(k);
+  a.v = static_cast<const float*>(v);
+  a.o_out = static_cast<float*>(out);
+  a.lse_out = lse;
+  a.B = c.B;
+  a.Hq = c.Hq;
+  a.Hkv = c.Hkv;
+  a.S = c.S;
+  a.scale = c.scale;
+  a.sched = s;
+  lca_status r;
+  if (c.d == 64) {
+    if ((r = ensure_smem(f32::attn_fwd_f32<64>, f32::fwd_smem<64>(), 1)) != LCA_OK) return r;
+    f32::attn_fwd_f32<64><<<grid, f32::kThreads, f32::fwd_smem<64>(), st>>>(a);
+  } else {
+    if ((r = ensure_smem(f32::attn_fwd_f32<128>, f32::fwd_smem<128>(), 2)) != LCA_OK) return r;
+    f32::attn_fwd_f32<128><<<grid, f32::kThreads, f32::fwd_smem<128>(), st>>>(a);
+  }
+  return launched("attn_fwd_f32");
+}
+
+// ---------------------------------------------------------------- backward
+size_t ws_d_bytes(const Common& c) {
+  const size_t n = static_cast<size_t>(c.B) * c.Hq * c.S * sizeof(float);
+  return (n + 255) & ~static_cast<size_t>(255);
+}
+size_t ws_bytes_of(const Common& c) {
+  size_t n = ws_d_bytes(c);
+  if (c.dtype == LCA_BF16) n += static_cast<size_t>(c.B) * c.S * c.Hq * c.d * sizeof(float);
+  return n;
+}
+
+lca_status run_bwd(const Common& c, const AttnSched& s, const void* q, const void* k,
+                   const void* v, const void* out, const float* lse, const void* dout, void* dq,
+                   void* dk, void* dv, void* ws, size_t ws_bytes, unsigned long long budget,
+                   cudaStream_t st) {
+  if (!ws) return fail(LCA_ERR_WORKSPACE, "workspace is NULL");
+  if (ws_bytes < ws_bytes_of(c))
+    return fail(LCA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes,
+                ws_bytes_of(c));
+  if (!aligned16(ws)) return fail(LCA_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+  float* Drow = static_cast<float*>(ws);
+  const int64_t rows = static_cast<int64_t>(c.B) * c.S * c.Hq;
+  const unsigned rd_blocks = static_cast<unsigned>((rows * 32 + 255) / 256);
+  const unsigned grid = static_cast<unsigned>(s.n_tiles) * c.B * c.Hkv;
+  if (c.dtype == LCA_BF16) {
+    float* acc = reinterpret_cast<float*>(static_cast<char*>(ws) + ws_d_bytes(c));
+    const size_t acc_bytes = static_cast<size_t>(rows) * c.d * sizeof(float);
+    cudaError_t e = cudaMemsetAsync(acc, 0, acc_bytes, st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(dq accumulator)");
+    bwd_rowdot<__nv_bfloat16, 128><<<rd_blocks, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), Drow,
+        c.B, c.S, c.Hq);
+    lca_status r = launched("bwd_rowdot");
+    if (r != LCA_OK) return r;
+    const int64_t tokens = static_cast<int64_t>(c.B) * c.S;
+    CUtensorMap mq, mk, mv, mdo;
+    if ((r = make_map(&mq, q, tokens, c.Hq)) != LCA_OK) return r;
+    if ((r = make_map(&mk, k, tokens, c.Hkv)) != LCA_OK) return r;
+    if ((r = make_map(&mv, v, tokens, c.Hkv)) != LCA_OK) return r;
+    if ((r = make_map(&mdo, dout, tokens, c.Hq)) != LCA_OK) return r;
+    if ((r = ensure_smem(attn_bwd_bf16_sm100, bwd::kSmemBytes, 3)) != LCA_OK) return r;
+    bwd::Args a;
+    a.B = c.B;
+    a.Hq = c.Hq;
+    a.Hkv = c.Hkv;
+    a.S = c.S;
+    a.scale = c.scale;
+    a.scale_log2 = c.scale * 1.4426950408889634f;
+    a.budget = budget;
+    a.lse = lse;
+    a.Drow = Drow;
+    a.dq_acc = acc;
+    a.dk = static_cast<__nv_bfloat16*>(dk);
+    a.dv = static_cast<__nv_bfloat16*>(dv);
+    a.sched = s;
+    attn_bwd_bf16_sm100<<<grid, bwd::kThreads, bwd::kSmemBytes, st>>>(mq, mk, mv, mdo, a);
+    if ((r = launched("attn_bwd_bf16_sm100")) != LCA_OK) return r;
+    const int64_t n8 = rows * c.d / 8;
+    dq_finalize<<<static_cast<unsigned>(std::min<int64_t>((n8 + 255) / 256, 148 * 16)), 256, 0,
+                  st>>>(acc, static_cast<__nv_bfloat16*>(dq), n8, c.scale);
+    return launched("dq_finalize");
+  }
+  // fp32
+  cudaError_t e = cudaMemsetAsync(dq, 0, static_cast<size_t>(rows) * c.d * sizeof(float), st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(dq)");
+  if (c.d == 64)
+    bwd_rowdot<float, 64><<<rd_blocks, 256, 0, st>>>(static_cast<const float*>(out),
+                                                       static_cast<const float*>(dout), Drow,
+                                                       c.B, c.S, c.Hq);
+  else
+    bwd_rowdot<float, 128><<<rd_blocks, 256, 0, st>>>(static_cast<const float*>(out),
+                                                        static_cast<const float*>(dout), Drow,
+                                                        c.B, c.S, c.Hq);
+  lca_status r = launched("bwd_rowdot");
+  if (r != LCA_OK) return r;
+  f32::Args a{};
+  a.q = static_cast<const float*>(q);
+  a.k = static_cast<const float*>(k);
+  a.v = static_cast<const float*>(v);
+  a.out = static_cast<const float*>(out);
+  a.lse = lse;
+  a.dout = static_cast<const float*>(dout);
+  a.D = Drow;
+  a.dq = static_cast<float*>(dq);
+  a.dk = static_cast<float*>(dk);
+  a.dv = static_cast<float*>(dv);
+  a.B = c.B;
+  a.Hq = c.Hq;
+  a.Hkv = c.Hkv;
+  a.S = c.S;
+  a.scale = c.scale;
+  a.sched = s;
+  if (c.d == 64) {
+    if ((r = ensure_smem(f32::attn_bwd_f32<64>, f32::bwd_smem<64>(), 4)) != LCA_OK) return r;
+    f32::attn_bwd_f32<64><<<grid, f32::kThreads, f32::bwd_smem<64>(), st>>>(a);
+  } else {
+    if ((r = ensure_smem(f32::attn_bwd_f32<128>, f32::bwd_smem<128>(), 5)) != LCA_OK) return r;
+    f32::attn_bwd_f32<128><<<grid, f32::kThreads, f32::bwd_smem<128>(), st>>>(a);
+  }
+  return launched("attn_bwd_f32");
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* lca_status_string(lca_status s) {
+  switch (s) {
+    case LCA_OK: return "LCA_OK";
+    case LCA_ERR_INVALID_ARG: return "LCA_ERR_INVALID_ARG";
+    case LCA_ERR_UNSUPPORTED: return "LCA_ERR_UNSUPPORTED";
+    case LCA_ERR_CUDA: return "LCA_ERR_CUDA";
+    case LCA_ERR_TIMEOUT: return "LCA_ERR_TIMEOUT";
+    case LCA_ERR_WORKSPACE: return "LCA_ERR_WORKSPACE";
+  }
+  return "LCA_ERR_UNKNOWN";
+}
+
+const char* lca_last_error(void) { return t_last_error.c_str(); }
+
+int lca_version(void) { return (1 << 16) | 0; }
+
+lca_status lca_attn_fwd(const lca_shape* shape, const void* q, const void* k, const void* v,
+                        int causal, int64_t kv_chunk, const lca_opts* opts, void* out,
+                        float* lse, void* stream) {
+  Common c;
+  lca_status r = check_shape(shape, &c);
+  if (r != LCA_OK) return r;
+  if ((r = check_ptrs({q, k, v, out, lse})) != LCA_OK) return r;
+  AttnSched s;
+  if ((r = make_chunk_sched(c, causal, kv_chunk, opts, &s)) != LCA_OK) return r;
+  return run_fwd(c, s, q, k, v, out, lse, budget_of(opts), static_cast<cudaStream_t>(stream));
+}
+
+size_t lca_attn_bwd_workspace_size(const lca_shape* shape) {
+  Common c;
+  const std::string keep = t_last_error;
+  if (check_shape(shape, &c) != LCA_OK) return 0;
+  t_last_error = keep;
+  return ws_bytes_of(c);
+}
+
+lca_status lca_attn_bwd(const lca_shape* shape, const void* q, const void* k, const void* v,
+                        const void* out, const float* lse, const void* dout, int causal,
+                        void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
+                        void* stream) {
+  Common c;
+  lca_status r = check_shape(shape, &c);
+  if (r != LCA_OK) return r;
+  if ((r = check_ptrs({q, k, v, out, lse, dout, dq, dk, dv})) != LCA_OK) return r;
+  AttnSched s;
+  if ((r = make_chunk_sched(c, causal, 0, nullptr, &s)) != LCA_OK) return r;
+  return run_bwd(c, s, q, k, v, out, lse, dout, dq, dk, dv, workspace, ws_bytes, kDefaultBudget,
+                 static_cast<cudaStream_t>(stream));
+}
+
+lca_status lca_s2attn_fwd(const lca_shape* shape, const void* q, const void* k, const void* v,
+                          int causal, int64_t group, int64_t shift_heads, void* out, float* lse,
+                          void* stream) {
+  Common c;
+  lca_status r = check_shape(shape, &c);
+  if (r != LCA_OK) return r;
+  if ((r = check_ptrs({q, k, v, out, lse})) != LCA_OK) return r;
+  AttnSched s;
+  if ((r = make_s2_sched(c, causal, group, shift_heads, &s)) != LCA_OK) return r;
+  return run_fwd(c, s, q, k, v, out, lse, kDefaultBudget, static_cast<cudaStream_t>(stream));
+}
+
+lca_status lca_s2attn_bwd(const lca_shape* shape, const void* q, const void* k, const void* v,
+                          const void* out, const float* lse, const void* dout, int causal,
+                          int64_t group, int64_t shift_heads, void* dq, void* dk, void* dv,
+                          void* workspace, size_t ws_bytes, void* stream) {
+  Common c;
+  lca_status r = check_shape(shape, &c);
+  if (r != LCA_OK) return r;
+  if ((r = check_ptrs({q, k, v, out, lse, dout, dq, dk, dv})) != LCA_OK) return r;
+  AttnSched s;
+  if ((r = make_s2_sched(c, causal, group, shift_heads, &s)) != LCA_OK) return r;
+  return run_bwd(c, s, q, k, v, out, lse, dout, dq, dk, dv, workspace, ws_bytes, kDefaultBudget,
+                 static_cast<cudaStream_t>(stream));
+}
+
+lca_status lca_lse_merge(int64_t rows, int64_t d, const float* o_a, const float* lse_a,
+                         const float* o_b, const float* lse_b, float* o_out, float* lse_out,
+                         void* stream) {
+  if (rows <= 0 || d <= 0 || d > (1 << 20))
+    return fail(LCA_ERR_INVALID_ARG, "rows and d must be positive");
+  if (!o_a || !lse_a || !o_b || !lse_b || !o_out || !lse_out)
+    return fail(LCA_ERR_INVALID_ARG, "NULL pointer");
+  const int64_t warps_needed = rows;
+  const unsigned blocks =
+      static_cast<unsigned>(std::min<int64_t>((warps_needed * 32 + 255) / 256, 148 * 32));
+  lse_merge_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      rows, static_cast<int>(d), o_a, lse_a, o_b, lse_b, o_out, lse_out);
+  return launched("lse_merge_kernel");
+}
+
+lca_status lca_check(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int h[2] = {0, 0};
+  e = cudaMemcpyFromSymbol(h, g_err, sizeof h);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  if (h[0]) {
+    const int z[2] = {0, 0};
+    cudaMemcpyToSymbol(g_err, z, sizeof z);
+    return fail(LCA_ERR_TIMEOUT, "a kernel wait ran out (site %d)", h[1]);
+  }
+  return LCA_OK;
+}
+
+}  // extern "C"

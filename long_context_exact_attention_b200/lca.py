@@ -1,0 +1,211 @@
+"""Python binding of liblca (include/lca.h) over torch tensors.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library.  torch supplies device memory and the current stream.  There is no
+fallback: if liblca.so is missing or the tensors are not CUDA tensors the
+call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblca.so")
+
+LCA_BF16, LCA_FP32 = 0, 1
+ORDERS = {"inorder": 0, "ring": 1, "custom": 2}
+STATUS = {0: "LCA_OK", 1: "LCA_ERR_INVALID_ARG", 2: "LCA_ERR_UNSUPPORTED",
+          3: "LCA_ERR_CUDA", 4: "LCA_ERR_TIMEOUT", 5: "LCA_ERR_WORKSPACE"}
+SYMBOLS = ["lca_attn_fwd", "lca_attn_bwd_workspace_size", "lca_attn_bwd",
+           "lca_s2attn_fwd", "lca_s2attn_bwd", "lca_lse_merge", "lca_check",
+           "lca_status_string", "lca_last_error", "lca_version"]
+
+
+class LcaError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"{STATUS.get(status, status)}: {detail}")
+        self.status = status
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int64), ("Hq", ctypes.c_int64), ("Hkv", ctypes.c_int64),
+                ("S", ctypes.c_int64), ("d", ctypes.c_int64), ("dtype", ctypes.c_int32),
+                ("scale", ctypes.c_float)]
+
+
+class Opts(ctypes.Structure):
+    _fields_ = [("order", ctypes.c_int32), ("chunk_perm", ctypes.POINTER(ctypes.c_int32)),
+                ("q_block", ctypes.c_int64), ("timeout_cycles", ctypes.c_uint64)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded liblca.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing; build it with "
+                "`python -m long_context_exact_attention_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I64, I32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        SP = ctypes.POINTER(Shape)
+        L.lca_attn_fwd.argtypes = [SP, P, P, P, I32, I64, ctypes.POINTER(Opts), P, P, P]
+        L.lca_attn_bwd_workspace_size.argtypes = [SP]
+        L.lca_attn_bwd_workspace_size.restype = ctypes.c_size_t
+        L.lca_attn_bwd.argtypes = [SP, P, P, P, P, P, P, I32, P, P, P, P, ctypes.c_size_t, P]
+        L.lca_s2attn_fwd.argtypes = [SP, P, P, P, I32, I64, I64, P, P, P]
+        L.lca_s2attn_bwd.argtypes = [SP, P, P, P, P, P, P, I32, I64, I64, P, P, P, P,
+                                     ctypes.c_size_t, P]
+        L.lca_lse_merge.argtypes = [I64, I64, P, P, P, P, P, P, P]
+        L.lca_check.argtypes = [P]
+        L.lca_status_string.restype = ctypes.c_char_p
+        L.lca_last_error.restype = ctypes.c_char_p
+        for fn in ("lca_attn_fwd", "lca_attn_bwd", "lca_s2attn_fwd", "lca_s2attn_bwd",
+                   "lca_lse_merge", "lca_check"):
+            getattr(L, fn).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _raise(st: int):
+    if st != 0:
+        raise LcaError(st, lib().lca_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _shape(q: torch.Tensor, k: torch.Tensor, scale) -> Shape:
+    if not (q.is_cuda and k.is_cuda):
+        raise ValueError("lca needs CUDA tensors")
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q is [B,S,Hq,d], k/v are [B,S,Hkv,d]")
+    B, S, Hq, d = q.shape
+    if k.shape[0] != B or k.shape[1] != S or k.shape[3] != d:
+        raise ValueError("k/v shape does not match q")
+    if q.dtype == torch.bfloat16:
+        dt = LCA_BF16
+    elif q.dtype == torch.float32:
+        dt = LCA_FP32
+    else:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    return Shape(B, Hq, k.shape[2], S, d, dt, float(scale or 0.0))
+
+
+def _check_tensors(dtype, *ts):
+    for t in ts:
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous CUDA tensors")
+        if t.dtype != dtype:
+            raise ValueError(f"dtype mismatch: {t.dtype} vs {dtype}")
+
+
+def attn_fwd(q, k, v, causal: bool = True, kv_chunk: int = 0, order: str = "inorder",
+             chunk_perm: Optional[Sequence[int]] = None, q_block: int = 0, scale=None,
+             out=None, lse=None, stream=None, timeout_cycles: int = 0):
+    """Exact attention forward (lca_attn_fwd).  Returns (out, lse)."""
+    sh = _shape(q, k, scale)
+    _check_tensors(q.dtype, q, k, v)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((q.shape[0], q.shape[2], q.shape[1]), device=q.device,
+                          dtype=torch.float32)
+    opts = Opts(ORDERS[order], None, int(q_block), int(timeout_cycles))
+    keep = None
+    if chunk_perm is not None:
+        keep = (ctypes.c_int32 * len(chunk_perm))(*[int(x) for x in chunk_perm])
+        opts.chunk_perm = ctypes.cast(keep, ctypes.POINTER(ctypes.c_int32))
+    _raise(lib().lca_attn_fwd(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), int(causal),
+                              int(kv_chunk), ctypes.byref(opts), _ptr(out), _ptr(lse),
+                              _stream(stream)))
+    return out, lse
+
+
+def workspace_size(q, k) -> int:
+    sh = _shape(q, k, None)
+    return int(lib().lca_attn_bwd_workspace_size(ctypes.byref(sh)))
+
+
+def _alloc_grads(q, k, v, dq, dk, dv, workspace):
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = torch.empty(workspace_size(q, k), device=q.device, dtype=torch.uint8)
+    return dq, dk, dv, workspace
+
+
+def attn_bwd(q, k, v, out, lse, dout, causal: bool = True, scale=None, dq=None, dk=None,
+             dv=None, workspace=None, stream=None):
+    """Gradients of sum(dout * out) (lca_attn_bwd).  Returns (dq, dk, dv)."""
+    sh = _shape(q, k, scale)
+    _check_tensors(q.dtype, q, k, v, out, dout)
+    dq, dk, dv, workspace = _alloc_grads(q, k, v, dq, dk, dv, workspace)
+    _raise(lib().lca_attn_bwd(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                              _ptr(dout), int(causal), _ptr(dq), _ptr(dk), _ptr(dv),
+                              _ptr(workspace), workspace.numel() * workspace.element_size(),
+                              _stream(stream)))
+    return dq, dk, dv
+
+
+def s2attn_fwd(q, k, v, group: int, shift_heads: int, causal: bool = True, scale=None,
+               out=None, lse=None, stream=None):
+    """LongLoRA S2-Attn forward (lca_s2attn_fwd).  Returns (out, lse)."""
+    sh = _shape(q, k, scale)
+    _check_tensors(q.dtype, q, k, v)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((q.shape[0], q.shape[2], q.shape[1]), device=q.device,
+                          dtype=torch.float32)
+    _raise(lib().lca_s2attn_fwd(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), int(causal),
+                                int(group), int(shift_heads), _ptr(out), _ptr(lse),
+                                _stream(stream)))
+    return out, lse
+
+
+def s2attn_bwd(q, k, v, out, lse, dout, group: int, shift_heads: int, causal: bool = True,
+               scale=None, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """LongLoRA S2-Attn backward (lca_s2attn_bwd).  Returns (dq, dk, dv)."""
+    sh = _shape(q, k, scale)
+    _check_tensors(q.dtype, q, k, v, out, dout)
+    dq, dk, dv, workspace = _alloc_grads(q, k, v, dq, dk, dv, workspace)
+    _raise(lib().lca_s2attn_bwd(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                _ptr(lse), _ptr(dout), int(causal), int(group),
+                                int(shift_heads), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(stream)))
+    return dq, dk, dv
+
+
+def lse_merge(o_a, lse_a, o_b, lse_b, o_out=None, lse_out=None, stream=None):
+    """Merge two float32 partial results (lca_lse_merge).  o_*: [rows, d],
+    lse_*: [rows].  Returns (o, lse)."""
+    for t in (o_a, lse_a, o_b, lse_b):
+        if not t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous():
+            raise ValueError("lse_merge takes contiguous float32 CUDA tensors")
+    rows, d = o_a.shape[0], o_a.numel() // max(o_a.shape[0], 1)
+    o_out = torch.empty_like(o_a) if o_out is None else o_out
+    lse_out = torch.empty_like(lse_a) if lse_out is None else lse_out
+    _raise(lib().lca_lse_merge(rows, d, _ptr(o_a), _ptr(lse_a), _ptr(o_b), _ptr(lse_b),
+                               _ptr(o_out), _ptr(lse_out), _stream(stream)))
+    return o_out, lse_out
+
+
+def check(stream=None):
+    """Synchronise and raise LcaError if a kernel wait ran out."""
+    _raise(lib().lca_check(_stream(stream)))

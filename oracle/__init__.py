@@ -30,12 +30,13 @@ here is "parity unpinned".
 """
 
 from .attention import (attention_forward, attention_rows, attention_backward,
-                        chunked_attention_forward)
+                        attention_backward_rows, chunked_attention_forward)
 from .s2attn import s2attn_forward, s2attn_backward, s2_token_of_position
 from .merge import lse_merge
 
 __all__ = [
     "attention_forward", "attention_rows", "attention_backward",
+    "attention_backward_rows",
     "chunked_attention_forward", "s2attn_forward", "s2attn_backward",
     "s2_token_of_position", "lse_merge",
 ]

@@ -203,3 +203,40 @@ def chunked_attention_forward(q, k, v, causal: bool, chunk: int, order,
             out[b, :, h] = o_run
             lse[b, h] = l_run
     return out, lse
+
+
+def attention_backward_rows(q, k, v, dout, causal: bool, b: int, g: int, rows,
+                            scale=None):
+    """Backward restricted to query ``rows`` of every query head that reads
+    key/value head ``g`` (batch ``b``).  Each row is the full-row definition.
+
+    Returns (dq [R, rep, d] for those rows, dk_part [S, d], dv_part [S, d])
+    where the *_part arrays hold only the rows' contributions
+    (dK_j += scale * sum_{i in rows} dS_ij q_i, dV_j += sum_{i in rows} P_ij dO_i).
+    Under a causal mask, a key j receives contributions only from rows
+    i >= j, so when ``rows`` is the tail [r0, S) the parts equal the full dK_j
+    and dV_j for every j >= r0."""
+    import torch  # noqa: F401  (tensor inputs are converted by _f64)
+    rows = np.asarray(rows, dtype=np.int64)
+    Hq, Hkv = q.shape[2], k.shape[2]
+    rep = Hq // Hkv
+    K = _f64(k[b, :, g])
+    V = _f64(v[b, :, g])
+    S, d = K.shape
+    sc = _scale(d, scale)
+    dq = np.zeros((len(rows), rep, d))
+    dk = np.zeros((S, d))
+    dv = np.zeros((S, d))
+    for r in range(rep):
+        h = g * rep + r
+        Q = _f64(q[b, :, h])[rows]
+        dO = _f64(dout[b, :, h])[rows]
+        s = _row_block((Q @ K.T) * sc, S, causal, rows)
+        p, _ = _softmax_rows(s)
+        dP = dO @ V.T
+        D = np.sum(p * dP, axis=1)
+        dS = p * (dP - D[:, None])
+        dq[:, r] = sc * (dS @ K)
+        dk += sc * (dS.T @ Q)
+        dv += p.T @ dO
+    return dq, dk, dv

@@ -359,3 +359,23 @@ def test_pins_catch_planted_mistakes(monkeypatch, mutant):
             return orig(x, heads, amount if calls["n"] % 4 else -amount)
         monkeypatch.setattr(S2, "_roll_heads", bad)
     assert not _pins_pass()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_rows_matches_full(causal):
+    rng = np.random.default_rng(31)
+    S, d, Hq, Hkv = 20, 4, 4, 2
+    q, k, v, do = rand(1, S, Hq, d, rng=rng), rand(1, S, Hkv, d, rng=rng), \
+        rand(1, S, Hkv, d, rng=rng), rand(1, S, Hq, d, rng=rng)
+    dq, dk, dv = oracle.attention_backward(q, k, v, do, causal)
+    rows = [3, 11, 19]
+    dqr, _, _ = oracle.attention_backward_rows(q, k, v, do, causal, 0, 1, rows)
+    np.testing.assert_allclose(dqr, dq[0, rows, 2:4], atol=1e-13)
+    # all rows: the parts are the full gradients
+    dqa, dka, dva = oracle.attention_backward_rows(q, k, v, do, causal, 0, 1, range(S))
+    np.testing.assert_allclose(dka, dk[0, :, 1], atol=1e-13)
+    np.testing.assert_allclose(dva, dv[0, :, 1], atol=1e-13)
+    if causal:  # tail rows give exact dK/dV for keys in the tail
+        _, dkt, dvt = oracle.attention_backward_rows(q, k, v, do, True, 0, 0, range(12, S))
+        np.testing.assert_allclose(dkt[12:], dk[0, 12:, 0], atol=1e-13)
+        np.testing.assert_allclose(dvt[12:], dv[0, 12:, 0], atol=1e-13)
