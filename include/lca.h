@@ -142,6 +142,36 @@ LCA_API lca_status lca_attn_bwd(const lca_shape* shape, const void* q, const voi
                         void* stream);
 
 /* ---------------------------------------------------------------------------
+ * lca_attn_bwd_noalloc -- lca_attn_bwd for callers that cannot allocate
+ * device memory.  No counterpart in the pages: it exists for callers such
+ * as a plugin inside a host framework that owns every device allocation and
+ * hands the plugin none, or code on a latency-critical path that cannot take
+ * cudaMalloc's cost and implicit synchronisation.  The caller still passes
+ * every input and output; the scratch that lca_attn_bwd takes as
+ * `workspace` (float32 D rows and, for bf16, a float32 dq accumulator:
+ * lca_attn_bwd_workspace_size bytes) comes instead from a fixed array of
+ * LCA_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads
+ * the library holds until the process exits.  The function allocates and
+ * frees nothing.
+ *   Set-up: the first call on each device looks up the array's device
+ *   address (cudaGetSymbolAddress) with that device current; make that first
+ *   call before any stream capture.
+ *   Sharing: every call on a device uses the same array and leaves its last
+ *   contents there (the parts that must start at zero are cleared by each
+ *   call).  Calls whose work overlaps on the GPU -- on different streams, or
+ *   from different host threads without ordering -- race on the array and
+ *   give wrong gradients; issue them in order, e.g. on one stream.
+ *   Errors: as lca_attn_bwd; LCA_ERR_WORKSPACE when the shape needs more
+ *   scratch than LCA_NOALLOC_SCRATCH_BYTES (use lca_attn_bwd then).
+ * ------------------------------------------------------------------------- */
+#define LCA_NOALLOC_SCRATCH_BYTES (64u << 20)
+LCA_API lca_status lca_attn_bwd_noalloc(const lca_shape* shape, const void* q,
+                                        const void* k, const void* v,
+                                        const void* out, const float* lse,
+                                        const void* dout, int causal, void* dq,
+                                        void* dk, void* dv, void* stream);
+
+/* ---------------------------------------------------------------------------
  * lca_s2attn_fwd -- LongLoRA shifted sparse attention (S2-Attn), forward.
  *   Positions are split into S/group groups of `group`; attention runs
  *   inside each group (causal by position within the group when `causal`).

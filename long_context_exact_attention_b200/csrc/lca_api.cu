@@ -475,3 +475,59 @@ lca_status lca_check(void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- no-alloc backward
+//
+// lca_attn_bwd_noalloc: the backward pass for callers that cannot allocate
+// device memory.  Its scratch (the float32 D rows and, for bf16, the float32
+// dq accumulator) lives in the fixed array below instead of a caller buffer.
+// The array is part of this library's device image, so every GPU that loads
+// the library holds LCA_NOALLOC_SCRATCH_BYTES of it until the process exits.
+// Host code may not use the array's name as a device address (on the host it
+// is only a stand-in); its device address is looked up once per device with
+// cudaGetSymbolAddress while that device is current.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[LCA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+lca_status noalloc_scratch_address(void** out) {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(LCA_ERR_UNSUPPORTED, "device ordinal %d >= 64", dev);
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(built-in scratch)");
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return LCA_OK;
+}
+
+}  // namespace
+
+extern "C" lca_status lca_attn_bwd_noalloc(const lca_shape* shape, const void* q, const void* k,
+                                           const void* v, const void* out, const float* lse,
+                                           const void* dout, int causal, void* dq, void* dk,
+                                           void* dv, void* stream) {
+  Common c;
+  lca_status r = check_shape(shape, &c);
+  if (r != LCA_OK) return r;
+  if ((r = check_ptrs({q, k, v, out, lse, dout, dq, dk, dv})) != LCA_OK) return r;
+  AttnSched s;
+  if ((r = make_chunk_sched(c, causal, 0, nullptr, &s)) != LCA_OK) return r;
+  const size_t need = ws_bytes_of(c);
+  if (need > LCA_NOALLOC_SCRATCH_BYTES)
+    return fail(LCA_ERR_WORKSPACE,
+                "this shape needs %zu bytes of scratch; the built-in scratch of "
+                "lca_attn_bwd_noalloc holds %zu (use lca_attn_bwd with a workspace)",
+                need, static_cast<size_t>(LCA_NOALLOC_SCRATCH_BYTES));
+  void* ws = nullptr;
+  if ((r = noalloc_scratch_address(&ws)) != LCA_OK) return r;
+  return run_bwd(c, s, q, k, v, out, lse, dout, dq, dk, dv, ws, LCA_NOALLOC_SCRATCH_BYTES,
+                 kDefaultBudget, static_cast<cudaStream_t>(stream));
+}

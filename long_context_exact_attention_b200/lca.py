@@ -21,6 +21,7 @@ ORDERS = {"inorder": 0, "ring": 1, "custom": 2}
 STATUS = {0: "LCA_OK", 1: "LCA_ERR_INVALID_ARG", 2: "LCA_ERR_UNSUPPORTED",
           3: "LCA_ERR_CUDA", 4: "LCA_ERR_TIMEOUT", 5: "LCA_ERR_WORKSPACE"}
 SYMBOLS = ["lca_attn_fwd", "lca_attn_bwd_workspace_size", "lca_attn_bwd",
+           "lca_attn_bwd_noalloc",
            "lca_s2attn_fwd", "lca_s2attn_bwd", "lca_lse_merge", "lca_check",
            "lca_status_string", "lca_last_error", "lca_version"]
 
@@ -60,6 +61,7 @@ def lib() -> ctypes.CDLL:
         L.lca_attn_bwd_workspace_size.argtypes = [SP]
         L.lca_attn_bwd_workspace_size.restype = ctypes.c_size_t
         L.lca_attn_bwd.argtypes = [SP, P, P, P, P, P, P, I32, P, P, P, P, ctypes.c_size_t, P]
+        L.lca_attn_bwd_noalloc.argtypes = [SP, P, P, P, P, P, P, I32, P, P, P, P]
         L.lca_s2attn_fwd.argtypes = [SP, P, P, P, I32, I64, I64, P, P, P]
         L.lca_s2attn_bwd.argtypes = [SP, P, P, P, P, P, P, I32, I64, I64, P, P, P, P,
                                      ctypes.c_size_t, P]
@@ -67,7 +69,8 @@ def lib() -> ctypes.CDLL:
         L.lca_check.argtypes = [P]
         L.lca_status_string.restype = ctypes.c_char_p
         L.lca_last_error.restype = ctypes.c_char_p
-        for fn in ("lca_attn_fwd", "lca_attn_bwd", "lca_s2attn_fwd", "lca_s2attn_bwd",
+        for fn in ("lca_attn_fwd", "lca_attn_bwd", "lca_attn_bwd_noalloc", "lca_s2attn_fwd",
+                   "lca_s2attn_bwd",
                    "lca_lse_merge", "lca_check"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
@@ -160,6 +163,23 @@ def attn_bwd(q, k, v, out, lse, dout, causal: bool = True, scale=None, dq=None, 
                               _ptr(dout), int(causal), _ptr(dq), _ptr(dk), _ptr(dv),
                               _ptr(workspace), workspace.numel() * workspace.element_size(),
                               _stream(stream)))
+    return dq, dk, dv
+
+
+def attn_bwd_noalloc(q, k, v, out, lse, dout, causal: bool = True, scale=None, dq=None,
+                     dk=None, dv=None, stream=None):
+    """lca_attn_bwd_noalloc: the backward pass with the library's built-in
+    scratch instead of a workspace, for callers that cannot allocate device
+    memory.  Calls that overlap on the GPU share that scratch and race.
+    Returns (dq, dk, dv)."""
+    sh = _shape(q, k, scale)
+    _check_tensors(q.dtype, q, k, v, out, dout)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _raise(lib().lca_attn_bwd_noalloc(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                      _ptr(lse), _ptr(dout), int(causal), _ptr(dq), _ptr(dk),
+                                      _ptr(dv), _stream(stream)))
     return dq, dk, dv
 
 
