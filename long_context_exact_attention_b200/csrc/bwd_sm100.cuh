@@ -13,15 +13,21 @@
 // query heads of its grouped-query group and over the query tiles that can
 // see the key tile, so dK/dV of a key tile finish inside one CTA.
 // Roles (10 warps):
-//   warp 0      TMA producer: K, V once; Q, dO tiles plus lse/D rows per step
+//   warp 0      TMA producer: K, V once; Q, dO tiles plus lse/D rows per
+//               step through a 2-stage ring
 //   warp 1      TMEM owner; lane 0 issues the five MMAs of every step
-//   warps 2..5  P/dS warpgroup: one key row per thread
+//   warps 2..5  P/dS warpgroup: one key row per thread.  P^T (bf16) is
+//               written back into the S^T columns it was computed from and
+//               feeds the dV product straight from tensor memory; dS^T goes
+//               to shared memory (it is the A operand of both dK and dQ)
 //   warps 6..9  dQ warpgroup: one query row per thread, drains dQ from TMEM
 //               and adds it to global memory; writes dV at the end
-// TMEM: S^T [0,128) | dP^T and then dQ [128,256) | dV [256,384) | dK [384,512)
-// Shared memory (128-byte swizzle): K | V | Q | dO | P^T | dS^T | lse | D.
+// TMEM: S^T then P^T [0,128) | dP^T then dQ [128,256) | dV | dK
+// Per step the tensor pipe runs S^T, dP^T, dV, dK, dQ; dV overlaps the dS
+// math, the next step's S^T overlaps the dQ drain.
 #pragma once
 
+#include "exp2_poly.cuh"
 #include "ptx.cuh"
 #include "sched.cuh"
 
@@ -37,25 +43,31 @@ constexpr int kThreads = 320;
 
 constexpr uint32_t kOffK = 0;
 constexpr uint32_t kOffV = kOffK + kTileB;
-constexpr uint32_t kOffQ = kOffV + kTileB;
-constexpr uint32_t kOffO = kOffQ + kTileB;    // dO
-constexpr uint32_t kOffP = kOffO + kTileB;    // P^T
-constexpr uint32_t kOffS = kOffP + kTileB;    // dS^T
-constexpr uint32_t kOffL = kOffS + kTileB;    // lse[128]
-constexpr uint32_t kOffD = kOffL + 512;       // D[128]
-constexpr uint32_t kOffBar = kOffD + 512;
-constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
+constexpr uint32_t kOffQ = kOffV + kTileB;        // 2 stages
+constexpr uint32_t kOffO = kOffQ + 2 * kTileB;    // dO, 2 stages
+constexpr uint32_t kOffS = kOffO + 2 * kTileB;    // dS^T
+constexpr uint32_t kOffL = kOffS + kTileB;        // lse[2][128]
+constexpr uint32_t kOffD = kOffL + 1024;          // D[2][128]
+constexpr uint32_t kOffBar = kOffD + 1024;
+constexpr uint32_t kUsed = kOffBar + 256;
+// Shared memory requested: what is used plus the slack that is left under
+// the 227 KB per-CTA limit; the kernel refuses to run if aligning its base
+// to 1024 bytes would need more than that slack.
+constexpr uint32_t kSmemBytes = 232448;
+constexpr uint32_t kSlack = kSmemBytes - kUsed;
 
 enum {
   B_KV = 0,
-  B_QFULL,
-  B_QEMPTY,
-  B_SFULL,
-  B_SFREE,   // 128 arrivals
-  B_PFULL,   // 128 arrivals
-  B_PFREE,
+  B_QFULL,        // +stage
+  B_QEMPTY = 3,   // +stage
+  B_SFULL = 5,
+  B_DPFULL,
+  B_PREADY,       // 128 arrivals
+  B_PTFREE,
+  B_DSREADY,      // 128 arrivals
+  B_DSFREE,
   B_DQFULL,
-  B_DQFREE,  // 128 arrivals
+  B_DQFREE,       // 128 arrivals
   B_DONE,
   B_DRAIN,
   NUM_BARS
@@ -64,6 +76,11 @@ enum {
 constexpr uint32_t kIdescKK = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T
 constexpr uint32_t kIdescKM = idesc_bf16_f32(128, 128, false, true);   // dV, dK
 constexpr uint32_t kIdescMM = idesc_bf16_f32(128, 128, true, true);    // dQ
+
+// Pairs q (of the 64 per row and tile) with bit (q % 8) set would take the
+// FMA-pipe polynomial exp2 instead of ex2.approx.  Measured on B200 the
+// mixes tried (3/8, 4/8) were slower than none, so none is used.
+constexpr uint32_t kPolyPairs = 0u;
 
 struct Args {
   int B, Hq, Hkv, S;
@@ -99,9 +116,17 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
+  if (base - raw > kSlack) {
+    // Cannot place the 1024-aligned layout inside the allocation: refuse.
+    if (threadIdx.x == 0) {
+      atomicOr(&g_err[0], 2);
+      atomicCAS(&g_err[1], 0, 100);
+    }
+    return;
+  }
   uint8_t* gbase = smem_raw + (base - raw);
   const uint32_t sK = base + kOffK, sV = base + kOffV, sQ = base + kOffQ, sO = base + kOffO;
-  const uint32_t sP = base + kOffP, sS = base + kOffS, sL = base + kOffL, sD = base + kOffD;
+  const uint32_t sS = base + kOffS, sL = base + kOffL, sD = base + kOffD;
   const float* lse_s = reinterpret_cast<const float*>(gbase + kOffL);
   const float* d_s = reinterpret_cast<const float*>(gbase + kOffD);
   const uint32_t bars = base + kOffBar;
@@ -129,7 +154,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NUM_BARS; ++i) {
-      const uint32_t cnt = (i == B_SFREE || i == B_PFULL || i == B_DQFREE) ? 128u : 1u;
+      const uint32_t cnt = (i == B_PREADY || i == B_DSREADY || i == B_DQFREE) ? 128u : 1u;
       mbar_init(bar(i), cnt);
     }
     *abort_flag = 0;
@@ -159,26 +184,29 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       tma_load_3d(sV, &tmV, bar(B_KV), 0, g, row0 + ktok0);
       tma_load_3d(sV + kHalf, &tmV, bar(B_KV), 64, g, row0 + ktok0);
       bool ok = true;
-      int issued = 0;
+      int issued0 = 0, issued1 = 0;
       for (int i = 0; i < nsteps && ok; ++i) {
+        const int st = i & 1;
         const int h = g * rep + i / nq;
         const int qt = qw.t + i % nq;
         const int qtok0 = token_tile(sc, qt, shifted) * kTile;
-        if (i >= 1) ok = wait_bar(bar(B_QEMPTY), (i - 1) & 1, wc, 111);
+        if (i >= 2) ok = wait_bar(bar(B_QEMPTY + st), ((i - 2) >> 1) & 1, wc, 111);
         if (!ok) break;
-        mbar_expect_tx(bar(B_QFULL), 2 * kTileB + 1024);
-        tma_load_3d(sQ, &tmQ, bar(B_QFULL), 0, h, row0 + qtok0);
-        tma_load_3d(sQ + kHalf, &tmQ, bar(B_QFULL), 64, h, row0 + qtok0);
-        tma_load_3d(sO, &tmDO, bar(B_QFULL), 0, h, row0 + qtok0);
-        tma_load_3d(sO + kHalf, &tmDO, bar(B_QFULL), 64, h, row0 + qtok0);
+        const uint32_t fb = bar(B_QFULL + st);
+        mbar_expect_tx(fb, 2 * kTileB + 1024);
+        tma_load_3d(sQ + st * kTileB, &tmQ, fb, 0, h, row0 + qtok0);
+        tma_load_3d(sQ + st * kTileB + kHalf, &tmQ, fb, 64, h, row0 + qtok0);
+        tma_load_3d(sO + st * kTileB, &tmDO, fb, 0, h, row0 + qtok0);
+        tma_load_3d(sO + st * kTileB + kHalf, &tmDO, fb, 64, h, row0 + qtok0);
         const size_t ro = (static_cast<size_t>(b) * a.Hq + h) * a.S + qtok0;
-        bulk_load(sL, a.lse + ro, 512, bar(B_QFULL));
-        bulk_load(sD, a.Drow + ro, 512, bar(B_QFULL));
-        ++issued;
+        bulk_load(sL + st * 512, a.lse + ro, 512, fb);
+        bulk_load(sD + st * 512, a.Drow + ro, 512, fb);
+        if (st) ++issued1; else ++issued0;
       }
       if (!ok) {
         drain_bar(bar(B_KV), 0, a.budget);
-        if (issued) drain_bar(bar(B_QFULL), (issued - 1) & 1, a.budget);
+        if (issued0) drain_bar(bar(B_QFULL), (issued0 - 1) & 1, a.budget);
+        if (issued1) drain_bar(bar(B_QFULL + 1), (issued1 - 1) & 1, a.budget);
       }
     }
   } else if (warp == 1) {
@@ -187,47 +215,56 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       const uint32_t tSt = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 384;
       bool ok = wait_bar(bar(B_KV), 0, wc, 211);
       for (int i = 0; i < nsteps && ok; ++i) {
-        ok = wait_bar(bar(B_QFULL), i & 1, wc, 212);
-        if (ok && i >= 1) ok = wait_bar(bar(B_SFREE), (i - 1) & 1, wc, 213);
-        if (ok && i >= 1) ok = wait_bar(bar(B_DQFREE), (i - 1) & 1, wc, 214);
+        const int st = i & 1;
+        const uint32_t q_s = sQ + st * kTileB, o_s = sO + st * kTileB;
+        ok = wait_bar(bar(B_QFULL + st), (i >> 1) & 1, wc, 212);
+        if (ok && i >= 1) ok = wait_bar(bar(B_PTFREE), (i - 1) & 1, wc, 213);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t off = (k >> 2) * kHalf + (k & 3) * 32;
-          mma_bf16_ss(tSt, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024),
-                      kIdescKK, k > 0);
-        }
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint32_t off = (k >> 2) * kHalf + (k & 3) * 32;
-          mma_bf16_ss(tdP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sO + off, 16, 1024),
+          mma_bf16_ss(tSt, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(q_s + off, 16, 1024),
                       kIdescKK, k > 0);
         }
         tc_commit(bar(B_SFULL));
-        ok = wait_bar(bar(B_PFULL), i & 1, wc, 215);
+        if (i >= 1) ok = wait_bar(bar(B_DQFREE), (i - 1) & 1, wc, 214);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const uint32_t offa = (k >> 2) * kHalf + (k & 3) * 32;
-          mma_bf16_ss(tdV, sdesc_sw128(sP + offa, 16, 1024),
-                      sdesc_sw128(sO + k * 2048, kHalf, 1024), kIdescKM, (i > 0 || k > 0));
+          const uint32_t off = (k >> 2) * kHalf + (k & 3) * 32;
+          mma_bf16_ss(tdP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(o_s + off, 16, 1024),
+                      kIdescKK, k > 0);
         }
+        tc_commit(bar(B_DPFULL));
+        ok = wait_bar(bar(B_PREADY), i & 1, wc, 215);
+        if (!ok) break;
+        tc_fence_after();
+        // dV += P^T dO, P^T read from tensor memory (8 columns per 16 queries)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          mma_bf16_ts(tdV, tSt + k * 8, sdesc_sw128(o_s + k * 2048, kHalf, 1024), kIdescKM,
+                      (i > 0 || k > 0));
+        }
+        tc_commit(bar(B_PTFREE));
+        ok = wait_bar(bar(B_DSREADY), i & 1, wc, 216);
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t offa = (k >> 2) * kHalf + (k & 3) * 32;
           mma_bf16_ss(tdK, sdesc_sw128(sS + offa, 16, 1024),
-                      sdesc_sw128(sQ + k * 2048, kHalf, 1024), kIdescKM, (i > 0 || k > 0));
+                      sdesc_sw128(q_s + k * 2048, kHalf, 1024), kIdescKM, (i > 0 || k > 0));
         }
-        tc_commit(bar(B_QEMPTY));
+        tc_commit(bar(B_QEMPTY + st));
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           mma_bf16_ss(tdP, sdesc_sw128(sS + k * 2048, kHalf, 1024),
                       sdesc_sw128(sK + k * 2048, kHalf, 1024), kIdescMM, k > 0);
         }
         tc_commit(bar(B_DQFULL));
-        tc_commit(bar(B_PFREE));
+        tc_commit(bar(B_DSFREE));
       }
       tc_commit(bar(B_DONE));
       tc_commit(bar(B_DRAIN));
@@ -240,50 +277,83 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     const uint32_t lad = static_cast<uint32_t>(wq * 32) << 16;
     const float c = a.scale_log2;
     const float L2E = 1.4426950408889634f;
+    const uint64_t c2 = f2_pack(c, c);
     bool ok = true;
     for (int i = 0; i < nsteps && ok; ++i) {
+      const int st = i & 1;
       const int qt = qw.t + i % nq;
+      const float* lse_r = lse_s + st * 128;
+      const float* d_r = d_s + st * 128;
       ok = wait_bar(bar(B_SFULL), i & 1, wc, 311);
-      if (ok) ok = wait_bar(bar(B_QFULL), i & 1, wc, 312);
-      if (ok && i >= 1) ok = wait_bar(bar(B_PFREE), (i - 1) & 1, wc, 313);
+      if (ok) ok = wait_bar(bar(B_QFULL + st), (i >> 1) & 1, wc, 312);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
       const bool diag = sc.causal && qt == kt;
-#pragma unroll 1
+      // ---- P^T = exp2(S^T c - lse log2e), written back over S^T as bf16
+      float p[128];
+#pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
-        float s[32], dp[32];
+        float s[32];
         tmem_ld32(tmem + lad + cc * 32, s);
-        tmem_ld32(tmem + lad + 128 + cc * 32, dp);
-        uint32_t pp[16], dd[16];
+        uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           const int q0 = cc * 32 + e;
-          float p0 = ex2_approx(fmaf(s[e], c, -lse_s[q0] * L2E));
-          float p1 = ex2_approx(fmaf(s[e + 1], c, -lse_s[q0 + 1] * L2E));
+          const uint64_t nl = f2_pack(-lse_r[q0] * L2E, -lse_r[q0 + 1] * L2E);
+          const uint64_t x = f2_fma(f2_pack(s[e], s[e + 1]), c2, nl);
+          float p0, p1;
+          if ((kPolyPairs >> ((q0 >> 1) & 7)) & 1u) {
+            f2_unpack(exp2_poly_x2(x), p0, p1);
+          } else {
+            f2_unpack(x, p0, p1);
+            p0 = ex2_approx(p0);
+            p1 = ex2_approx(p1);
+          }
           if (diag && r > q0) p0 = 0.f;
           if (diag && r > q0 + 1) p1 = 0.f;
-          const float d0 = p0 * (dp[e] - d_s[q0]);
-          const float d1 = p1 * (dp[e + 1] - d_s[q0 + 1]);
-          pp[e >> 1] = pack_bf16x2(p0, p1);
-          dd[e >> 1] = pack_bf16x2(d0, d1);
+          p[q0] = p0;
+          p[q0 + 1] = p1;
+          pk[e >> 1] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tmem + lad + cc * 16, pk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(B_PREADY));
+      // ---- dS^T = P^T o (dP^T - D) -> shared memory
+      ok = wait_bar(bar(B_DPFULL), i & 1, wc, 313);
+      if (ok && i >= 1) ok = wait_bar(bar(B_DSFREE), (i - 1) & 1, wc, 314);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        float dp[32];
+        tmem_ld32(tmem + lad + 128 + cc * 32, dp);
+        uint32_t dd[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int q0 = cc * 32 + e;
+          const uint64_t t = f2_sub(f2_pack(dp[e], dp[e + 1]), f2_pack(d_r[q0], d_r[q0 + 1]));
+          float t0, t1;
+          f2_unpack(t, t0, t1);
+          dd[e >> 1] = pack_bf16x2(p[q0] * t0, p[q0 + 1] * t1);
         }
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
           const int ch = cc * 4 + v;
           const int half = ch >> 3, cw = ch & 7;
           const uint32_t off = half * kHalf + r * 128 + ((cw ^ (r & 7)) << 4);
-          st_shared_v4(sP + off, pp[4 * v], pp[4 * v + 1], pp[4 * v + 2], pp[4 * v + 3]);
           st_shared_v4(sS + off, dd[4 * v], dd[4 * v + 1], dd[4 * v + 2], dd[4 * v + 3]);
         }
       }
-      tc_fence_before();
-      mbar_arrive(bar(B_SFREE));
       fence_async_smem();
-      mbar_arrive(bar(B_PFULL));
+      tc_fence_before();
+      mbar_arrive(bar(B_DSREADY));
     }
     // ---- dK = scale * acc -> bf16
-    if (ok) ok = wait_bar(bar(B_DONE), 0, wc, 314);
+    if (ok) ok = wait_bar(bar(B_DONE), 0, wc, 315);
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
       tc_fence_after();
@@ -317,13 +387,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       float dq[128];
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        float tmp[32];
-        tmem_ld32(tmem + lad + 128 + cc * 32, tmp);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) dq[cc * 32 + e] = tmp[e];
-      }
+      tmem_ld128(tmem + lad + 128, dq);
       tc_fence_before();
       mbar_arrive(bar(B_DQFREE));
       float4* dst = reinterpret_cast<float4*>(

@@ -24,12 +24,18 @@
 // keys 0-63, 64-127 for P), rows of 128 bytes.
 #pragma once
 
+#include "exp2_poly.cuh"
 #include "ptx.cuh"
 #include "sched.cuh"
 
 namespace lca {
 
 namespace fwd {
+
+// Pairs q (of the 64 per row and tile) with bit (q % 8) set would take the
+// FMA-pipe polynomial exp2 instead of ex2.approx.  Measured on B200 the
+// mixes tried (3/8, 4/8) were slower than none, so none is used.
+constexpr uint32_t kPolyPairs = 0u;
 
 constexpr int kTile = 128;
 constexpr int kD = 128;
@@ -135,7 +141,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       KvWalk w;
       w.init(&sc, qt);
       int t, j = 0;
-      int k_issued[2] = {0, 0}, v_issued[2] = {0, 0};
+      int k_issued0 = 0, k_issued1 = 0, v_issued0 = 0, v_issued1 = 0;
       bool ok = true;
       while (ok && w.next(t)) {
         const int st = j & 1;
@@ -145,22 +151,22 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         mbar_expect_tx(bar(B_KFULL + st), kTileB);
         tma_load_3d(sK + st * kTileB, &tmK, bar(B_KFULL + st), 0, g, tok);
         tma_load_3d(sK + st * kTileB + kHalf, &tmK, bar(B_KFULL + st), 64, g, tok);
-        ++k_issued[st];
+        if (st) ++k_issued1; else ++k_issued0;
         if (j >= 2) ok = wait_bar(bar(B_VEMPTY + st), ((j - 2) >> 1) & 1, wc, 102);
         if (!ok) break;
         mbar_expect_tx(bar(B_VFULL + st), kTileB);
         tma_load_3d(sV + st * kTileB, &tmV, bar(B_VFULL + st), 0, g, tok);
         tma_load_3d(sV + st * kTileB + kHalf, &tmV, bar(B_VFULL + st), 64, g, tok);
-        ++v_issued[st];
+        if (st) ++v_issued1; else ++v_issued0;
         ++j;
       }
       if (!ok) {
         // Unwind: let the copies already issued land before the CTA exits.
         drain_bar(bar(B_Q), 0, a.budget);
-        for (int st = 0; st < 2; ++st) {
-          if (k_issued[st]) drain_bar(bar(B_KFULL + st), (k_issued[st] - 1) & 1, a.budget);
-          if (v_issued[st]) drain_bar(bar(B_VFULL + st), (v_issued[st] - 1) & 1, a.budget);
-        }
+        if (k_issued0) drain_bar(bar(B_KFULL), (k_issued0 - 1) & 1, a.budget);
+        if (k_issued1) drain_bar(bar(B_KFULL + 1), (k_issued1 - 1) & 1, a.budget);
+        if (v_issued0) drain_bar(bar(B_VFULL), (v_issued0 - 1) & 1, a.budget);
+        if (v_issued1) drain_bar(bar(B_VFULL + 1), (v_issued1 - 1) & 1, a.budget);
       }
     }
   } else if (warp == 1) {
@@ -231,31 +237,67 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       float s[128];
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        float tmp[32];
-        tmem_ld32(tS + st * 128 + cc * 32, tmp);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[cc * 32 + i] = tmp[i];
-      }
+      tmem_ld128(tS + st * 128, s);
       tc_fence_before();
       mbar_arrive(bar(B_SFREE + st));
       const bool diag = sc.causal && (t == qt);
-      float mx = -INFINITY;
+      if (diag) {
 #pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        if (diag && i > r) s[i] = -INFINITY;
-        mx = fmaxf(mx, s[i]);
+        for (int i = 0; i < 128; ++i)
+          if (i > r) s[i] = -INFINITY;
       }
+      // Row max: eight independent chains of 3-input max.
+      float mx8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(s[2 * k], s[2 * k + 1]);
+#pragma unroll
+      for (int i = 16; i < 128; i += 16) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx8[k] = fmax3(mx8[k], s[i + 2 * k], s[i + 2 * k + 1]);
+      }
+      const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                             fmaxf(mx8[6], mx8[7]));
       const float m_cand = fmaxf(m_run, mx * c);
       const float m_new = (m_cand > m_run + 8.0f || m_run == -INFINITY) ? m_cand : m_run;
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
       const float alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_use);
-      float rsum = 0.f;
+      // P = 2^(s*c - m) in pairs; off the diagonal 3 of every 8 pairs go
+      // through the FMA-pipe polynomial, the rest through ex2.approx.
+      uint32_t pk[64];
+      uint64_t acc[4] = {0, 0, 0, 0};
+      const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-m_use, -m_use);
+      if (diag) {
 #pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        s[i] = ex2_approx(fmaf(s[i], c, -m_use));
-        rsum += s[i];
+        for (int q = 0; q < 64; ++q) {
+          float a, b;
+          f2_unpack(f2_fma(f2_pack(s[2 * q], s[2 * q + 1]), c2, nm2), a, b);
+          a = ex2_approx(a);
+          b = ex2_approx(b);
+          acc[q & 3] = f2_add(acc[q & 3], f2_pack(a, b));
+          pk[q] = pack_bf16x2(a, b);
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 64; ++q) {
+          const uint64_t x = f2_fma(f2_pack(s[2 * q], s[2 * q + 1]), c2, nm2);
+          float a, b;
+          if ((kPolyPairs >> (q & 7)) & 1u) {
+            f2_unpack(exp2_poly_x2(x), a, b);
+          } else {
+            f2_unpack(x, a, b);
+            a = ex2_approx(a);
+            b = ex2_approx(b);
+          }
+          acc[q & 3] = f2_add(acc[q & 3], f2_pack(a, b));
+          pk[q] = pack_bf16x2(a, b);
+        }
+      }
+      float rsum;
+      {
+        const uint64_t t01 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+        float lo, hi;
+        f2_unpack(t01, lo, hi);
+        rsum = lo + hi;
       }
       l_run = l_run * alpha + rsum;
       m_run = m_new;
@@ -281,10 +323,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       for (int ch = 0; ch < 16; ++ch) {
         const int half = ch >> 3, cw = ch & 7;
         const uint32_t addr = sP + half * kHalf + r * 128 + ((cw ^ (r & 7)) << 4);
-        st_shared_v4(addr, pack_bf16x2(s[ch * 8 + 0], s[ch * 8 + 1]),
-                     pack_bf16x2(s[ch * 8 + 2], s[ch * 8 + 3]),
-                     pack_bf16x2(s[ch * 8 + 4], s[ch * 8 + 5]),
-                     pack_bf16x2(s[ch * 8 + 6], s[ch * 8 + 7]));
+        st_shared_v4(addr, pk[ch * 4 + 0], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
       }
       fence_async_smem();
       tc_fence_before();

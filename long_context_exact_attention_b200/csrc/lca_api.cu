@@ -469,7 +469,9 @@ lca_status lca_check(void* stream) {
   if (h[0]) {
     const int z[2] = {0, 0};
     cudaMemcpyToSymbol(g_err, z, sizeof z);
-    return fail(LCA_ERR_TIMEOUT, "a kernel wait ran out (site %d)", h[1]);
+    if (h[0] & 1) return fail(LCA_ERR_TIMEOUT, "a kernel wait ran out (site %d)", h[1]);
+    return fail(LCA_ERR_CUDA, "a kernel could not align its shared-memory layout (site %d)",
+                h[1]);
   }
   return LCA_OK;
 }

@@ -97,6 +97,11 @@ WORKLOADS = {
         Workload("llama2_13b_s1m", B=1, Hq=40, Hkv=40, S=1048576, d=128,
                  dtype="bf16", causal=True, seed=4, std=0.5, kv_chunk=16384,
                  q_block=16384, order="ring", backward=False),
+        # a quarter of the 32K layer's heads: the case ncu captures in full
+        # (inputs 4 x 64 MiB, still larger than L2 together)
+        Workload("llama2_7b_s32k_h8", B=1, Hq=8, Hkv=8, S=32768, d=128,
+                 dtype="bf16", causal=True, seed=1, std=0.5, rope=True,
+                 kv_chunk=4096, order="ring"),
     ]
 }
 

@@ -1,0 +1,145 @@
+"""GPU parity at the five named workloads' full sizes, in the launch
+configuration bench.py times.  Where the whole output is too costly for the
+oracle, whole heads or exact sampled rows are checked (each sampled row is
+the oracle's full-row definition over every visible key), plus properties
+that hold at any size (global gradient identities, chunk-order invariance).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from long_context_exact_attention_b200 import lca
+from long_context_exact_attention_b200.inputs import WORKLOADS, chunk_permutation, make_inputs
+
+from gpu_util import (BF16_LSE_ABS, BF16_OUT_ABS, BF16_OUT_REL, GRAD_REL, assert_fwd_close,
+                      assert_grads_close, host, max_abs, rel_fro)
+
+pytestmark = pytest.mark.gpu
+
+
+def sample_rows(S, chunk, n_random, seed):
+    rows = set()
+    for c0 in range(0, S, chunk):
+        rows.update((c0, c0 + chunk - 1))
+    rng = np.random.default_rng(seed)
+    rows.update(rng.integers(0, S, n_random).tolist())
+    return np.array(sorted(rows))
+
+
+def check_rows(x, out, lse, w, heads, rows):
+    """Exact oracle rows vs GPU rows for the given heads."""
+    outs, refs = [], []
+    for h in heads:
+        g = h // (w.Hq // w.Hkv)
+        ro, rl = oracle.attention_rows(x["q"][:, :, h:h + 1], x["k"][:, :, g:g + 1],
+                                       x["v"][:, :, g:g + 1], w.causal, 0, 0, rows)
+        idx = torch.as_tensor(rows, device=out.device)
+        go = host(out[0, idx, h])
+        gl = host(lse[0, h, idx])
+        assert max_abs(go, ro) <= BF16_OUT_ABS, (h, max_abs(go, ro))
+        assert max_abs(gl, rl) <= BF16_LSE_ABS, (h, max_abs(gl, rl))
+        outs.append(go)
+        refs.append(ro)
+    r = rel_fro(np.stack(outs), np.stack(refs))
+    assert r <= BF16_OUT_REL, r
+
+
+def test_llama2_7b_s32k_ring_fwd_bwd():
+    w = WORKLOADS["llama2_7b_s32k"]
+    x = make_inputs(w, "cuda")
+    out, lse = lca.attn_fwd(x["q"], x["k"], x["v"], causal=True, kv_chunk=w.kv_chunk,
+                            order=w.order)
+    dq, dk, dv = lca.attn_bwd(x["q"], x["k"], x["v"], out, lse, x["dout"], causal=True)
+    torch.cuda.synchronize()
+    lca.check()
+    # two whole heads, forward and backward
+    for h in (0, w.Hq - 1):
+        sl = slice(h, h + 1)
+        ro, rl = oracle.attention_forward(x["q"][:, :, sl], x["k"][:, :, sl], x["v"][:, :, sl],
+                                          True)
+        assert_fwd_close(host(out[:, :, sl]), host(lse[:, sl]), ro, rl)
+        rg = oracle.attention_backward(x["q"][:, :, sl], x["k"][:, :, sl], x["v"][:, :, sl],
+                                       x["dout"][:, :, sl], True)
+        assert_grads_close([host(dq[:, :, sl]), host(dk[:, :, sl]), host(dv[:, :, sl])], rg)
+    # sampled rows in every head
+    rows = sample_rows(w.S, w.kv_chunk, 8, 1)
+    check_rows(x, out, lse, w, range(w.Hq), rows)
+
+
+def test_longlora_s2_s8k_fwd_bwd():
+    w = WORKLOADS["longlora_s2_s8k"]
+    x = make_inputs(w, "cuda")
+    out, lse = lca.s2attn_fwd(x["q"], x["k"], x["v"], w.group, w.shift_heads, causal=True)
+    dq, dk, dv = lca.s2attn_bwd(x["q"], x["k"], x["v"], out, lse, x["dout"], w.group,
+                                w.shift_heads, causal=True)
+    torch.cuda.synchronize()
+    lca.check()
+    ro, rl = oracle.s2attn_forward(x["q"], x["k"], x["v"], w.group, w.shift_heads, True)
+    assert_fwd_close(host(out), host(lse), ro, rl)
+    rg = oracle.s2attn_backward(x["q"], x["k"], x["v"], x["dout"], w.group, w.shift_heads, True)
+    assert_grads_close([host(dq), host(dk), host(dv)], rg)
+
+
+def test_llama3_8b_gqa_s128k_fwd_bwd_permuted():
+    w = WORKLOADS["llama3_8b_gqa_s128k"]
+    x = make_inputs(w, "cuda")
+    n = w.S // w.kv_chunk
+    out, lse = lca.attn_fwd(x["q"], x["k"], x["v"], causal=True, kv_chunk=w.kv_chunk)
+    out_p, lse_p = lca.attn_fwd(x["q"], x["k"], x["v"], causal=True, kv_chunk=w.kv_chunk,
+                                order="custom", chunk_perm=chunk_permutation(n, w.seed))
+    torch.cuda.synchronize()
+    # order-permuted run matches the in-order run (float32 rounding only)
+    assert max_abs(host(lse_p), host(lse)) <= 1e-4
+    assert (out_p.float() - out.float()).abs().max().item() <= 4e-3
+    rows = sample_rows(w.S, w.kv_chunk, 32, 3)
+    check_rows(x, out, lse, w, (0, 7, 20, 31), rows)
+    check_rows(x, out_p, lse_p, w, (3, 28), rows)
+
+    dq, dk, dv = lca.attn_bwd(x["q"], x["k"], x["v"], out, lse, x["dout"], causal=True)
+    torch.cuda.synchronize()
+    lca.check()
+    rep = w.Hq // w.Hkv
+    for g in (0, 5):
+        # dQ on sampled rows, exact per row
+        dq_r, _, _ = oracle.attention_backward_rows(x["q"], x["k"], x["v"], x["dout"], True, 0,
+                                                    g, rows)
+        got = host(dq[0, torch.as_tensor(rows, device="cuda"), g * rep:(g + 1) * rep])
+        assert rel_fro(got, dq_r) <= GRAD_REL, rel_fro(got, dq_r)
+    # dK/dV exact for keys in the last 1024 positions (only rows >= j contribute)
+    tail = np.arange(w.S - 1024, w.S)
+    _, dk_t, dv_t = oracle.attention_backward_rows(x["q"], x["k"], x["v"], x["dout"], True, 0,
+                                                   7, tail)
+    assert rel_fro(host(dk[0, -1024:, 7]), dk_t[-1024:]) <= GRAD_REL
+    assert rel_fro(host(dv[0, -1024:, 7]), dv_t[-1024:]) <= GRAD_REL
+    # global identities over all positions: sum_j dK_j = 0, sum_j dV_j = sum_i dO_i
+    dk64 = dk.double()
+    ratio = (dk64.sum(1).abs() / dk64.abs().sum(1)).max().item()
+    assert ratio <= 1e-2, ratio
+    want = x["dout"].double().sum(1).view(1, w.Hkv, rep, w.d).sum(2)
+    got = dv.double().sum(1)
+    assert ((got - want).norm() / want.norm()).item() <= 1e-2
+
+
+def test_llama2_13b_s1m_forward_sampled_blocks():
+    w = WORKLOADS["llama2_13b_s1m"]
+    x = make_inputs(w, "cuda", with_dout=False)
+    out, lse = lca.attn_fwd(x["q"], x["k"], x["v"], causal=True, kv_chunk=w.kv_chunk,
+                            order=w.order, q_block=w.q_block)
+    torch.cuda.synchronize()
+    lca.check()
+    blk = w.q_block
+    # query block 0 of head 0 in full: causal attention of the first block
+    sl = slice(0, blk)
+    ro, rl = oracle.attention_forward(x["q"][:, sl, :1], x["k"][:, sl, :1], x["v"][:, sl, :1],
+                                      True)
+    assert_fwd_close(host(out[:, sl, :1]), host(lse[:, :1, sl]), ro, rl)
+    # 8 sampled query blocks, 64 exact rows each (first, last and 62 random)
+    rng = np.random.default_rng(4)
+    rows = []
+    for b in (0, 9, 18, 27, 36, 45, 54, 63):
+        r0 = b * blk
+        rows += [r0, r0 + blk - 1] + (r0 + rng.integers(0, blk, 62)).tolist()
+    rows = np.array(sorted(set(rows)))
+    check_rows(x, out, lse, w, (0, 13, 26, 39), rows)
