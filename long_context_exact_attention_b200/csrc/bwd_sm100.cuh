@@ -7,22 +7,27 @@
 //   S^T  = K Q^T                  P^T = exp2(S^T * c - lse_i * log2 e)
 //   dP^T = V dO^T                 dS^T = P^T o (dP^T - D_i)
 //   dV  += P^T dO                 dK  += dS^T Q          (TMEM accumulators)
-//   dQ_i = dS K  -> fp32 atomics into the dq accumulator (scale applied later)
+//   dQ^T = K^T dS^T -> fp32 atomics into the dq accumulator (scale applied
+//                     later); computed transposed so that a warp's 32 lanes
+//                     hold 32 consecutive head dims of one query row and each
+//                     atomic instruction covers one whole 128-byte line
 //
 // One CTA per (key tile of 128, key/value head, batch); it loops over the
 // query heads of its grouped-query group and over the query tiles that can
 // see the key tile, so dK/dV of a key tile finish inside one CTA.
-// Roles (10 warps):
-//   warp 0      TMA producer: K, V once; Q, dO tiles plus lse/D rows per
-//               step through a 2-stage ring
-//   warp 1      TMEM owner; lane 0 issues the five MMAs of every step
-//   warps 2..5  P/dS warpgroup: one key row per thread.  P^T (bf16) is
-//               written back into the S^T columns it was computed from and
-//               feeds the dV product straight from tensor memory; dS^T goes
-//               to shared memory (it is the A operand of both dK and dQ)
-//   warps 6..9  dQ warpgroup: one query row per thread, drains dQ from TMEM
-//               and adds it to global memory; writes dV at the end
-// TMEM: S^T then P^T [0,128) | dP^T then dQ [128,256) | dV | dK
+// Roles (14 warps):
+//   warp 0       TMA producer: K, V once; Q, dO tiles plus lse/D rows per
+//                step through a 2-stage ring
+//   warp 1       TMEM owner; lane 0 issues the five MMAs of every step
+//   warps 2..9   P/dS: two warpgroups, one key row per thread, warpgroup h
+//                taking query columns [64h, 64h+64).  P^T (bf16) is written
+//                back inside the S^T columns the same warpgroup read
+//                ([64h, 64h+32)) and feeds the dV product straight from
+//                tensor memory; dS^T goes to shared memory (it is an operand
+//                of both dK and dQ^T)
+//   warps 10..13 dQ warpgroup: one head dim per thread, drains dQ^T from
+//                TMEM and adds it to global memory; writes dV at the end
+// TMEM: S^T then P^T [0,128) | dP^T then dQ^T [128,256) | dV | dK
 // Per step the tensor pipe runs S^T, dP^T, dV, dK, dQ; dV overlaps the dS
 // math, the next step's S^T overlaps the dQ drain.
 #pragma once
@@ -39,7 +44,7 @@ constexpr int kTile = 128;
 constexpr int kD = 128;
 constexpr uint32_t kHalf = kTile * 64 * 2;
 constexpr uint32_t kTileB = 2 * kHalf;
-constexpr int kThreads = 320;
+constexpr int kThreads = 448;
 
 constexpr uint32_t kOffK = 0;
 constexpr uint32_t kOffV = kOffK + kTileB;
@@ -75,7 +80,7 @@ enum {
 
 constexpr uint32_t kIdescKK = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T
 constexpr uint32_t kIdescKM = idesc_bf16_f32(128, 128, false, true);   // dV, dK
-constexpr uint32_t kIdescMM = idesc_bf16_f32(128, 128, true, true);    // dQ
+constexpr uint32_t kIdescMM = idesc_bf16_f32(128, 128, true, true);    // dQ^T
 
 // Pairs q (of the 64 per row and tile) with bit (q % 8) set would take the
 // FMA-pipe polynomial exp2 instead of ex2.approx.  Measured on B200 the
@@ -154,7 +159,9 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NUM_BARS; ++i) {
-      const uint32_t cnt = (i == B_PREADY || i == B_DSREADY || i == B_DQFREE) ? 128u : 1u;
+      const uint32_t cnt = (i == B_PREADY || i == B_DSREADY)  ? 256u
+                           : (i == B_DQFREE)                 ? 128u
+                                                             : 1u;
       mbar_init(bar(i), cnt);
     }
     *abort_flag = 0;
@@ -241,11 +248,12 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         ok = wait_bar(bar(B_PREADY), i & 1, wc, 215);
         if (!ok) break;
         tc_fence_after();
-        // dV += P^T dO, P^T read from tensor memory (8 columns per 16 queries)
+        // dV += P^T dO, P^T read from tensor memory: queries [0,64) at columns
+        // [0,32), queries [64,128) at [64,96), 8 columns per 16 queries
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          mma_bf16_ts(tdV, tSt + k * 8, sdesc_sw128(o_s + k * 2048, kHalf, 1024), kIdescKM,
-                      (i > 0 || k > 0));
+          mma_bf16_ts(tdV, tSt + (k >> 2) * 64 + (k & 3) * 8,
+                      sdesc_sw128(o_s + k * 2048, kHalf, 1024), kIdescKM, (i > 0 || k > 0));
         }
         tc_commit(bar(B_PTFREE));
         ok = wait_bar(bar(B_DSREADY), i & 1, wc, 216);
@@ -258,10 +266,12 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
                       sdesc_sw128(q_s + k * 2048, kHalf, 1024), kIdescKM, (i > 0 || k > 0));
         }
         tc_commit(bar(B_QEMPTY + st));
+        // dQ^T = K^T dS^T: A = K (head dims contiguous), B = dS^T (queries
+        // contiguous), both MN-major; K steps of 16 keys
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          mma_bf16_ss(tdP, sdesc_sw128(sS + k * 2048, kHalf, 1024),
-                      sdesc_sw128(sK + k * 2048, kHalf, 1024), kIdescMM, k > 0);
+          mma_bf16_ss(tdP, sdesc_sw128(sK + k * 2048, kHalf, 1024),
+                      sdesc_sw128(sS + k * 2048, kHalf, 1024), kIdescMM, k > 0);
         }
         tc_commit(bar(B_DQFULL));
         tc_commit(bar(B_DSFREE));
@@ -270,10 +280,11 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       tc_commit(bar(B_DRAIN));
       drain_bar(bar(B_DRAIN), 0, a.budget);
     }
-  } else if (warp < 6) {
-    // =================================================== P / dS warpgroup
+  } else if (warp < 10) {
+    // =================================================== P / dS warpgroups
+    const int hq = (warp - 2) >> 2;   // query-column half of this warpgroup
     const int wq = warp & 3;
-    const int r = wq * 32 + lane;  // key row
+    const int r = wq * 32 + lane;      // key row
     const uint32_t lad = static_cast<uint32_t>(wq * 32) << 16;
     const float c = a.scale_log2;
     const float L2E = 1.4426950408889634f;
@@ -282,41 +293,35 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     for (int i = 0; i < nsteps && ok; ++i) {
       const int st = i & 1;
       const int qt = qw.t + i % nq;
-      const float* lse_r = lse_s + st * 128;
-      const float* d_r = d_s + st * 128;
+      const float* lse_r = lse_s + st * 128 + hq * 64;
+      const float* d_r = d_s + st * 128 + hq * 64;
       ok = wait_bar(bar(B_SFULL), i & 1, wc, 311);
       if (ok) ok = wait_bar(bar(B_QFULL + st), (i >> 1) & 1, wc, 312);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
       const bool diag = sc.causal && qt == kt;
-      // ---- P^T = exp2(S^T c - lse log2e), written back over S^T as bf16
-      float p[128];
+      // ---- P^T = exp2(S^T c - lse log2e) for queries [64hq, 64hq+64),
+      // written back as bf16 over columns [64hq, 64hq+32) of S^T
+      float p[64];
+      tmem_ld64(tmem + lad + hq * 64, p);
+      {
+        uint32_t pk[32];
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        float s[32];
-        tmem_ld32(tmem + lad + cc * 32, s);
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int q0 = cc * 32 + e;
-          const uint64_t nl = f2_pack(-lse_r[q0] * L2E, -lse_r[q0 + 1] * L2E);
-          const uint64_t x = f2_fma(f2_pack(s[e], s[e + 1]), c2, nl);
+        for (int e = 0; e < 64; e += 2) {
+          const int q0 = hq * 64 + e;
+          const uint64_t nl = f2_pack(-lse_r[e] * L2E, -lse_r[e + 1] * L2E);
           float p0, p1;
-          if ((kPolyPairs >> ((q0 >> 1) & 7)) & 1u) {
-            f2_unpack(exp2_poly_x2(x), p0, p1);
-          } else {
-            f2_unpack(x, p0, p1);
-            p0 = ex2_approx(p0);
-            p1 = ex2_approx(p1);
-          }
+          f2_unpack(f2_fma(f2_pack(p[e], p[e + 1]), c2, nl), p0, p1);
+          p0 = ex2_approx(p0);
+          p1 = ex2_approx(p1);
           if (diag && r > q0) p0 = 0.f;
           if (diag && r > q0 + 1) p1 = 0.f;
-          p[q0] = p0;
-          p[q0 + 1] = p1;
+          p[e] = p0;
+          p[e + 1] = p1;
           pk[e >> 1] = pack_bf16x2(p0, p1);
         }
-        tmem_st16(tmem + lad + cc * 16, pk);
+        tmem_st32u(tmem + lad + hq * 64, pk);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -328,23 +333,22 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       if (!ok) break;
       tc_fence_after();
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
         float dp[32];
-        tmem_ld32(tmem + lad + 128 + cc * 32, dp);
+        tmem_ld32(tmem + lad + 128 + hq * 64 + cc * 32, dp);
         uint32_t dd[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const int q0 = cc * 32 + e;
-          const uint64_t t = f2_sub(f2_pack(dp[e], dp[e + 1]), f2_pack(d_r[q0], d_r[q0 + 1]));
+          const int ql = cc * 32 + e;
+          const uint64_t t = f2_sub(f2_pack(dp[e], dp[e + 1]), f2_pack(d_r[ql], d_r[ql + 1]));
           float t0, t1;
           f2_unpack(t, t0, t1);
-          dd[e >> 1] = pack_bf16x2(p[q0] * t0, p[q0 + 1] * t1);
+          dd[e >> 1] = pack_bf16x2(p[ql] * t0, p[ql + 1] * t1);
         }
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
-          const int ch = cc * 4 + v;
-          const int half = ch >> 3, cw = ch & 7;
-          const uint32_t off = half * kHalf + r * 128 + ((cw ^ (r & 7)) << 4);
+          const int cw = cc * 4 + v;  // 16-byte chunk within this half's 128-byte row
+          const uint32_t off = hq * kHalf + r * 128 + ((cw ^ (r & 7)) << 4);
           st_shared_v4(sS + off, dd[4 * v], dd[4 * v + 1], dd[4 * v + 2], dd[4 * v + 3]);
         }
       }
@@ -352,14 +356,14 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(B_DSREADY));
     }
-    // ---- dK = scale * acc -> bf16
+    // ---- dK = scale * acc -> bf16 (columns split between the two halves)
     if (ok) ok = wait_bar(bar(B_DONE), 0, wc, 315);
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
       tc_fence_after();
       __nv_bfloat16* row = a.dk + ((static_cast<size_t>(b) * a.S + ktok0 + r) * a.Hkv + g) * kD;
 #pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 2 * hq; cc < 2 * hq + 2; ++cc) {
         float o[32];
         tmem_ld32(tmem + lad + 384 + cc * 32, o);
 #pragma unroll
@@ -376,7 +380,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
   } else {
     // =================================================== dQ warpgroup
     const int wq = warp & 3;
-    const int r = wq * 32 + lane;  // query row (dQ) / key row (dV)
+    const int r = wq * 32 + lane;  // head dim (dQ^T) / key row (dV)
     const uint32_t lad = static_cast<uint32_t>(wq * 32) << 16;
     bool ok = true;
     for (int i = 0; i < nsteps && ok; ++i) {
@@ -386,16 +390,19 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       ok = __all_sync(0xffffffffu, wait_bar(bar(B_DQFULL), i & 1, wc, 411));
       if (!ok) break;
       tc_fence_after();
-      float dq[128];
-      tmem_ld128(tmem + lad + 128, dq);
+      // row q of this query tile, head dim r: lanes of a warp cover 32
+      // consecutive floats of one row
+      float* dst = a.dq_acc + ((static_cast<size_t>(b) * a.S + qtok0) * a.Hq + h) * kD + r;
+      const size_t row_stride = static_cast<size_t>(a.Hq) * kD;
+      float dq[64];
+      tmem_ld64(tmem + lad + 128, dq);
+#pragma unroll
+      for (int q = 0; q < 64; ++q) atomicAdd(dst + q * row_stride, dq[q]);
+      tmem_ld64(tmem + lad + 192, dq);
       tc_fence_before();
       mbar_arrive(bar(B_DQFREE));
-      float4* dst = reinterpret_cast<float4*>(
-          a.dq_acc + ((static_cast<size_t>(b) * a.S + qtok0 + r) * a.Hq + h) * kD);
 #pragma unroll
-      for (int v = 0; v < 32; ++v) {
-        atomicAdd(dst + v, make_float4(dq[4 * v], dq[4 * v + 1], dq[4 * v + 2], dq[4 * v + 3]));
-      }
+      for (int q = 0; q < 64; ++q) atomicAdd(dst + (64 + q) * row_stride, dq[q]);
     }
     // ---- dV -> bf16
     if (ok) ok = wait_bar(bar(B_DONE), 0, wc, 412);

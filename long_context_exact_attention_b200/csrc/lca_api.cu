@@ -221,6 +221,8 @@ lca_status run_fwd(const Common& c, const AttnSched& s, const void* q, const voi
   const int64_t tokens = static_cast<int64_t>(c.B) * c.S;
   const unsigned grid = static_cast<unsigned>(s.n_tiles) * c.B * c.Hq;
   if (c.dtype == LCA_BF16) {
+    // one CTA per pair of 128-row query tiles
+    const unsigned grid2 = static_cast<unsigned>((s.n_tiles + 1) / 2) * c.B * c.Hq;
     CUtensorMap mq, mk, mv;
     lca_status r;
     if ((r = make_map(&mq, q, tokens, c.Hq)) != LCA_OK) return r;
@@ -237,7 +239,7 @@ lca_status run_fwd(const Common& c, const AttnSched& s, const void* q, const voi
     a.out = static_cast<__nv_bfloat16*>(out);
     a.lse = lse;
     a.sched = s;
-    attn_fwd_bf16_sm100<<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(mq, mk, mv, a);
+    attn_fwd_bf16_sm100<<<grid2, fwd::kThreads, fwd::kSmemBytes, st>>>(mq, mk, mv, a);
     return launched("attn_fwd_bf16_sm100");
   }
   f32::Args a{};
