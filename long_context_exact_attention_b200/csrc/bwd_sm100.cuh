@@ -7,32 +7,28 @@
 //   S^T  = K Q^T                  P^T = exp2(S^T * c - lse_i * log2 e)
 //   dP^T = V dO^T                 dS^T = P^T o (dP^T - D_i)
 //   dV  += P^T dO                 dK  += dS^T Q          (TMEM accumulators)
-//   dQ^T = K^T dS^T -> fp32 atomics into the dq accumulator (scale applied
-//                     later); computed transposed so that a warp's 32 lanes
-//                     hold 32 consecutive head dims of one query row and each
-//                     atomic instruction covers one whole 128-byte line
+//   dQ^T = K^T dS^T -> added into the fp32 dq accumulator by TMA bulk
+//                      reduce-add (scale applied later)
 //
 // One CTA per (key tile of 128, key/value head, batch); it loops over the
 // query heads of its grouped-query group and over the query tiles that can
 // see the key tile, so dK/dV of a key tile finish inside one CTA.
-// Roles (14 warps):
-//   warp 0       TMA producer: K, V once; Q, dO tiles plus lse/D rows per
-//                step through a 2-stage ring
-//   warp 1       TMEM owner; lane 0 issues the five MMAs of every step
-//   warps 2..9   P/dS: two warpgroups, one key row per thread, warpgroup h
-//                taking query columns [64h, 64h+64).  P^T (bf16) is written
-//                back inside the S^T columns the same warpgroup read
-//                ([64h, 64h+32)) and feeds the dV product straight from
-//                tensor memory; dS^T goes to shared memory (it is an operand
-//                of both dK and dQ^T)
-//   warps 10..13 dQ warpgroup: one head dim per thread, drains dQ^T from
-//                TMEM and adds it to global memory; writes dV at the end
+// Roles (16 warps, four warpgroups):
+//   warpgroup 0  warp 0: TMA producer (K, V once; Q + lse/D rows through a
+//                2-stage ring, dO single-staged); warp 1: TMEM owner, lane 0
+//                issues the five MMAs of every step; warps 2-3 idle.  The
+//                warpgroup gives up registers to the other three.
+//   warpgroups 1, 2  P/dS: one key row per thread, warpgroup h taking query
+//                columns [64(h-1), 64h).  P^T (bf16) is written back inside
+//                the S^T columns the same warpgroup read and feeds the dV
+//                product straight from tensor memory; dS^T goes to shared
+//                memory (an operand of both dK and dQ^T)
+//   warpgroup 3  dQ: one head dim per thread; moves dQ^T from TMEM through
+//                shared memory (one [64 query x 32 dim] box per warp) into
+//                a TMA reduce-add of the accumulator; writes dV at the end
 // TMEM: S^T then P^T [0,128) | dP^T then dQ^T [128,256) | dV | dK
-// Per step the tensor pipe runs S^T, dP^T, dV, dK, dQ; dV overlaps the dS
-// math, the next step's S^T overlaps the dQ drain.
 #pragma once
 
-#include "exp2_poly.cuh"
 #include "ptx.cuh"
 #include "sched.cuh"
 
@@ -44,14 +40,21 @@ constexpr int kTile = 128;
 constexpr int kD = 128;
 constexpr uint32_t kHalf = kTile * 64 * 2;
 constexpr uint32_t kTileB = 2 * kHalf;
-constexpr int kThreads = 448;
+constexpr int kThreads = 512;
+// Registers per thread at launch (launch bounds 512 x 1 CTA) and the split
+// the warpgroups take with setmaxnreg: 56 + 3 * 152 = 4 * 128.
+constexpr int kRegsLaunch = 128;
+constexpr int kRegsCtl = 56;
+constexpr int kRegsWork = 152;
+static_assert(kRegsCtl + 3 * kRegsWork == 4 * kRegsLaunch, "register split");
 
 constexpr uint32_t kOffK = 0;
 constexpr uint32_t kOffV = kOffK + kTileB;
 constexpr uint32_t kOffQ = kOffV + kTileB;        // 2 stages
-constexpr uint32_t kOffO = kOffQ + 2 * kTileB;    // dO, 2 stages
-constexpr uint32_t kOffS = kOffO + 2 * kTileB;    // dS^T
-constexpr uint32_t kOffL = kOffS + kTileB;        // lse[2][128]
+constexpr uint32_t kOffO = kOffQ + 2 * kTileB;    // dO, 1 stage
+constexpr uint32_t kOffS = kOffO + kTileB;        // dS^T
+constexpr uint32_t kOffR = kOffS + kTileB;        // dQ staging, 4 warps x 8 KB
+constexpr uint32_t kOffL = kOffR + 4 * 8192;      // lse[2][128]
 constexpr uint32_t kOffD = kOffL + 1024;          // D[2][128]
 constexpr uint32_t kOffBar = kOffD + 1024;
 constexpr uint32_t kUsed = kOffBar + 256;
@@ -60,16 +63,19 @@ constexpr uint32_t kUsed = kOffBar + 256;
 // to 1024 bytes would need more than that slack.
 constexpr uint32_t kSmemBytes = 232448;
 constexpr uint32_t kSlack = kSmemBytes - kUsed;
+static_assert(kUsed <= kSmemBytes, "shared memory");
 
 enum {
   B_KV = 0,
   B_QFULL,        // +stage
   B_QEMPTY = 3,   // +stage
-  B_SFULL = 5,
+  B_OFULL = 5,
+  B_OEMPTY,
+  B_SFULL,
   B_DPFULL,
-  B_PREADY,       // 128 arrivals
+  B_PREADY,       // 256 arrivals
   B_PTFREE,
-  B_DSREADY,      // 128 arrivals
+  B_DSREADY,      // 256 arrivals
   B_DSFREE,
   B_DQFULL,
   B_DQFREE,       // 128 arrivals
@@ -82,11 +88,6 @@ constexpr uint32_t kIdescKK = idesc_bf16_f32(128, 128, false, false);  // S^T, d
 constexpr uint32_t kIdescKM = idesc_bf16_f32(128, 128, false, true);   // dV, dK
 constexpr uint32_t kIdescMM = idesc_bf16_f32(128, 128, true, true);    // dQ^T
 
-// Pairs q (of the 64 per row and tile) with bit (q % 8) set would take the
-// FMA-pipe polynomial exp2 instead of ex2.approx.  Measured on B200 the
-// mixes tried (3/8, 4/8) were slower than none, so none is used.
-constexpr uint32_t kPolyPairs = 0u;
-
 struct Args {
   int B, Hq, Hkv, S;
   float scale;
@@ -94,7 +95,6 @@ struct Args {
   unsigned long long budget;
   const float* lse;      // [B,Hq,S]
   const float* Drow;     // [B,Hq,S]
-  float* dq_acc;         // [B,S,Hq,d] fp32, zeroed
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   AttnSched sched;
@@ -116,6 +116,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
                         const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV,
                         const __grid_constant__ CUtensorMap tmDO,
+                        const __grid_constant__ CUtensorMap tmDQ,
                         const __grid_constant__ bwd::Args a) {
   using namespace bwd;
   extern __shared__ uint8_t smem_raw[];
@@ -131,7 +132,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
   }
   uint8_t* gbase = smem_raw + (base - raw);
   const uint32_t sK = base + kOffK, sV = base + kOffV, sQ = base + kOffQ, sO = base + kOffO;
-  const uint32_t sS = base + kOffS, sL = base + kOffL, sD = base + kOffD;
+  const uint32_t sS = base + kOffS, sR = base + kOffR, sL = base + kOffL, sD = base + kOffD;
   const float* lse_s = reinterpret_cast<const float*>(gbase + kOffL);
   const float* d_s = reinterpret_cast<const float*>(gbase + kOffD);
   const uint32_t bars = base + kOffBar;
@@ -141,6 +142,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int wg = warp >> 2;
 
   const AttnSched& sc = a.sched;
   const int rep = a.Hq / a.Hkv;
@@ -159,7 +161,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NUM_BARS; ++i) {
-      const uint32_t cnt = (i == B_PREADY || i == B_DSREADY)  ? 256u
+      const uint32_t cnt = (i == B_PREADY || i == B_DSREADY) ? 256u
                            : (i == B_DQFREE)                 ? 128u
                                                              : 1u;
       mbar_init(bar(i), cnt);
@@ -178,9 +180,10 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
   WaitCtl wc{abort_flag, a.budget};
   const int row0 = b * a.S;
 
-  if (warp == 0) {
-    // =================================================== TMA producer
-    if (lane == 0) {
+  if (wg == 0) {
+    regs_dec<kRegsCtl>();
+    if (warp == 0 && lane == 0) {
+      // =================================================== TMA producer
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
@@ -191,7 +194,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       tma_load_3d(sV, &tmV, bar(B_KV), 0, g, row0 + ktok0);
       tma_load_3d(sV + kHalf, &tmV, bar(B_KV), 64, g, row0 + ktok0);
       bool ok = true;
-      int issued0 = 0, issued1 = 0;
+      int issued0 = 0, issued1 = 0, o_issued = 0;
       for (int i = 0; i < nsteps && ok; ++i) {
         const int st = i & 1;
         const int h = g * rep + i / nq;
@@ -200,30 +203,33 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         if (i >= 2) ok = wait_bar(bar(B_QEMPTY + st), ((i - 2) >> 1) & 1, wc, 111);
         if (!ok) break;
         const uint32_t fb = bar(B_QFULL + st);
-        mbar_expect_tx(fb, 2 * kTileB + 1024);
+        mbar_expect_tx(fb, kTileB + 1024);
         tma_load_3d(sQ + st * kTileB, &tmQ, fb, 0, h, row0 + qtok0);
         tma_load_3d(sQ + st * kTileB + kHalf, &tmQ, fb, 64, h, row0 + qtok0);
-        tma_load_3d(sO + st * kTileB, &tmDO, fb, 0, h, row0 + qtok0);
-        tma_load_3d(sO + st * kTileB + kHalf, &tmDO, fb, 64, h, row0 + qtok0);
         const size_t ro = (static_cast<size_t>(b) * a.Hq + h) * a.S + qtok0;
         bulk_load(sL + st * 512, a.lse + ro, 512, fb);
         bulk_load(sD + st * 512, a.Drow + ro, 512, fb);
         if (st) ++issued1; else ++issued0;
+        if (i >= 1) ok = wait_bar(bar(B_OEMPTY), (i - 1) & 1, wc, 112);
+        if (!ok) break;
+        mbar_expect_tx(bar(B_OFULL), kTileB);
+        tma_load_3d(sO, &tmDO, bar(B_OFULL), 0, h, row0 + qtok0);
+        tma_load_3d(sO + kHalf, &tmDO, bar(B_OFULL), 64, h, row0 + qtok0);
+        ++o_issued;
       }
       if (!ok) {
         drain_bar(bar(B_KV), 0, a.budget);
         if (issued0) drain_bar(bar(B_QFULL), (issued0 - 1) & 1, a.budget);
         if (issued1) drain_bar(bar(B_QFULL + 1), (issued1 - 1) & 1, a.budget);
+        if (o_issued) drain_bar(bar(B_OFULL), (o_issued - 1) & 1, a.budget);
       }
-    }
-  } else if (warp == 1) {
-    // =================================================== MMA issuer
-    if (lane == 0) {
+    } else if (warp == 1 && lane == 0) {
+      // =================================================== MMA issuer
       const uint32_t tSt = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 384;
       bool ok = wait_bar(bar(B_KV), 0, wc, 211);
       for (int i = 0; i < nsteps && ok; ++i) {
         const int st = i & 1;
-        const uint32_t q_s = sQ + st * kTileB, o_s = sO + st * kTileB;
+        const uint32_t q_s = sQ + st * kTileB;
         ok = wait_bar(bar(B_QFULL + st), (i >> 1) & 1, wc, 212);
         if (ok && i >= 1) ok = wait_bar(bar(B_PTFREE), (i - 1) & 1, wc, 213);
         if (!ok) break;
@@ -235,17 +241,18 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
                       kIdescKK, k > 0);
         }
         tc_commit(bar(B_SFULL));
-        if (i >= 1) ok = wait_bar(bar(B_DQFREE), (i - 1) & 1, wc, 214);
+        ok = wait_bar(bar(B_OFULL), i & 1, wc, 214);
+        if (ok && i >= 1) ok = wait_bar(bar(B_DQFREE), (i - 1) & 1, wc, 215);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t off = (k >> 2) * kHalf + (k & 3) * 32;
-          mma_bf16_ss(tdP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(o_s + off, 16, 1024),
+          mma_bf16_ss(tdP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sO + off, 16, 1024),
                       kIdescKK, k > 0);
         }
         tc_commit(bar(B_DPFULL));
-        ok = wait_bar(bar(B_PREADY), i & 1, wc, 215);
+        ok = wait_bar(bar(B_PREADY), i & 1, wc, 216);
         if (!ok) break;
         tc_fence_after();
         // dV += P^T dO, P^T read from tensor memory: queries [0,64) at columns
@@ -253,10 +260,11 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           mma_bf16_ts(tdV, tSt + (k >> 2) * 64 + (k & 3) * 8,
-                      sdesc_sw128(o_s + k * 2048, kHalf, 1024), kIdescKM, (i > 0 || k > 0));
+                      sdesc_sw128(sO + k * 2048, kHalf, 1024), kIdescKM, (i > 0 || k > 0));
         }
         tc_commit(bar(B_PTFREE));
-        ok = wait_bar(bar(B_DSREADY), i & 1, wc, 216);
+        tc_commit(bar(B_OEMPTY));
+        ok = wait_bar(bar(B_DSREADY), i & 1, wc, 217);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -280,9 +288,10 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       tc_commit(bar(B_DRAIN));
       drain_bar(bar(B_DRAIN), 0, a.budget);
     }
-  } else if (warp < 10) {
+  } else if (wg <= 2) {
+    regs_inc<kRegsWork>();
     // =================================================== P / dS warpgroups
-    const int hq = (warp - 2) >> 2;   // query-column half of this warpgroup
+    const int hq = wg - 1;             // query-column half of this warpgroup
     const int wq = warp & 3;
     const int r = wq * 32 + lane;      // key row
     const uint32_t lad = static_cast<uint32_t>(wq * 32) << 16;
@@ -332,15 +341,15 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
+      float dp[64];
+      tmem_ld64(tmem + lad + 128 + hq * 64, dp);
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
-        float dp[32];
-        tmem_ld32(tmem + lad + 128 + hq * 64 + cc * 32, dp);
         uint32_t dd[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           const int ql = cc * 32 + e;
-          const uint64_t t = f2_sub(f2_pack(dp[e], dp[e + 1]), f2_pack(d_r[ql], d_r[ql + 1]));
+          const uint64_t t = f2_sub(f2_pack(dp[ql], dp[ql + 1]), f2_pack(d_r[ql], d_r[ql + 1]));
           float t0, t1;
           f2_unpack(t, t0, t1);
           dd[e >> 1] = pack_bf16x2(p[ql] * t0, p[ql + 1] * t1);
@@ -378,10 +387,14 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       }
     }
   } else {
+    regs_inc<kRegsWork>();
     // =================================================== dQ warpgroup
     const int wq = warp & 3;
     const int r = wq * 32 + lane;  // head dim (dQ^T) / key row (dV)
     const uint32_t lad = static_cast<uint32_t>(wq * 32) << 16;
+    // this warp's staging box: [64 queries][32 head dims] fp32, rows of 128 B
+    const uint32_t stage = sR + wq * 8192 + lane * 4;
+    if (lane == 0) tma_prefetch_desc(&tmDQ);
     bool ok = true;
     for (int i = 0; i < nsteps && ok; ++i) {
       const int h = g * rep + i / nq;
@@ -390,20 +403,32 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       ok = __all_sync(0xffffffffu, wait_bar(bar(B_DQFULL), i & 1, wc, 411));
       if (!ok) break;
       tc_fence_after();
-      // row q of this query tile, head dim r: lanes of a warp cover 32
-      // consecutive floats of one row
-      float* dst = a.dq_acc + ((static_cast<size_t>(b) * a.S + qtok0) * a.Hq + h) * kD + r;
-      const size_t row_stride = static_cast<size_t>(a.Hq) * kD;
-      float dq[64];
-      tmem_ld64(tmem + lad + 128, dq);
-#pragma unroll
-      for (int q = 0; q < 64; ++q) atomicAdd(dst + q * row_stride, dq[q]);
-      tmem_ld64(tmem + lad + 192, dq);
+      float dq0[64], dq1[64];
+      tmem_ld64(tmem + lad + 128, dq0);
+      tmem_ld64(tmem + lad + 192, dq1);
       tc_fence_before();
       mbar_arrive(bar(B_DQFREE));
 #pragma unroll
-      for (int q = 0; q < 64; ++q) atomicAdd(dst + (64 + q) * row_stride, dq[q]);
+      for (int half = 0; half < 2; ++half) {
+        // the previous reduce from this buffer must have read it
+        if (lane == 0) bulk_wait_read0();
+        __syncwarp();
+#pragma unroll
+        for (int q = 0; q < 64; ++q) {
+          asm volatile("st.shared.f32 [%0], %1;" ::"r"(stage + q * 128),
+                       "f"(half ? dq1[q] : dq0[q])
+                       : "memory");
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_3d(&tmDQ, sR + wq * 8192, wq * 32, h, row0 + qtok0 + half * 64);
+          bulk_commit();
+        }
+      }
     }
+    if (lane == 0) bulk_wait0();
+    __syncwarp();
     // ---- dV -> bf16
     if (ok) ok = wait_bar(bar(B_DONE), 0, wc, 412);
     ok = __all_sync(0xffffffffu, ok);

@@ -187,6 +187,45 @@ lca_status make_map(CUtensorMap* m, const void* ptr, int64_t tokens, int64_t hea
   return LCA_OK;
 }
 
+// fp32 [tokens][heads][128] accumulator viewed 3-D; box = 32 head dims x 1
+// head x 64 tokens, no swizzle (the box's rows are 128 bytes).
+lca_status make_map_acc(CUtensorMap* m, const void* ptr, int64_t tokens, int64_t heads) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(LCA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(heads),
+                              static_cast<cuuint64_t>(tokens)};
+  const cuuint64_t strides[2] = {128 * 4, static_cast<cuuint64_t>(heads) * 128 * 4};
+  const cuuint32_t box[3] = {32, 1, 64};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(LCA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return LCA_OK;
+}
+
+// The backward kernel's warpgroups redistribute registers with setmaxnreg;
+// the split adds up to exactly the registers the CTA is launched with, so
+// refuse to launch a build whose register count differs.
+lca_status check_bwd_regs() {
+  static int regs = -1;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lk(mu);
+  if (regs < 0) {
+    cudaFuncAttributes attr{};
+    const cudaError_t e = cudaFuncGetAttributes(&attr, attn_bwd_bf16_sm100);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes(backward)");
+    regs = attr.numRegs;
+  }
+  if (regs != bwd::kRegsLaunch)
+    return fail(LCA_ERR_UNSUPPORTED,
+                "backward kernel built with %d registers per thread; its register split "
+                "needs exactly %d",
+                regs, bwd::kRegsLaunch);
+  return LCA_OK;
+}
+
 // Raise the dynamic shared-memory limit of a kernel once per device.
 template <typename K>
 lca_status ensure_smem(K kernel, size_t bytes, int slot) {
@@ -300,11 +339,13 @@ lca_status run_bwd(const Common& c, const AttnSched& s, const void* q, const voi
     lca_status r = launched("bwd_rowdot");
     if (r != LCA_OK) return r;
     const int64_t tokens = static_cast<int64_t>(c.B) * c.S;
-    CUtensorMap mq, mk, mv, mdo;
+    CUtensorMap mq, mk, mv, mdo, mdq;
     if ((r = make_map(&mq, q, tokens, c.Hq)) != LCA_OK) return r;
     if ((r = make_map(&mk, k, tokens, c.Hkv)) != LCA_OK) return r;
     if ((r = make_map(&mv, v, tokens, c.Hkv)) != LCA_OK) return r;
     if ((r = make_map(&mdo, dout, tokens, c.Hq)) != LCA_OK) return r;
+    if ((r = make_map_acc(&mdq, acc, tokens, c.Hq)) != LCA_OK) return r;
+    if ((r = check_bwd_regs()) != LCA_OK) return r;
     if ((r = ensure_smem(attn_bwd_bf16_sm100, bwd::kSmemBytes, 3)) != LCA_OK) return r;
     bwd::Args a;
     a.B = c.B;
@@ -316,11 +357,10 @@ lca_status run_bwd(const Common& c, const AttnSched& s, const void* q, const voi
     a.budget = budget;
     a.lse = lse;
     a.Drow = Drow;
-    a.dq_acc = acc;
     a.dk = static_cast<__nv_bfloat16*>(dk);
     a.dv = static_cast<__nv_bfloat16*>(dv);
     a.sched = s;
-    attn_bwd_bf16_sm100<<<grid, bwd::kThreads, bwd::kSmemBytes, st>>>(mq, mk, mv, mdo, a);
+    attn_bwd_bf16_sm100<<<grid, bwd::kThreads, bwd::kSmemBytes, st>>>(mq, mk, mv, mdo, mdq, a);
     if ((r = launched("attn_bwd_bf16_sm100")) != LCA_OK) return r;
     const int64_t n8 = rows * c.d / 8;
     dq_finalize<<<static_cast<unsigned>(std::min<int64_t>((n8 + 255) / 256, 148 * 16)), 256, 0,
