@@ -146,10 +146,11 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
 
   const AttnSched& sc = a.sched;
   const int rep = a.Hq / a.Hkv;
-  const int BG = a.B * a.Hkv;
-  // Longest causal work first: key tile 0 sees every query tile.
-  const int kt = static_cast<int>(blockIdx.x) / BG;
-  const int bg = static_cast<int>(blockIdx.x) % BG;
+  // Head-major order (the CTAs in flight update one or two heads' dq rows,
+  // which stay in L2), longest causal work first within a head: key tile 0
+  // sees every query tile.
+  const int kt = static_cast<int>(blockIdx.x) % sc.n_tiles;
+  const int bg = static_cast<int>(blockIdx.x) / sc.n_tiles;
   const int g = bg % a.Hkv;
   const int b = bg / a.Hkv;
   const bool shifted = head_shifted(sc, g * rep);

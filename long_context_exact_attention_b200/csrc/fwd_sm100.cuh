@@ -103,12 +103,13 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work item: a pair of query tiles; longest causal pairs first
+  // ---- work item: a pair of query tiles.  Head-major order (the CTAs in
+  // flight share one or two heads' K/V in L2), longest causal pairs first
+  // within a head.
   const AttnSched& sc = a.sched;
   const int n_pairs = (sc.n_tiles + 1) >> 1;
-  const int BH = a.B * a.Hq;
-  const int pr = n_pairs - 1 - static_cast<int>(blockIdx.x) / BH;
-  const int bh = static_cast<int>(blockIdx.x) % BH;
+  const int pr = n_pairs - 1 - static_cast<int>(blockIdx.x) % n_pairs;
+  const int bh = static_cast<int>(blockIdx.x) / n_pairs;
   const int h = bh % a.Hq;
   const int b = bh / a.Hq;
   const int g = h / (a.Hq / a.Hkv);
