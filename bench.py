@@ -132,6 +132,26 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(rows)}
 
 
+# ---------------------------------------------------------------- ranks
+
+def max_over_ranks(value, device=None):
+    """Maximum of a per-rank float over all ranks of the default process
+    group (the value itself when there is no group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device or "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_step, world, steps, max_ms):
+    """Whole-job throughput: every rank runs `steps` steps of the same
+    workload (replicas), timed by the slowest rank."""
+    return flops_per_step * world * steps / (max_ms * 1e-3) / 1e12
+
+
 # ---------------------------------------------------------------- CPU oracle
 
 def oracle_sample(w, seconds_target=12.0, max_rows=None):
@@ -276,12 +296,9 @@ def main():
     total_ms = start.elapsed_time(stop)
     fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
     bwd_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dev)
     ms_step = total_ms / args.steps
-    value = flops_step * world * args.steps / (total_ms * 1e-3) / 1e12
+    value = whole_job_tflops(flops_step, world, args.steps, total_ms)
 
     # ---- end to end through the C ABI with pinned host buffers
     e2e = None
@@ -315,12 +332,8 @@ def main():
                 e2e_step()
             s1.record(stream)
             s1.synchronize()
-        e_ms = s0.elapsed_time(s1)
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": flops_step * world * n_e2e / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e_ms = max_over_ranks(s0.elapsed_time(s1), dev)
+        e2e = {"value": whole_job_tflops(flops_step, world, n_e2e, e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e_ms / n_e2e}
 

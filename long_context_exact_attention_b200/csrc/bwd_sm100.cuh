@@ -74,7 +74,6 @@ enum {
   B_SFULL,
   B_DPFULL,
   B_PREADY,       // 256 arrivals
-  B_PTFREE,
   B_DSREADY,      // 256 arrivals
   B_DSFREE,
   B_DQFULL,
@@ -226,15 +225,13 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       }
     } else if (warp == 1 && lane == 0) {
       // =================================================== MMA issuer
+      // Order per step i: dP^T_i, dV_i, S^T_{i+1}, dK_i, dQ^T_i.  S^T_{i+1}
+      // goes right behind dV_i, the last reader of the S^T/P^T columns (the
+      // tensor pipe runs this thread's MMAs in order), so the next step's
+      // P phase overlaps dK_i and dQ^T_i.
       const uint32_t tSt = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 384;
-      bool ok = wait_bar(bar(B_KV), 0, wc, 211);
-      for (int i = 0; i < nsteps && ok; ++i) {
-        const int st = i & 1;
-        const uint32_t q_s = sQ + st * kTileB;
-        ok = wait_bar(bar(B_QFULL + st), (i >> 1) & 1, wc, 212);
-        if (ok && i >= 1) ok = wait_bar(bar(B_PTFREE), (i - 1) & 1, wc, 213);
-        if (!ok) break;
-        tc_fence_after();
+      auto issue_s = [&](int i) {
+        const uint32_t q_s = sQ + (i & 1) * kTileB;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t off = (k >> 2) * kHalf + (k & 3) * 32;
@@ -242,6 +239,16 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
                       kIdescKK, k > 0);
         }
         tc_commit(bar(B_SFULL));
+      };
+      bool ok = wait_bar(bar(B_KV), 0, wc, 211);
+      if (ok && nsteps > 0) ok = wait_bar(bar(B_QFULL), 0, wc, 212);
+      if (ok && nsteps > 0) {
+        tc_fence_after();
+        issue_s(0);
+      }
+      for (int i = 0; i < nsteps && ok; ++i) {
+        const int st = i & 1;
+        const uint32_t q_s = sQ + st * kTileB;
         ok = wait_bar(bar(B_OFULL), i & 1, wc, 214);
         if (ok && i >= 1) ok = wait_bar(bar(B_DQFREE), (i - 1) & 1, wc, 215);
         if (!ok) break;
@@ -263,8 +270,13 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
           mma_bf16_ts(tdV, tSt + (k >> 2) * 64 + (k & 3) * 8,
                       sdesc_sw128(sO + k * 2048, kHalf, 1024), kIdescKM, (i > 0 || k > 0));
         }
-        tc_commit(bar(B_PTFREE));
         tc_commit(bar(B_OEMPTY));
+        if (i + 1 < nsteps) {
+          ok = wait_bar(bar(B_QFULL + (st ^ 1)), ((i + 1) >> 1) & 1, wc, 213);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(i + 1);
+        }
         ok = wait_bar(bar(B_DSREADY), i & 1, wc, 217);
         if (!ok) break;
         tc_fence_after();
