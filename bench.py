@@ -258,11 +258,18 @@ def main():
     def step(ev=None):
         if ev:
             ev[0].record(stream)
-        lca.attn_fwd(q, k, v, causal=w.causal, kv_chunk=w.kv_chunk, order=w.order,
-                     q_block=w.q_block, out=out, lse=lse, stream=stream)
+        if w.s2:
+            lca.s2attn_fwd(q, k, v, w.group, w.shift_heads, causal=w.causal, out=out, lse=lse,
+                           stream=stream)
+        else:
+            lca.attn_fwd(q, k, v, causal=w.causal, kv_chunk=w.kv_chunk, order=w.order,
+                         q_block=w.q_block, out=out, lse=lse, stream=stream)
         if ev:
             ev[1].record(stream)
-        if w.backward:
+        if w.backward and w.s2:
+            lca.s2attn_bwd(q, k, v, out, lse, dout, w.group, w.shift_heads, causal=w.causal,
+                           dq=dq, dk=dk, dv=dv, workspace=ws, stream=stream)
+        elif w.backward:
             lca.attn_bwd(q, k, v, out, lse, dout, causal=w.causal, dq=dq, dk=dk, dv=dv,
                          workspace=ws, stream=stream)
         if ev:
@@ -368,6 +375,7 @@ def main():
         "data": "synthetic", "impl": "lca",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "S": w.S, "d": w.d,
                    "causal": w.causal, "kv_chunk": w.kv_chunk, "order": w.order,
+                   "s2_group": w.group or None, "s2_shift_heads": w.shift_heads or None,
                    "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (q, k, v, dout 256 MiB each); no flush"},
         "fwd_tflops": w.fwd_flops() / (fwd_t * 1e-3) / 1e12, "fwd_ms": fwd_t,
