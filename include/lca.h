@@ -24,10 +24,11 @@
  *
  * Element types
  *   LCA_BF16: q, k, v, out, dout, dq, dk, dv are bfloat16; accumulation in
- *             float32 on the tensor cores; requires d == 128 and S a multiple
- *             of 128.
+ *             float32 on the tensor cores; requires d == 128; tiles of 128.
  *   LCA_FP32: every tensor float32, exact float32 arithmetic on CUDA cores;
- *             d in {64, 128}, S a multiple of 64.
+ *             d in {64, 128}; tiles of 64.
+ *   Any S >= 1: when S is not a multiple of the tile the last tile is
+ *   partial (ragged); S2-Attn needs S to be a multiple of its group.
  *
  * Ownership and memory
  *   The caller allocates every device buffer (inputs, outputs, workspace)
@@ -98,7 +99,8 @@ typedef struct {
 
 /* ---------------------------------------------------------------------------
  * lca_attn_fwd -- exact attention forward over key/value chunks.
- *   The keys are split into S / kv_chunk chunks (kv_chunk == 0: one chunk).
+ *   The keys are split into ceil(S / kv_chunk) chunks (kv_chunk == 0: one
+ *   chunk; the last chunk may be partial).
  *   Each query tile attends to the chunks in the order opts selects; the
  *   partial (O, lse) of every chunk is folded into the running result in
  *   unnormalised form (running max m, running sum l, running O*l), which is
@@ -107,8 +109,8 @@ typedef struct {
  *   q, k, v: inputs (layouts above).  out: [B,S,Hq,d] output, same dtype.
  *   lse: [B,Hq,S] float32 output.  opts may be NULL (in-order).
  *   Errors: LCA_ERR_INVALID_ARG when a pointer is NULL or misaligned, a
- *   dimension is <= 0, Hq % Hkv != 0, kv_chunk is not a multiple of the tile
- *   or does not divide S, the chunk count exceeds LCA_MAX_CHUNKS, or the
+ *   dimension is <= 0, Hq % Hkv != 0, kv_chunk is not a multiple of the
+ *   tile, the chunk count exceeds LCA_MAX_CHUNKS, or the
  *   permutation is invalid; LCA_ERR_UNSUPPORTED for shapes outside the
  *   element-type limits above.
  * ------------------------------------------------------------------------- */
@@ -118,8 +120,9 @@ LCA_API lca_status lca_attn_fwd(const lca_shape* shape, const void* q, const voi
                         void* stream);
 
 /* Bytes of device workspace lca_attn_bwd / lca_s2attn_bwd need: float32
- * rows D_i = dout_i . out_i ([B,Hq,S]) and, for bf16, a float32 dq
- * accumulator ([B,S,Hq,d]).  Returns 0 for an invalid shape. */
+ * rows D_i = dout_i . out_i and a copy of lse, each [B,Hq,S rounded up to
+ * the tile], and, for bf16, a float32 dq accumulator ([B,S,Hq,d]).  Returns
+ * 0 for an invalid shape. */
 LCA_API size_t lca_attn_bwd_workspace_size(const lca_shape* shape);
 
 /* ---------------------------------------------------------------------------

@@ -1,7 +1,8 @@
 // aux_kernels.cuh -- small memory-bound kernels around the attention passes.
 //
 //   bwd_rowdot   D_i = sum_c dout_ic * out_ic (float32), the row term of
-//                dS = P o (dP - D) in the backward pass
+//                dS = P o (dP - D) in the backward pass, plus a copy of lse,
+//                both into rows padded to whole tiles
 //   dq_finalize  dq = scale * dq_acc, float32 accumulator -> bf16
 //   lse_merge    combine two partial (O, lse) results over disjoint key
 //                sets (Ring Attention with Blockwise Transformers, Summary:
@@ -13,10 +14,13 @@
 
 namespace lca {
 
-// One warp per (token, head) row; rows ordered [B, S, H]; D written [B, H, S].
+// One warp per (token, head) row; rows ordered [B, S, H].  Writes D and a
+// copy of lse into [B, H, S_pad] arrays whose entries past S stay as the
+// caller zeroed them.
 template <typename T, int D>
 __global__ void bwd_rowdot(const T* __restrict__ out, const T* __restrict__ dout,
-                           float* __restrict__ Dst, int B, int S, int H) {
+                           const float* __restrict__ lse, float* __restrict__ Dst,
+                           float* __restrict__ lse_pad, int B, int S, int S_pad, int H) {
   const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int64_t nrows = static_cast<int64_t>(B) * S * H;
@@ -43,7 +47,9 @@ __global__ void bwd_rowdot(const T* __restrict__ out, const T* __restrict__ dout
     const int64_t bs = row / H;
     const int s = static_cast<int>(bs % S);
     const int b = static_cast<int>(bs / S);
-    Dst[(static_cast<int64_t>(b) * H + h) * S + s] = acc;
+    const int64_t bh = static_cast<int64_t>(b) * H + h;
+    Dst[bh * S_pad + s] = acc;
+    lse_pad[bh * S_pad + s] = lse[bh * S + s];
   }
 }
 

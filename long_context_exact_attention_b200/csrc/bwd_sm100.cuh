@@ -9,6 +9,10 @@
 //   dV  += P^T dO                 dK  += dS^T Q          (TMEM accumulators)
 //   dQ^T = K^T dS^T -> added into the fp32 dq accumulator by TMA bulk
 //                      reduce-add (scale applied later)
+// Ragged S: rows past S of the last tile load as zeros (Q, K, V, dO by TMA;
+// lse and D from copies padded with zeros), which makes their
+// contributions to dK, dV and dQ vanish; stores and reduce-adds past S are
+// dropped.
 //
 // One CTA per (key tile of 128, key/value head, batch); it loops over the
 // query heads of its grouped-query group and over the query tiles that can
@@ -89,11 +93,12 @@ constexpr uint32_t kIdescMM = idesc_bf16_f32(128, 128, true, true);    // dQ^T
 
 struct Args {
   int B, Hq, Hkv, S;
+  int S_pad;             // row length of the padded lse / D copies
   float scale;
   float scale_log2;
   unsigned long long budget;
-  const float* lse;      // [B,Hq,S]
-  const float* Drow;     // [B,Hq,S]
+  const float* lse;      // [B,Hq,S_pad], zero past S
+  const float* Drow;     // [B,Hq,S_pad], zero past S
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   AttnSched sched;
@@ -178,7 +183,6 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   WaitCtl wc{abort_flag, a.budget};
-  const int row0 = b * a.S;
 
   if (wg == 0) {
     regs_dec<kRegsCtl>();
@@ -189,10 +193,10 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmDO);
       mbar_expect_tx(bar(B_KV), 2 * kTileB);
-      tma_load_3d(sK, &tmK, bar(B_KV), 0, g, row0 + ktok0);
-      tma_load_3d(sK + kHalf, &tmK, bar(B_KV), 64, g, row0 + ktok0);
-      tma_load_3d(sV, &tmV, bar(B_KV), 0, g, row0 + ktok0);
-      tma_load_3d(sV + kHalf, &tmV, bar(B_KV), 64, g, row0 + ktok0);
+      tma_load_4d(sK, &tmK, bar(B_KV), 0, g, ktok0, b);
+      tma_load_4d(sK + kHalf, &tmK, bar(B_KV), 64, g, ktok0, b);
+      tma_load_4d(sV, &tmV, bar(B_KV), 0, g, ktok0, b);
+      tma_load_4d(sV + kHalf, &tmV, bar(B_KV), 64, g, ktok0, b);
       bool ok = true;
       int issued0 = 0, issued1 = 0, o_issued = 0;
       for (int i = 0; i < nsteps && ok; ++i) {
@@ -204,17 +208,17 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         if (!ok) break;
         const uint32_t fb = bar(B_QFULL + st);
         mbar_expect_tx(fb, kTileB + 1024);
-        tma_load_3d(sQ + st * kTileB, &tmQ, fb, 0, h, row0 + qtok0);
-        tma_load_3d(sQ + st * kTileB + kHalf, &tmQ, fb, 64, h, row0 + qtok0);
-        const size_t ro = (static_cast<size_t>(b) * a.Hq + h) * a.S + qtok0;
+        tma_load_4d(sQ + st * kTileB, &tmQ, fb, 0, h, qtok0, b);
+        tma_load_4d(sQ + st * kTileB + kHalf, &tmQ, fb, 64, h, qtok0, b);
+        const size_t ro = (static_cast<size_t>(b) * a.Hq + h) * a.S_pad + qtok0;
         bulk_load(sL + st * 512, a.lse + ro, 512, fb);
         bulk_load(sD + st * 512, a.Drow + ro, 512, fb);
         if (st) ++issued1; else ++issued0;
         if (i >= 1) ok = wait_bar(bar(B_OEMPTY), (i - 1) & 1, wc, 112);
         if (!ok) break;
         mbar_expect_tx(bar(B_OFULL), kTileB);
-        tma_load_3d(sO, &tmDO, bar(B_OFULL), 0, h, row0 + qtok0);
-        tma_load_3d(sO + kHalf, &tmDO, bar(B_OFULL), 64, h, row0 + qtok0);
+        tma_load_4d(sO, &tmDO, bar(B_OFULL), 0, h, qtok0, b);
+        tma_load_4d(sO + kHalf, &tmDO, bar(B_OFULL), 64, h, qtok0, b);
         ++o_issued;
       }
       if (!ok) {
@@ -381,21 +385,28 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     // ---- dK = scale * acc -> bf16 (columns split between the two halves)
     if (ok) ok = wait_bar(bar(B_DONE), 0, wc, 315);
     ok = __all_sync(0xffffffffu, ok);
+    // every lane takes part in the TMEM loads (warp-collective); key rows
+    // past S (ragged last tile) only skip their stores
+    const bool row_in = ktok0 + r < a.S;
     if (ok) {
       tc_fence_after();
-      __nv_bfloat16* row = a.dk + ((static_cast<size_t>(b) * a.S + ktok0 + r) * a.Hkv + g) * kD;
+      __nv_bfloat16* row =
+          a.dk + ((static_cast<size_t>(b) * a.S + (row_in ? ktok0 + r : 0)) * a.Hkv + g) * kD;
 #pragma unroll 1
       for (int cc = 2 * hq; cc < 2 * hq + 2; ++cc) {
         float o[32];
+        __syncwarp();
         tmem_ld32(tmem + lad + 384 + cc * 32, o);
+        if (row_in) {
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          uint4 pk;
-          pk.x = pack_bf16x2(o[v * 8 + 0] * a.scale, o[v * 8 + 1] * a.scale);
-          pk.y = pack_bf16x2(o[v * 8 + 2] * a.scale, o[v * 8 + 3] * a.scale);
-          pk.z = pack_bf16x2(o[v * 8 + 4] * a.scale, o[v * 8 + 5] * a.scale);
-          pk.w = pack_bf16x2(o[v * 8 + 6] * a.scale, o[v * 8 + 7] * a.scale);
-          *reinterpret_cast<uint4*>(row + cc * 32 + v * 8) = pk;
+          for (int v = 0; v < 4; ++v) {
+            uint4 pk;
+            pk.x = pack_bf16x2(o[v * 8 + 0] * a.scale, o[v * 8 + 1] * a.scale);
+            pk.y = pack_bf16x2(o[v * 8 + 2] * a.scale, o[v * 8 + 3] * a.scale);
+            pk.z = pack_bf16x2(o[v * 8 + 4] * a.scale, o[v * 8 + 5] * a.scale);
+            pk.w = pack_bf16x2(o[v * 8 + 6] * a.scale, o[v * 8 + 7] * a.scale);
+            *reinterpret_cast<uint4*>(row + cc * 32 + v * 8) = pk;
+          }
         }
       }
     }
@@ -435,7 +446,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         fence_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_reduce_add_3d(&tmDQ, sR + wq * 8192, wq * 32, h, row0 + qtok0 + half * 64);
+          tma_reduce_add_4d(&tmDQ, sR + wq * 8192, wq * 32, h, qtok0 + half * 64, b);
           bulk_commit();
         }
       }
@@ -445,21 +456,26 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     // ---- dV -> bf16
     if (ok) ok = wait_bar(bar(B_DONE), 0, wc, 412);
     ok = __all_sync(0xffffffffu, ok);
+    const bool row_in = ktok0 + r < a.S;
     if (ok) {
       tc_fence_after();
-      __nv_bfloat16* row = a.dv + ((static_cast<size_t>(b) * a.S + ktok0 + r) * a.Hkv + g) * kD;
+      __nv_bfloat16* row =
+          a.dv + ((static_cast<size_t>(b) * a.S + (row_in ? ktok0 + r : 0)) * a.Hkv + g) * kD;
 #pragma unroll 1
       for (int cc = 0; cc < 4; ++cc) {
         float o[32];
+        __syncwarp();
         tmem_ld32(tmem + lad + 256 + cc * 32, o);
+        if (row_in) {
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          uint4 pk;
-          pk.x = pack_bf16x2(o[v * 8 + 0], o[v * 8 + 1]);
-          pk.y = pack_bf16x2(o[v * 8 + 2], o[v * 8 + 3]);
-          pk.z = pack_bf16x2(o[v * 8 + 4], o[v * 8 + 5]);
-          pk.w = pack_bf16x2(o[v * 8 + 6], o[v * 8 + 7]);
-          *reinterpret_cast<uint4*>(row + cc * 32 + v * 8) = pk;
+          for (int v = 0; v < 4; ++v) {
+            uint4 pk;
+            pk.x = pack_bf16x2(o[v * 8 + 0], o[v * 8 + 1]);
+            pk.y = pack_bf16x2(o[v * 8 + 2], o[v * 8 + 3]);
+            pk.z = pack_bf16x2(o[v * 8 + 4], o[v * 8 + 5]);
+            pk.w = pack_bf16x2(o[v * 8 + 6], o[v * 8 + 7]);
+            *reinterpret_cast<uint4*>(row + cc * 32 + v * 8) = pk;
+          }
         }
       }
     }

@@ -143,12 +143,11 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      const int row0 = b * a.S;
       mbar_expect_tx(bar(B_Q), has1 ? 2 * kTileB : kTileB);
       for (int t = 0; t < (has1 ? 2 : 1); ++t) {
-        const int tok = row0 + token_tile(sc, qt0 + t, shifted) * kTile;
-        tma_load_3d(sQ + t * kTileB, &tmQ, bar(B_Q), 0, h, tok);
-        tma_load_3d(sQ + t * kTileB + kHalf, &tmQ, bar(B_Q), 64, h, tok);
+        const int tok = token_tile(sc, qt0 + t, shifted) * kTile;
+        tma_load_4d(sQ + t * kTileB, &tmQ, bar(B_Q), 0, h, tok, b);
+        tma_load_4d(sQ + t * kTileB + kHalf, &tmQ, bar(B_Q), 64, h, tok, b);
       }
       KvWalk w;
       w.init(&sc, qt_last);
@@ -157,18 +156,18 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       bool ok = true;
       while (ok && w.next(t)) {
         const int st = j & 1;
-        const int tok = row0 + token_tile(sc, t, shifted) * kTile;
+        const int tok = token_tile(sc, t, shifted) * kTile;
         if (j >= 2) ok = wait_bar(bar(B_KEMPTY + st), ((j - 2) >> 1) & 1, wc, 101);
         if (!ok) break;
         mbar_expect_tx(bar(B_KFULL + st), kTileB);
-        tma_load_3d(sK + st * kTileB, &tmK, bar(B_KFULL + st), 0, g, tok);
-        tma_load_3d(sK + st * kTileB + kHalf, &tmK, bar(B_KFULL + st), 64, g, tok);
+        tma_load_4d(sK + st * kTileB, &tmK, bar(B_KFULL + st), 0, g, tok, b);
+        tma_load_4d(sK + st * kTileB + kHalf, &tmK, bar(B_KFULL + st), 64, g, tok, b);
         if (st) ++k_issued1; else ++k_issued0;
         if (j >= 2) ok = wait_bar(bar(B_VEMPTY + st), ((j - 2) >> 1) & 1, wc, 102);
         if (!ok) break;
         mbar_expect_tx(bar(B_VFULL + st), kTileB);
-        tma_load_3d(sV + st * kTileB, &tmV, bar(B_VFULL + st), 0, g, tok);
-        tma_load_3d(sV + st * kTileB + kHalf, &tmV, bar(B_VFULL + st), 64, g, tok);
+        tma_load_4d(sV + st * kTileB, &tmV, bar(B_VFULL + st), 0, g, tok, b);
+        tma_load_4d(sV + st * kTileB + kHalf, &tmV, bar(B_VFULL + st), 64, g, tok, b);
         if (st) ++v_issued1; else ++v_issued0;
         ++j;
       }
@@ -277,6 +276,16 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 128; ++i)
             if (i > r) s[i] = -INFINITY;
+        } else {
+          // last key tile of a ragged sequence: keys past S are zero-filled
+          // rows, masked here (on the diagonal the causal mask covers them
+          // for every stored row)
+          const int kv_valid = sc.S - token_tile(sc, t, shifted) * kTile;
+          if (kv_valid < kTile) {
+#pragma unroll
+            for (int i = 0; i < 128; ++i)
+              if (i >= kv_valid) s[i] = -INFINITY;
+          }
         }
         // Row max: eight independent chains of 3-input max.
         float mx8[8];
@@ -342,28 +351,34 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       if (ok && cnt >= 1) ok = wait_bar(bar(B_OREADY + tq), (cnt - 1) & 1, wc, 303);
       ok = __all_sync(0xffffffffu, ok && cnt >= 1);
       const int tok = token_tile(sc, qt, shifted) * kTile + r;
+      // Every lane takes part in the TMEM loads (warp-collective); rows past
+      // S (ragged last tile) only skip their stores.
+      const bool row_in = tok < sc.S;
       if (ok) {
         tc_fence_after();
         const float inv = (l_run > 0.f) ? 1.0f / l_run : 0.f;
         __nv_bfloat16* orow =
-            a.out + ((static_cast<size_t>(b) * a.S + tok) * a.Hq + h) * kD;
+            a.out + ((static_cast<size_t>(b) * a.S + (row_in ? tok : 0)) * a.Hq + h) * kD;
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           float o[32];
+          __syncwarp();
           tmem_ld32(tO + q4 * 32, o);
+          if (row_in) {
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 pk;
-            pk.x = pack_bf16x2(o[v * 8 + 0] * inv, o[v * 8 + 1] * inv);
-            pk.y = pack_bf16x2(o[v * 8 + 2] * inv, o[v * 8 + 3] * inv);
-            pk.z = pack_bf16x2(o[v * 8 + 4] * inv, o[v * 8 + 5] * inv);
-            pk.w = pack_bf16x2(o[v * 8 + 6] * inv, o[v * 8 + 7] * inv);
-            *reinterpret_cast<uint4*>(orow + q4 * 32 + v * 8) = pk;
+            for (int v = 0; v < 4; ++v) {
+              uint4 pk;
+              pk.x = pack_bf16x2(o[v * 8 + 0] * inv, o[v * 8 + 1] * inv);
+              pk.y = pack_bf16x2(o[v * 8 + 2] * inv, o[v * 8 + 3] * inv);
+              pk.z = pack_bf16x2(o[v * 8 + 4] * inv, o[v * 8 + 5] * inv);
+              pk.w = pack_bf16x2(o[v * 8 + 6] * inv, o[v * 8 + 7] * inv);
+              *reinterpret_cast<uint4*>(orow + q4 * 32 + v * 8) = pk;
+            }
           }
         }
         const float lse = (l_run > 0.f) ? (m_run + lg2_approx(l_run)) * 0.69314718055994531f
                                         : -INFINITY;
-        a.lse[(static_cast<size_t>(b) * a.Hq + h) * a.S + tok] = lse;
+        if (row_in) a.lse[(static_cast<size_t>(b) * a.Hq + h) * a.S + tok] = lse;
       }
     }
   }

@@ -49,6 +49,9 @@ struct Common {
   int tile;
 };
 
+// S rounded up to the tile of the element type's path.
+int s_pad_of(const Common& c) { return (c.S + c.tile - 1) / c.tile * c.tile; }
+
 lca_status check_shape(const lca_shape* sh, Common* c) {
   if (!sh) return fail(LCA_ERR_INVALID_ARG, "shape is NULL");
   if (sh->B <= 0 || sh->Hq <= 0 || sh->Hkv <= 0 || sh->S <= 0 || sh->d <= 0)
@@ -78,8 +81,6 @@ lca_status check_shape(const lca_shape* sh, Common* c) {
       return fail(LCA_ERR_UNSUPPORTED, "fp32 path needs d in {64, 128}");
     c->tile = 64;
   }
-  if (sh->S % c->tile)
-    return fail(LCA_ERR_UNSUPPORTED, "S must be a multiple of %d", c->tile);
   return LCA_OK;
 }
 
@@ -97,13 +98,14 @@ lca_status check_ptrs(std::initializer_list<const void*> ps) {
 lca_status make_chunk_sched(const Common& c, int causal, int64_t kv_chunk, const lca_opts* o,
                             AttnSched* s) {
   std::memset(s, 0, sizeof *s);
-  s->n_tiles = c.S / c.tile;
+  s->S = c.S;
+  s->n_tiles = (c.S + c.tile - 1) / c.tile;
   s->causal = causal ? 1 : 0;
-  const int64_t chunk = kv_chunk == 0 ? c.S : kv_chunk;
-  if (chunk < 0 || chunk % c.tile || c.S % chunk)
-    return fail(LCA_ERR_INVALID_ARG, "kv_chunk must be a multiple of %d dividing S", c.tile);
+  if (kv_chunk < 0 || kv_chunk % c.tile)
+    return fail(LCA_ERR_INVALID_ARG, "kv_chunk must be a non-negative multiple of %d", c.tile);
+  const int64_t chunk = kv_chunk == 0 ? static_cast<int64_t>(s->n_tiles) * c.tile : kv_chunk;
   s->tiles_per_chunk = static_cast<int>(chunk / c.tile);
-  s->n_chunks = static_cast<int>(c.S / chunk);
+  s->n_chunks = static_cast<int>((s->n_tiles + s->tiles_per_chunk - 1) / s->tiles_per_chunk);
   if (s->n_chunks > LCA_MAX_CHUNKS)
     return fail(LCA_ERR_INVALID_ARG, "%d chunks exceed LCA_MAX_CHUNKS", s->n_chunks);
   s->order = o ? o->order : LCA_ORDER_INORDER;
@@ -138,6 +140,7 @@ lca_status make_s2_sched(const Common& c, int causal, int64_t group, int64_t shi
   const int rep = c.Hq / c.Hkv;
   if ((c.Hq - shift_heads) % rep)
     return fail(LCA_ERR_INVALID_ARG, "shifted heads must cover whole grouped-query groups");
+  s->S = c.S;
   s->n_tiles = c.S / c.tile;
   s->causal = causal ? 1 : 0;
   s->s2 = 1;
@@ -170,16 +173,19 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [tokens][heads][128] bf16 viewed 3-D; box = 64 head dims x 1 head x 128 tokens.
-lca_status make_map(CUtensorMap* m, const void* ptr, int64_t tokens, int64_t heads) {
+// [B][S][heads][128] bf16 viewed 4-D (head dim, head, token, batch); box =
+// 64 head dims x 1 head x 128 tokens x 1 batch.  Token rows past S (ragged
+// last tile) load as zeros.
+lca_status make_map(CUtensorMap* m, const void* ptr, int64_t B, int64_t S, int64_t heads) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(LCA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-  const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(heads),
-                              static_cast<cuuint64_t>(tokens)};
-  const cuuint64_t strides[2] = {128 * 2, static_cast<cuuint64_t>(heads) * 128 * 2};
-  const cuuint32_t box[3] = {64, 1, 128};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
+  const cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(heads), static_cast<cuuint64_t>(S),
+                              static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {128 * 2, static_cast<cuuint64_t>(heads) * 128 * 2,
+                                 static_cast<cuuint64_t>(S) * heads * 128 * 2};
+  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims,
                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -187,17 +193,19 @@ lca_status make_map(CUtensorMap* m, const void* ptr, int64_t tokens, int64_t hea
   return LCA_OK;
 }
 
-// fp32 [tokens][heads][128] accumulator viewed 3-D; box = 32 head dims x 1
-// head x 64 tokens, no swizzle (the box's rows are 128 bytes).
-lca_status make_map_acc(CUtensorMap* m, const void* ptr, int64_t tokens, int64_t heads) {
+// fp32 [B][S][heads][128] accumulator viewed 4-D; box = 32 head dims x 1
+// head x 64 tokens x 1 batch, no swizzle (the box's rows are 128 bytes);
+// reduce-adds of rows past S are dropped.
+lca_status make_map_acc(CUtensorMap* m, const void* ptr, int64_t B, int64_t S, int64_t heads) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(LCA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-  const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(heads),
-                              static_cast<cuuint64_t>(tokens)};
-  const cuuint64_t strides[2] = {128 * 4, static_cast<cuuint64_t>(heads) * 128 * 4};
-  const cuuint32_t box[3] = {32, 1, 64};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims,
+  const cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(heads), static_cast<cuuint64_t>(S),
+                              static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {128 * 4, static_cast<cuuint64_t>(heads) * 128 * 4,
+                                 static_cast<cuuint64_t>(S) * heads * 128 * 4};
+  const cuuint32_t box[4] = {32, 1, 64, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(ptr), dims,
                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -257,16 +265,15 @@ unsigned long long budget_of(const lca_opts* o) {
 lca_status run_fwd(const Common& c, const AttnSched& s, const void* q, const void* k,
                    const void* v, void* out, float* lse, unsigned long long budget,
                    cudaStream_t st) {
-  const int64_t tokens = static_cast<int64_t>(c.B) * c.S;
   const unsigned grid = static_cast<unsigned>(s.n_tiles) * c.B * c.Hq;
   if (c.dtype == LCA_BF16) {
     // one CTA per pair of 128-row query tiles
     const unsigned grid2 = static_cast<unsigned>((s.n_tiles + 1) / 2) * c.B * c.Hq;
     CUtensorMap mq, mk, mv;
     lca_status r;
-    if ((r = make_map(&mq, q, tokens, c.Hq)) != LCA_OK) return r;
-    if ((r = make_map(&mk, k, tokens, c.Hkv)) != LCA_OK) return r;
-    if ((r = make_map(&mv, v, tokens, c.Hkv)) != LCA_OK) return r;
+    if ((r = make_map(&mq, q, c.B, c.S, c.Hq)) != LCA_OK) return r;
+    if ((r = make_map(&mk, k, c.B, c.S, c.Hkv)) != LCA_OK) return r;
+    if ((r = make_map(&mv, v, c.B, c.S, c.Hkv)) != LCA_OK) return r;
     if ((r = ensure_smem(attn_fwd_bf16_sm100, fwd::kSmemBytes, 0)) != LCA_OK) return r;
     fwd::Args a;
     a.B = c.B;
@@ -291,6 +298,7 @@ lca_status run_fwd(const Common& c, const AttnSched& s, const void* q, const voi
   a.Hq = c.Hq;
   a.Hkv = c.Hkv;
   a.S = c.S;
+  a.S_pad = s_pad_of(c);
   a.scale = c.scale;
   a.sched = s;
   lca_status r;
@@ -305,12 +313,14 @@ lca_status run_fwd(const Common& c, const AttnSched& s, const void* q, const voi
 }
 
 // ---------------------------------------------------------------- backward
+// Workspace: D rows and a copy of lse, each [B][Hq][S_pad] with S_pad = S
+// rounded up to the tile (zero past S), then (bf16) the fp32 dq accumulator.
 size_t ws_d_bytes(const Common& c) {
-  const size_t n = static_cast<size_t>(c.B) * c.Hq * c.S * sizeof(float);
+  const size_t n = static_cast<size_t>(c.B) * c.Hq * s_pad_of(c) * sizeof(float);
   return (n + 255) & ~static_cast<size_t>(255);
 }
 size_t ws_bytes_of(const Common& c) {
-  size_t n = ws_d_bytes(c);
+  size_t n = 2 * ws_d_bytes(c);
   if (c.dtype == LCA_BF16) n += static_cast<size_t>(c.B) * c.S * c.Hq * c.d * sizeof(float);
   return n;
 }
@@ -324,27 +334,34 @@ lca_status run_bwd(const Common& c, const AttnSched& s, const void* q, const voi
     return fail(LCA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes,
                 ws_bytes_of(c));
   if (!aligned16(ws)) return fail(LCA_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+  const int S_pad = s_pad_of(c);
   float* Drow = static_cast<float*>(ws);
+  float* lse_pad = reinterpret_cast<float*>(static_cast<char*>(ws) + ws_d_bytes(c));
   const int64_t rows = static_cast<int64_t>(c.B) * c.S * c.Hq;
   const unsigned rd_blocks = static_cast<unsigned>((rows * 32 + 255) / 256);
   const unsigned grid = static_cast<unsigned>(s.n_tiles) * c.B * c.Hkv;
+  cudaError_t e;
+  if (S_pad != c.S) {
+    // entries past S must read as zeros
+    e = cudaMemsetAsync(ws, 0, 2 * ws_d_bytes(c), st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(padded rows)");
+  }
+  lca_status r;
   if (c.dtype == LCA_BF16) {
-    float* acc = reinterpret_cast<float*>(static_cast<char*>(ws) + ws_d_bytes(c));
+    float* acc = reinterpret_cast<float*>(static_cast<char*>(ws) + 2 * ws_d_bytes(c));
     const size_t acc_bytes = static_cast<size_t>(rows) * c.d * sizeof(float);
-    cudaError_t e = cudaMemsetAsync(acc, 0, acc_bytes, st);
+    e = cudaMemsetAsync(acc, 0, acc_bytes, st);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(dq accumulator)");
     bwd_rowdot<__nv_bfloat16, 128><<<rd_blocks, 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), Drow,
-        c.B, c.S, c.Hq);
-    lca_status r = launched("bwd_rowdot");
-    if (r != LCA_OK) return r;
-    const int64_t tokens = static_cast<int64_t>(c.B) * c.S;
+        static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse,
+        Drow, lse_pad, c.B, c.S, S_pad, c.Hq);
+    if ((r = launched("bwd_rowdot")) != LCA_OK) return r;
     CUtensorMap mq, mk, mv, mdo, mdq;
-    if ((r = make_map(&mq, q, tokens, c.Hq)) != LCA_OK) return r;
-    if ((r = make_map(&mk, k, tokens, c.Hkv)) != LCA_OK) return r;
-    if ((r = make_map(&mv, v, tokens, c.Hkv)) != LCA_OK) return r;
-    if ((r = make_map(&mdo, dout, tokens, c.Hq)) != LCA_OK) return r;
-    if ((r = make_map_acc(&mdq, acc, tokens, c.Hq)) != LCA_OK) return r;
+    if ((r = make_map(&mq, q, c.B, c.S, c.Hq)) != LCA_OK) return r;
+    if ((r = make_map(&mk, k, c.B, c.S, c.Hkv)) != LCA_OK) return r;
+    if ((r = make_map(&mv, v, c.B, c.S, c.Hkv)) != LCA_OK) return r;
+    if ((r = make_map(&mdo, dout, c.B, c.S, c.Hq)) != LCA_OK) return r;
+    if ((r = make_map_acc(&mdq, acc, c.B, c.S, c.Hq)) != LCA_OK) return r;
     if ((r = check_bwd_regs()) != LCA_OK) return r;
     if ((r = ensure_smem(attn_bwd_bf16_sm100, bwd::kSmemBytes, 3)) != LCA_OK) return r;
     bwd::Args a;
@@ -352,10 +369,11 @@ lca_status run_bwd(const Common& c, const AttnSched& s, const void* q, const voi
     a.Hq = c.Hq;
     a.Hkv = c.Hkv;
     a.S = c.S;
+    a.S_pad = S_pad;
     a.scale = c.scale;
     a.scale_log2 = c.scale * 1.4426950408889634f;
     a.budget = budget;
-    a.lse = lse;
+    a.lse = lse_pad;
     a.Drow = Drow;
     a.dk = static_cast<__nv_bfloat16*>(dk);
     a.dv = static_cast<__nv_bfloat16*>(dv);
@@ -368,24 +386,23 @@ lca_status run_bwd(const Common& c, const AttnSched& s, const void* q, const voi
     return launched("dq_finalize");
   }
   // fp32
-  cudaError_t e = cudaMemsetAsync(dq, 0, static_cast<size_t>(rows) * c.d * sizeof(float), st);
+  e = cudaMemsetAsync(dq, 0, static_cast<size_t>(rows) * c.d * sizeof(float), st);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(dq)");
   if (c.d == 64)
     bwd_rowdot<float, 64><<<rd_blocks, 256, 0, st>>>(static_cast<const float*>(out),
-                                                       static_cast<const float*>(dout), Drow,
-                                                       c.B, c.S, c.Hq);
+                                                       static_cast<const float*>(dout), lse, Drow,
+                                                       lse_pad, c.B, c.S, S_pad, c.Hq);
   else
     bwd_rowdot<float, 128><<<rd_blocks, 256, 0, st>>>(static_cast<const float*>(out),
-                                                        static_cast<const float*>(dout), Drow,
-                                                        c.B, c.S, c.Hq);
-  lca_status r = launched("bwd_rowdot");
-  if (r != LCA_OK) return r;
+                                                        static_cast<const float*>(dout), lse,
+                                                        Drow, lse_pad, c.B, c.S, S_pad, c.Hq);
+  if ((r = launched("bwd_rowdot")) != LCA_OK) return r;
   f32::Args a{};
   a.q = static_cast<const float*>(q);
   a.k = static_cast<const float*>(k);
   a.v = static_cast<const float*>(v);
   a.out = static_cast<const float*>(out);
-  a.lse = lse;
+  a.lse = lse_pad;
   a.dout = static_cast<const float*>(dout);
   a.D = Drow;
   a.dq = static_cast<float*>(dq);
@@ -395,6 +412,7 @@ lca_status run_bwd(const Common& c, const AttnSched& s, const void* q, const voi
   a.Hq = c.Hq;
   a.Hkv = c.Hkv;
   a.S = c.S;
+  a.S_pad = S_pad;
   a.scale = c.scale;
   a.sched = s;
   if (c.d == 64) {

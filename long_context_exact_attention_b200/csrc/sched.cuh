@@ -7,6 +7,9 @@
 // walk stays inside the query's group and each position tile maps to one
 // contiguous token tile because G/2 is a whole number of tiles.
 //
+// Ragged lengths: when S is not a multiple of the tile, the last tile is
+// partial and the last chunk may hold fewer tiles.
+//
 // Chunk order (Ring Attention with Blockwise Transformers, Summary: a query
 // block meets the key/value blocks in the order the ring delivers them, and
 // the result does not depend on it).  Keys are split into chunks of
@@ -23,7 +26,8 @@
 namespace lca {
 
 struct AttnSched {
-  int n_tiles;             // S / tile
+  int S;                   // sequence length in tokens
+  int n_tiles;             // ceil(S / tile); the last tile may be partial
   int causal;
   int s2;                  // 1: S2-Attn walk
   int tiles_per_chunk;     // chunked walk
@@ -85,6 +89,7 @@ struct KvWalk {
       const int c = chunk_at(ci++);
       t = c * s->tiles_per_chunk;
       t_end = t + s->tiles_per_chunk;
+      if (t_end > s->n_tiles) t_end = s->n_tiles;  // last chunk may be partial
       if (s->causal && t_end > qt + 1) t_end = qt + 1;
     }
     tile = t++;

@@ -10,6 +10,8 @@
 // query heads of its group and the visible query tiles; dK and dV live in
 // registers, dQ is accumulated with shared-memory atomics per query tile and
 // flushed to the float32 dq output with global atomics.
+// Ragged S: rows past S of the last tile load as zeros and are not stored;
+// keys past S are masked in the forward.
 #pragma once
 
 #include "sched.cuh"
@@ -22,9 +24,10 @@ constexpr int kThreads = 256; // 8 warps
 constexpr int kRowsPerWarp = kT / (kThreads / 32);
 
 struct Args {
-  const float *q, *k, *v, *out, *lse, *dout, *D;
+  const float *q, *k, *v, *out, *lse, *dout, *D;  // lse, D: padded [B,Hq,S_pad]
   float *o_out, *lse_out, *dq, *dk, *dv;
   int B, Hq, Hkv, S;
+  int S_pad;
   float scale;
   AttnSched sched;
 };
@@ -60,7 +63,8 @@ __global__ void __launch_bounds__(kThreads) attn_fwd_f32(const __grid_constant__
 
   for (int i = threadIdx.x; i < kT * D; i += kThreads) {
     const int r = i / D, c = i % D;
-    sQ[i] = a.q[((static_cast<size_t>(b) * a.S + qtok0 + r) * a.Hq + h) * D + c];
+    sQ[i] = (qtok0 + r < a.S) ? a.q[((static_cast<size_t>(b) * a.S + qtok0 + r) * a.Hq + h) * D + c]
+                              : 0.f;
   }
   float m[kRowsPerWarp], l[kRowsPerWarp], o[kRowsPerWarp][E];
 #pragma unroll
@@ -78,12 +82,14 @@ __global__ void __launch_bounds__(kThreads) attn_fwd_f32(const __grid_constant__
     __syncthreads();
     for (int i = threadIdx.x; i < kT * D; i += kThreads) {
       const int r = i / D, c = i % D;
+      const bool in = ktok0 + r < a.S;
       const size_t src = ((static_cast<size_t>(b) * a.S + ktok0 + r) * a.Hkv + g) * D + c;
-      sK[r * KP + c] = a.k[src];
-      sV[r * D + c] = a.v[src];
+      sK[r * KP + c] = in ? a.k[src] : 0.f;
+      sV[r * D + c] = in ? a.v[src] : 0.f;
     }
     __syncthreads();
     const bool diag = sc.causal && t == qt;
+    const int kv_valid = a.S - ktok0;  // keys past S (ragged last tile) are masked
 #pragma unroll 1
     for (int rr = 0; rr < kRowsPerWarp; ++rr) {
       const int r = warp * kRowsPerWarp + rr;
@@ -95,8 +101,8 @@ __global__ void __launch_bounds__(kThreads) attn_fwd_f32(const __grid_constant__
       }
       s0 *= a.scale;
       s1 *= a.scale;
-      if (diag && lane > r) s0 = -INFINITY;
-      if (diag && lane + 32 > r) s1 = -INFINITY;
+      if ((diag && lane > r) || lane >= kv_valid) s0 = -INFINITY;
+      if ((diag && lane + 32 > r) || lane + 32 >= kv_valid) s1 = -INFINITY;
       const float mx = warp_max(fmaxf(s0, s1));
       const float m_new = fmaxf(m[rr], mx);
       const float alpha = (m[rr] == -INFINITY) ? 0.f : expf(m[rr] - m_new);
@@ -120,6 +126,7 @@ __global__ void __launch_bounds__(kThreads) attn_fwd_f32(const __grid_constant__
   for (int rr = 0; rr < kRowsPerWarp; ++rr) {
     const int r = warp * kRowsPerWarp + rr;
     const int tok = qtok0 + r;
+    if (tok >= a.S) continue;
     const float inv = l[rr] > 0.f ? 1.f / l[rr] : 0.f;
     float* orow = a.o_out + ((static_cast<size_t>(b) * a.S + tok) * a.Hq + h) * D;
 #pragma unroll
@@ -154,9 +161,10 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_f32(const __grid_constant__
 
   for (int i = threadIdx.x; i < kT * D; i += kThreads) {
     const int r = i / D, c = i % D;
+    const bool in = ktok0 + r < a.S;
     const size_t src = ((static_cast<size_t>(b) * a.S + ktok0 + r) * a.Hkv + g) * D + c;
-    sK[i] = a.k[src];
-    sV[i] = a.v[src];
+    sK[i] = in ? a.k[src] : 0.f;
+    sV[i] = in ? a.v[src] : 0.f;
   }
   float dk[kRowsPerWarp][E], dv[kRowsPerWarp][E];
 #pragma unroll
@@ -173,13 +181,14 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_f32(const __grid_constant__
       __syncthreads();
       for (int i = threadIdx.x; i < kT * D; i += kThreads) {
         const int r = i / D, c = i % D;
+        const bool in = qtok0 + r < a.S;
         const size_t src = ((static_cast<size_t>(b) * a.S + qtok0 + r) * a.Hq + h) * D + c;
-        sQ[r * P + c] = a.q[src];
-        sO[r * P + c] = a.dout[src];
+        sQ[r * P + c] = in ? a.q[src] : 0.f;
+        sO[r * P + c] = in ? a.dout[src] : 0.f;
         sdQ[i] = 0.f;
       }
       for (int i = threadIdx.x; i < kT; i += kThreads) {
-        const size_t ri = (static_cast<size_t>(b) * a.Hq + h) * a.S + qtok0 + i;
+        const size_t ri = (static_cast<size_t>(b) * a.Hq + h) * a.S_pad + qtok0 + i;
         sL[i] = a.lse[ri];
         sD[i] = a.D[ri];
       }
@@ -226,13 +235,16 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_f32(const __grid_constant__
       __syncthreads();
       for (int i = threadIdx.x; i < kT * D; i += kThreads) {
         const int r = i / D, c = i % D;
-        atomicAdd(&a.dq[((static_cast<size_t>(b) * a.S + qtok0 + r) * a.Hq + h) * D + c], sdQ[i]);
+        if (qtok0 + r < a.S)
+          atomicAdd(&a.dq[((static_cast<size_t>(b) * a.S + qtok0 + r) * a.Hq + h) * D + c],
+                    sdQ[i]);
       }
     }
   }
 #pragma unroll
   for (int rr = 0; rr < kRowsPerWarp; ++rr) {
     const int j = warp * kRowsPerWarp + rr;
+    if (ktok0 + j >= a.S) continue;
     const size_t dst = ((static_cast<size_t>(b) * a.S + ktok0 + j) * a.Hkv + g) * D;
 #pragma unroll
     for (int e = 0; e < E; ++e) {

@@ -54,8 +54,7 @@ def fwd(sh, kv_chunk=0, opts=None, ptrs=None):
 
 @pytest.mark.parametrize("kw,code", [
     (dict(B=0), 1), (dict(Hq=3, Hkv=2), 1), (dict(d=64), 2), (dict(d=96, dtype=1), 2),
-    (dict(S=200), 2), (dict(S=96, dtype=1, d=64), 2), (dict(dtype=7), 1),
-    (dict(scale=-1.0), 1),
+    (dict(S=0), 1), (dict(dtype=7), 1), (dict(scale=-1.0), 1),
 ])
 def test_bad_shapes_rejected(kw, code):
     assert fwd(shape(**kw)) == code
@@ -69,8 +68,10 @@ def test_bad_pointers_rejected():
     assert b"aligned" in lca.lib().lca_last_error()
 
 
-@pytest.mark.parametrize("kv_chunk", [100, 384, -128])
+@pytest.mark.parametrize("kv_chunk", [100, 200, -128])
 def test_bad_chunks_rejected(kv_chunk):
+    # a chunk must be a whole number of tiles (the last chunk of a sequence
+    # may be partial, so it need not divide S)
     assert fwd(shape(S=512), kv_chunk=kv_chunk) == 1
 
 
@@ -101,7 +102,11 @@ def test_workspace_errors():
     L = lca.lib()
     sh = shape()
     need = L.lca_attn_bwd_workspace_size(ctypes.byref(sh))
-    assert need == 4 * 1 * 4 * 256 + 4 * 256 * 4 * 128
+    # D rows and the lse copy ([B,Hq,S rounded up to the tile]) + fp32 dq
+    assert need == 2 * 4 * 1 * 4 * 256 + 4 * 256 * 4 * 128
+    ragged = shape(S=300)
+    assert L.lca_attn_bwd_workspace_size(ctypes.byref(ragged)) == \
+        2 * 4 * 1 * 4 * 384 + 4 * 300 * 4 * 128
     assert L.lca_attn_bwd_workspace_size(ctypes.byref(shape(B=0))) == 0
     args = [ctypes.byref(sh)] + [FAKE] * 6 + [1] + [FAKE] * 3
     assert L.lca_attn_bwd(*args, None, need, None) == 5

@@ -24,7 +24,7 @@ def probe():
 
     def run(n_tiles, causal, s2=0, tpc=None, n_chunks=1, order=0, qb=None, gt=0, st=0, fsh=0,
             perm=()):
-        tpc = tpc or n_tiles // n_chunks
+        tpc = tpc or -(-n_tiles // n_chunks)
         qb = qb or tpc
         args = [BIN] + [str(a) for a in (n_tiles, causal, s2, tpc, n_chunks, order, qb, gt, st,
                                          fsh)] + [str(p) for p in perm]
@@ -75,6 +75,20 @@ def test_chunk_walks(probe, causal, n_chunks, order, qb, perm):
         for c in chunks:
             ts = [t for t in seq if t // tpc == c]
             assert ts == sorted(ts)
+    for kt, (a, b) in qr.items():
+        assert list(range(a, b)) == [qt for qt in range(n) if kt in walks[qt]]
+
+
+@pytest.mark.parametrize("causal", [0, 1])
+@pytest.mark.parametrize("n,tpc,order,perm", [(10, 4, 0, ()), (10, 4, 1, ()), (7, 3, 2, (2, 0, 1)),
+                                             (5, 8, 0, ())])
+def test_partial_last_chunk(probe, causal, n, tpc, order, perm):
+    n_chunks = -(-n // tpc)
+    walks, qr, _ = probe(n, causal, tpc=tpc, n_chunks=n_chunks, order=order, perm=perm)
+    for qt, seq in walks.items():
+        visible = [t for t in range(n) if (t <= qt or not causal)]
+        assert sorted(seq) == visible, (qt, seq)
+        assert max(seq) < n
     for kt, (a, b) in qr.items():
         assert list(range(a, b)) == [qt for qt in range(n) if kt in walks[qt]]
 
