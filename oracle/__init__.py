@@ -19,6 +19,8 @@ bound memory:
   shift half the heads by half a group, split into groups, attend inside
   each group, shift back (LongLoRA: Efficient Fine-tuning of Long-Context
   Large Language Models, Summary).
+* ``packed``     -- a packed batch of variable-length sequences: each
+  sequence is an independent problem, so the definition applied per slice.
 * ``merge``      -- the (O, lse) combination of partial results over key
   chunks, whose order does not matter (Ring Attention, Summary).
 * ``brute``      -- pure-Python loops on tiny inputs, an independent
@@ -33,10 +35,12 @@ from .attention import (attention_forward, attention_rows, attention_backward,
                         attention_backward_rows, chunked_attention_forward)
 from .s2attn import s2attn_forward, s2attn_backward, s2_token_of_position
 from .merge import lse_merge
+from .packed import packed_attention_forward, packed_attention_backward
 
 __all__ = [
     "attention_forward", "attention_rows", "attention_backward",
     "attention_backward_rows",
     "chunked_attention_forward", "s2attn_forward", "s2attn_backward",
-    "s2_token_of_position", "lse_merge",
+    "s2_token_of_position", "lse_merge", "packed_attention_forward",
+    "packed_attention_backward",
 ]

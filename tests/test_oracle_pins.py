@@ -198,12 +198,13 @@ def test_merge_two_halves_is_softmax_of_union():
 
 
 @pytest.mark.parametrize("causal", [False, True])
-def test_chunk_order_independence(causal):
-    rng = np.random.default_rng(11)
-    S, d, chunk = 24, 4, 6
+@pytest.mark.parametrize("S,chunk", [(24, 6), (23, 5), (10, 7)])
+def test_chunk_order_independence(causal, S, chunk):
+    rng = np.random.default_rng(11 + S + chunk)
+    d = 4
     q, k, v = rand(1, S, 2, d, rng=rng), rand(1, S, 1, d, rng=rng), rand(1, S, 1, d, rng=rng)
     ref_o, ref_l = oracle.attention_forward(q, k, v, causal)
-    n = S // chunk
+    n = -(-S // chunk)
     orders = [list(range(n)), list(reversed(range(n)))] + \
              [list(rng.permutation(n)) for _ in range(4)]
     for order in orders:
@@ -309,6 +310,67 @@ def test_finite_differences_s2(causal):
     _fd_check(lambda a, b, c: oracle.s2attn_forward(a, b, c, G, 1, causal),
               lambda a, b, c, g: oracle.s2attn_backward(a, b, c, g, G, 1, causal),
               [q, k, v], do)
+
+
+# ---------------------------------------------------------------- packed batches
+
+def _segment_visible(cu, causal):
+    """Block-diagonal mask over the whole packed axis: tokens see each other
+    iff they lie in the same sequence (and, causal, the key is not later)."""
+    seg = {}
+    for b, (c0, c1) in enumerate(zip(cu, cu[1:])):
+        for t in range(c0, c1):
+            seg[t] = b
+
+    def vis(i, j):
+        if i not in seg or seg.get(j) != seg[i]:
+            return False
+        return (j <= i) if causal else True
+    return vis
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("cu", [[0, 4, 4, 9, 13], [0, 13], [0, 1, 2, 13], [2, 5, 11]])
+def test_packed_matches_block_diagonal_brute(causal, cu):
+    """Slicing per sequence (oracle.packed) against one masked attention over
+    the packed axis (brute force): a wrong offset, a leak across sequences or
+    a mask counted from the packed axis instead of the sequence fails."""
+    rng = np.random.default_rng(sum(cu) + causal)
+    T, Hq, Hkv, d = 13, 2, 1, 3
+    q, k, v = rand(T, Hq, d, rng=rng), rand(T, Hkv, d, rng=rng), rand(T, Hkv, d, rng=rng)
+    out, lse = oracle.packed_attention_forward(q, k, v, cu, causal)
+    vis = _segment_visible(cu, causal)
+    covered = [t for t in range(T) if cu[0] <= t < cu[-1]]
+    for h in range(Hq):
+        o_b, l_b = brute.attend(as_lists(q[:, h]), as_lists(k[:, h // (Hq // Hkv)]),
+                                as_lists(v[:, h // (Hq // Hkv)]), vis, 1 / math.sqrt(d))
+        np.testing.assert_allclose(out[covered, h], np.array(o_b)[covered], atol=1e-12)
+        np.testing.assert_allclose(lse[h, covered], np.array(l_b)[covered], atol=1e-12)
+    outside = [t for t in range(T) if t not in covered]
+    assert np.isnan(out[outside]).all() and np.isnan(lse[:, outside]).all()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_finite_differences_packed(causal):
+    rng = np.random.default_rng(77 + causal)
+    cu = [0, 3, 3, 7]
+    T, Hq, Hkv, d = 7, 2, 1, 2
+    q, k, v = rand(T, Hq, d, rng=rng), rand(T, Hkv, d, rng=rng), rand(T, Hkv, d, rng=rng)
+    do = rand(T, Hq, d, rng=rng)
+    _fd_check(lambda a, b, c: oracle.packed_attention_forward(a, b, c, cu, causal),
+              lambda a, b, c, g: oracle.packed_attention_backward(a, b, c, g, cu, causal),
+              [q, k, v], do)
+
+
+def test_packed_backward_outside_rows():
+    rng = np.random.default_rng(5)
+    cu = [1, 4, 6]
+    T, H, d = 8, 1, 2
+    q, k, v, do = (rand(T, H, d, rng=rng) for _ in range(4))
+    dq, dk, dv = oracle.packed_attention_backward(q, k, v, do, cu, True)
+    assert (dq[[0, 6, 7]] == 0).all()
+    assert np.isnan(dk[[0, 6, 7]]).all() and np.isnan(dv[[0, 6, 7]]).all()
+    assert np.isfinite(dk[1:6]).all()
 
 
 # ---------------------------------------------------------------- planted mistakes
