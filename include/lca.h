@@ -89,8 +89,11 @@ typedef struct {
 typedef struct {
   int32_t order;              /* lca_order                                   */
   const int32_t* chunk_perm;  /* HOST array of n_chunks entries (CUSTOM only) */
-  int64_t q_block;            /* RING: query-block length, 0 = kv_chunk; must
-                                 be a multiple of the tile (128 bf16, 64 fp32) */
+  int64_t q_block;            /* RING: query-block length in tokens, 0 =
+                                 kv_chunk.  A query tile follows the ring
+                                 position of the block holding its first row;
+                                 the bf16 path walks two query tiles together,
+                                 in the order of the second.                 */
   uint64_t timeout_cycles;    /* per-wait budget in SM clocks; 0 = default
                                  (2^31, about one second)                    */
 } lca_opts;
@@ -99,8 +102,11 @@ typedef struct {
 
 /* ---------------------------------------------------------------------------
  * lca_attn_fwd -- exact attention forward over key/value chunks.
- *   The keys are split into ceil(S / kv_chunk) chunks (kv_chunk == 0: one
- *   chunk; the last chunk may be partial).
+ *   The keys are split into ceil(S / kv_chunk) chunks of kv_chunk keys
+ *   (kv_chunk == 0 or >= S: one chunk; the last chunk may be partial).
+ *   kv_chunk need not be a multiple of the tile: a key tile that straddles
+ *   a chunk boundary is visited once per chunk, each visit masked to that
+ *   chunk's keys.
  *   Each query tile attends to the chunks in the order opts selects; the
  *   partial (O, lse) of every chunk is folded into the running result in
  *   unnormalised form (running max m, running sum l, running O*l), which is
@@ -109,8 +115,8 @@ typedef struct {
  *   q, k, v: inputs (layouts above).  out: [B,S,Hq,d] output, same dtype.
  *   lse: [B,Hq,S] float32 output.  opts may be NULL (in-order).
  *   Errors: LCA_ERR_INVALID_ARG when a pointer is NULL or misaligned, a
- *   dimension is <= 0, Hq % Hkv != 0, kv_chunk is not a multiple of the
- *   tile, the chunk count exceeds LCA_MAX_CHUNKS, or the
+ *   dimension is <= 0, Hq % Hkv != 0, kv_chunk or q_block is negative,
+ *   the chunk count exceeds LCA_MAX_CHUNKS, or the
  *   permutation is invalid; LCA_ERR_UNSUPPORTED for shapes outside the
  *   element-type limits above.
  * ------------------------------------------------------------------------- */
@@ -203,6 +209,49 @@ LCA_API lca_status lca_s2attn_bwd(const lca_shape* shape, const void* q, const v
                           void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Packed variable-length batches.  No counterpart in the pages, which train
+ * on fixed-length sequences; callers that pack documents of different
+ * lengths into one token axis need it ("nearly 1M"-token contexts are not a
+ * multiple of any tile either).
+ *   shape->B is the number of sequences n and shape->S the total number of
+ *   packed tokens T.  Sequence b holds tokens [cu_seqlens[b], cu_seqlens[b+1])
+ *   and attends only to itself (causal by position inside the sequence);
+ *   cu_seqlens is a DEVICE array of n + 1 int32 offsets, nondecreasing, from
+ *   0 up to at most T, and no sequence is longer than max_seqlen (which sets
+ *   the grid and the workspace).  Empty sequences are allowed.
+ *   Layouts: q, out, dout, dq [T, Hq, d]; k, v, dk, dv [T, Hkv, d];
+ *   lse [Hq, T] float32.  Token rows outside every sequence are left
+ *   untouched in out, lse, dk and dv and are set to zero in dq.  The last
+ *   tile of a sequence reads the rows that follow it (the next sequence, or
+ *   rows outside every sequence) and multiplies them by zero, so every row
+ *   of q, k, v and dout below T must hold finite values.
+ *   Chunking and chunk order apply inside each sequence; LCA_ORDER_CUSTOM is
+ *   rejected (sequences have different chunk counts).
+ *   Errors: as the dense calls, plus LCA_ERR_INVALID_ARG for a NULL or
+ *   misaligned cu_seqlens or max_seqlen outside [1, T].  Offsets that are
+ *   out of order, out of range or longer than max_seqlen cannot be checked
+ *   before launch (they live on the device): the kernels skip the affected
+ *   sequence and lca_check() then returns LCA_ERR_INVALID_ARG.
+ * ------------------------------------------------------------------------- */
+LCA_API lca_status lca_attn_fwd_varlen(const lca_shape* shape, const int32_t* cu_seqlens,
+                                       int64_t max_seqlen, const void* q, const void* k,
+                                       const void* v, int causal, int64_t kv_chunk,
+                                       const lca_opts* opts, void* out, float* lse,
+                                       void* stream);
+
+/* Workspace bytes of lca_attn_bwd_varlen: D rows and a copy of lse, each
+ * [n, Hq, max_seqlen rounded up to the tile] float32, and, for bf16, a
+ * float32 dq accumulator [T, Hq, d].  0 for an invalid shape. */
+LCA_API size_t lca_attn_bwd_varlen_workspace_size(const lca_shape* shape, int64_t max_seqlen);
+
+LCA_API lca_status lca_attn_bwd_varlen(const lca_shape* shape, const int32_t* cu_seqlens,
+                                       int64_t max_seqlen, const void* q, const void* k,
+                                       const void* v, const void* out, const float* lse,
+                                       const void* dout, int causal, void* dq, void* dk,
+                                       void* dv, void* workspace, size_t ws_bytes,
+                                       void* stream);
+
+/* ---------------------------------------------------------------------------
  * lca_lse_merge -- combine two partial attention results over disjoint key
  * sets (Ring Attention, Summary: per-block results combine independently of
  * order):  lse = M + ln(e^(lse_a-M) + e^(lse_b-M)), M = max(lse_a, lse_b);
@@ -218,7 +267,8 @@ LCA_API lca_status lca_lse_merge(int64_t rows, int64_t d, const float* o_a,
 
 /* Synchronises `stream`, then reports and clears the device error word of
  * the current device: LCA_ERR_TIMEOUT if a kernel wait ran out since the
- * last check, LCA_ERR_CUDA if the stream holds a CUDA error, else LCA_OK. */
+ * last check, LCA_ERR_INVALID_ARG if a kernel met invalid packed sequence
+ * offsets, LCA_ERR_CUDA if the stream holds a CUDA error, else LCA_OK. */
 LCA_API lca_status lca_check(void* stream);
 
 /* Static description of a status code. */

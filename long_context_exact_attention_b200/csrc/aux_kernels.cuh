@@ -2,7 +2,7 @@
 //
 //   bwd_rowdot   D_i = sum_c dout_ic * out_ic (float32), the row term of
 //                dS = P o (dP - D) in the backward pass, plus a copy of lse,
-//                both into rows padded to whole tiles
+//                both into per-sequence rows padded to whole tiles
 //   dq_finalize  dq = scale * dq_acc, float32 accumulator -> bf16
 //   lse_merge    combine two partial (O, lse) results over disjoint key
 //                sets (Ring Attention with Blockwise Transformers, Summary:
@@ -14,19 +14,44 @@
 
 namespace lca {
 
-// One warp per (token, head) row; rows ordered [B, S, H].  Writes D and a
-// copy of lse into [B, H, S_pad] arrays whose entries past S stay as the
-// caller zeroed them.
+// One warp per padded row (sequence b, position s < S_pad, head h), h
+// fastest so that neighbouring warps read neighbouring memory.  Sequence b
+// occupies tensor rows [b*S, b*S + S) or, packed, [cu[b], cu[b+1]); lse is
+// [B,H,S] or, packed, [H, total].  Writes D and a copy of lse into
+// [B,H,S_pad] arrays; positions past a sequence's end get D = 0 and
+// lse = +inf (P = 0 for those query rows in the backward pass).  Packed
+// offsets that are out of order or out of range make the sequence empty
+// here; the attention kernels report them.
 template <typename T, int D>
 __global__ void bwd_rowdot(const T* __restrict__ out, const T* __restrict__ dout,
                            const float* __restrict__ lse, float* __restrict__ Dst,
-                           float* __restrict__ lse_pad, int B, int S, int S_pad, int H) {
-  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+                           float* __restrict__ lse_pad, int B, int S, int S_pad, int H,
+                           const int* __restrict__ cu_seqlens) {
+  const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  const int64_t nrows = static_cast<int64_t>(B) * S * H;
-  if (row >= nrows) return;
-  const T* o = out + row * D;
-  const T* g = dout + row * D;
+  if (w >= static_cast<int64_t>(B) * S_pad * H) return;
+  const int h = static_cast<int>(w % H);
+  const int s = static_cast<int>((w / H) % S_pad);
+  const int b = static_cast<int>(w / (static_cast<int64_t>(H) * S_pad));
+  int64_t r0 = static_cast<int64_t>(b) * S, l0 = (static_cast<int64_t>(b) * H + h) * S;
+  int len = S;
+  if (cu_seqlens) {
+    const int c0 = cu_seqlens[b], c1 = cu_seqlens[b + 1];
+    const bool valid = c0 >= 0 && c1 >= c0 && c1 <= S;
+    r0 = c0;
+    l0 = static_cast<int64_t>(h) * S + c0;
+    len = valid ? c1 - c0 : 0;
+  }
+  const int64_t dst = (static_cast<int64_t>(b) * H + h) * S_pad + s;
+  if (s >= len) {
+    if (lane == 0) {
+      Dst[dst] = 0.f;
+      lse_pad[dst] = INFINITY;
+    }
+    return;
+  }
+  const T* o = out + ((r0 + s) * H + h) * D;
+  const T* g = dout + ((r0 + s) * H + h) * D;
   float acc = 0.f;
 #pragma unroll
   for (int c = lane; c < D; c += 32) {
@@ -43,13 +68,8 @@ __global__ void bwd_rowdot(const T* __restrict__ out, const T* __restrict__ dout
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (lane == 0) {
-    const int h = static_cast<int>(row % H);
-    const int64_t bs = row / H;
-    const int s = static_cast<int>(bs % S);
-    const int b = static_cast<int>(bs / S);
-    const int64_t bh = static_cast<int64_t>(b) * H + h;
-    Dst[bh * S_pad + s] = acc;
-    lse_pad[bh * S_pad + s] = lse[bh * S + s];
+    Dst[dst] = acc;
+    lse_pad[dst] = lse[l0 + s];
   }
 }
 

@@ -9,10 +9,12 @@
 //   dV  += P^T dO                 dK  += dS^T Q          (TMEM accumulators)
 //   dQ^T = K^T dS^T -> added into the fp32 dq accumulator by TMA bulk
 //                      reduce-add (scale applied later)
-// Ragged S: rows past S of the last tile load as zeros (Q, K, V, dO by TMA;
-// lse and D from copies padded with zeros), which makes their
-// contributions to dK, dV and dQ vanish; stores and reduce-adds past S are
-// dropped.
+// Ragged and packed sequences: the rows of the last tile past the end of a
+// sequence load whatever follows it (zeros past the tensor's end, or the
+// next packed sequence).  Their lse copy is +inf, so P and dS vanish in
+// those query columns, and key rows past the end get P = 0; their dK/dV are
+// not stored.  The dQ^T columns of such query rows are exact zeros, so their
+// reduce-adds leave the next sequence's accumulator unchanged.
 //
 // One CTA per (key tile of 128, key/value head, batch); it loops over the
 // query heads of its grouped-query group and over the query tiles that can
@@ -92,13 +94,14 @@ constexpr uint32_t kIdescKM = idesc_bf16_f32(128, 128, false, true);   // dV, dK
 constexpr uint32_t kIdescMM = idesc_bf16_f32(128, 128, true, true);    // dQ^T
 
 struct Args {
-  int B, Hq, Hkv, S;
+  int B, Hq, Hkv;
+  int S;                 // tokens per batch entry of the tensors (packed: all sequences)
   int S_pad;             // row length of the padded lse / D copies
   float scale;
   float scale_log2;
   unsigned long long budget;
-  const float* lse;      // [B,Hq,S_pad], zero past S
-  const float* Drow;     // [B,Hq,S_pad], zero past S
+  const float* lse;      // [B,Hq,S_pad], +inf past each sequence's end
+  const float* Drow;     // [B,Hq,S_pad], zero past each sequence's end
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   AttnSched sched;
@@ -128,10 +131,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
   const uint32_t base = (raw + 1023u) & ~1023u;
   if (base - raw > kSlack) {
     // Cannot place the 1024-aligned layout inside the allocation: refuse.
-    if (threadIdx.x == 0) {
-      atomicOr(&g_err[0], 2);
-      atomicCAS(&g_err[1], 0, 100);
-    }
+    if (threadIdx.x == 0) record_error(kErrSmemAlign, 100);
     return;
   }
   uint8_t* gbase = smem_raw + (base - raw);
@@ -157,10 +157,16 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
   const int bg = static_cast<int>(blockIdx.x) / sc.n_tiles;
   const int g = bg % a.Hkv;
   const int b = bg / a.Hkv;
+  SeqView sv;
+  if (!seq_view(sc, b, a.S, &sv)) {
+    if (threadIdx.x == 0 && kt == 0) record_error(kErrSeqOffsets, 151);
+    return;
+  }
+  if (kt >= sv.n_tiles) return;  // a shorter packed sequence: no work here
   const bool shifted = head_shifted(sc, g * rep);
   const int ktok0 = token_tile(sc, kt, shifted) * kTile;
   QWalk qw;
-  qw.init(&sc, kt);
+  qw.init(&sc, kt, sv.n_tiles);
   const int nq = qw.count();
   const int nsteps = rep * nq;
 
@@ -193,10 +199,11 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmDO);
       mbar_expect_tx(bar(B_KV), 2 * kTileB);
-      tma_load_4d(sK, &tmK, bar(B_KV), 0, g, ktok0, b);
-      tma_load_4d(sK + kHalf, &tmK, bar(B_KV), 64, g, ktok0, b);
-      tma_load_4d(sV, &tmV, bar(B_KV), 0, g, ktok0, b);
-      tma_load_4d(sV + kHalf, &tmV, bar(B_KV), 64, g, ktok0, b);
+      const int ktok = sv.tokb + ktok0;
+      tma_load_4d(sK, &tmK, bar(B_KV), 0, g, ktok, sv.bm);
+      tma_load_4d(sK + kHalf, &tmK, bar(B_KV), 64, g, ktok, sv.bm);
+      tma_load_4d(sV, &tmV, bar(B_KV), 0, g, ktok, sv.bm);
+      tma_load_4d(sV + kHalf, &tmV, bar(B_KV), 64, g, ktok, sv.bm);
       bool ok = true;
       int issued0 = 0, issued1 = 0, o_issued = 0;
       for (int i = 0; i < nsteps && ok; ++i) {
@@ -208,8 +215,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         if (!ok) break;
         const uint32_t fb = bar(B_QFULL + st);
         mbar_expect_tx(fb, kTileB + 1024);
-        tma_load_4d(sQ + st * kTileB, &tmQ, fb, 0, h, qtok0, b);
-        tma_load_4d(sQ + st * kTileB + kHalf, &tmQ, fb, 64, h, qtok0, b);
+        tma_load_4d(sQ + st * kTileB, &tmQ, fb, 0, h, sv.tokb + qtok0, sv.bm);
+        tma_load_4d(sQ + st * kTileB + kHalf, &tmQ, fb, 64, h, sv.tokb + qtok0, sv.bm);
         const size_t ro = (static_cast<size_t>(b) * a.Hq + h) * a.S_pad + qtok0;
         bulk_load(sL + st * 512, a.lse + ro, 512, fb);
         bulk_load(sD + st * 512, a.Drow + ro, 512, fb);
@@ -217,8 +224,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         if (i >= 1) ok = wait_bar(bar(B_OEMPTY), (i - 1) & 1, wc, 112);
         if (!ok) break;
         mbar_expect_tx(bar(B_OFULL), kTileB);
-        tma_load_4d(sO, &tmDO, bar(B_OFULL), 0, h, qtok0, b);
-        tma_load_4d(sO + kHalf, &tmDO, bar(B_OFULL), 64, h, qtok0, b);
+        tma_load_4d(sO, &tmDO, bar(B_OFULL), 0, h, sv.tokb + qtok0, sv.bm);
+        tma_load_4d(sO + kHalf, &tmDO, bar(B_OFULL), 64, h, sv.tokb + qtok0, sv.bm);
         ++o_issued;
       }
       if (!ok) {
@@ -315,6 +322,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     const float c = a.scale_log2;
     const float L2E = 1.4426950408889634f;
     const uint64_t c2 = f2_pack(c, c);
+    const bool key_out = ktok0 + r >= sv.len;  // key row past the sequence's end
     bool ok = true;
     for (int i = 0; i < nsteps && ok; ++i) {
       const int st = i & 1;
@@ -347,6 +355,12 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
           p[e + 1] = p1;
           pk[e >> 1] = pack_bf16x2(p0, p1);
         }
+        if (key_out) {
+#pragma unroll
+          for (int e = 0; e < 64; ++e) p[e] = 0.f;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) pk[e] = 0u;
+        }
         tmem_st32u(tmem + lad + hq * 64, pk);
       }
       tmem_st_wait();
@@ -371,6 +385,10 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
           f2_unpack(t, t0, t1);
           dd[e >> 1] = pack_bf16x2(p[ql] * t0, p[ql + 1] * t1);
         }
+        if (key_out) {  // P = 0 there; keep dS = 0 whatever dP holds
+#pragma unroll
+          for (int e = 0; e < 16; ++e) dd[e] = 0u;
+        }
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
           const int cw = cc * 4 + v;  // 16-byte chunk within this half's 128-byte row
@@ -386,18 +404,18 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     if (ok) ok = wait_bar(bar(B_DONE), 0, wc, 315);
     ok = __all_sync(0xffffffffu, ok);
     // every lane takes part in the TMEM loads (warp-collective); key rows
-    // past S (ragged last tile) only skip their stores
-    const bool row_in = ktok0 + r < a.S;
+    // past the sequence's end (ragged last tile) only skip their stores
     if (ok) {
       tc_fence_after();
-      __nv_bfloat16* row =
-          a.dk + ((static_cast<size_t>(b) * a.S + (row_in ? ktok0 + r : 0)) * a.Hkv + g) * kD;
+      const size_t trow =
+          static_cast<size_t>(sv.bm) * a.S + sv.tokb + (key_out ? 0 : ktok0 + r);
+      __nv_bfloat16* row = a.dk + (trow * a.Hkv + g) * kD;
 #pragma unroll 1
       for (int cc = 2 * hq; cc < 2 * hq + 2; ++cc) {
         float o[32];
         __syncwarp();
         tmem_ld32(tmem + lad + 384 + cc * 32, o);
-        if (row_in) {
+        if (!key_out) {
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
             uint4 pk;
@@ -446,7 +464,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         fence_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_reduce_add_4d(&tmDQ, sR + wq * 8192, wq * 32, h, qtok0 + half * 64, b);
+          tma_reduce_add_4d(&tmDQ, sR + wq * 8192, wq * 32, h, sv.tokb + qtok0 + half * 64,
+                            sv.bm);
           bulk_commit();
         }
       }
@@ -456,11 +475,11 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     // ---- dV -> bf16
     if (ok) ok = wait_bar(bar(B_DONE), 0, wc, 412);
     ok = __all_sync(0xffffffffu, ok);
-    const bool row_in = ktok0 + r < a.S;
+    const bool row_in = ktok0 + r < sv.len;
     if (ok) {
       tc_fence_after();
-      __nv_bfloat16* row =
-          a.dv + ((static_cast<size_t>(b) * a.S + (row_in ? ktok0 + r : 0)) * a.Hkv + g) * kD;
+      const size_t trow = static_cast<size_t>(sv.bm) * a.S + sv.tokb + (row_in ? ktok0 + r : 0);
+      __nv_bfloat16* row = a.dv + (trow * a.Hkv + g) * kD;
 #pragma unroll 1
       for (int cc = 0; cc < 4; ++cc) {
         float o[32];

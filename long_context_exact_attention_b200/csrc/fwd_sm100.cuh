@@ -67,7 +67,8 @@ constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false, false);   // Q K^T
 constexpr uint32_t kIdescO = idesc_bf16_f32(128, 128, false, true);    // P V (V MN-major)
 
 struct Args {
-  int B, Hq, Hkv, S;
+  int B, Hq, Hkv;
+  int S;  // tokens per batch entry of the tensors (packed: all sequences)
   float scale_log2;
   unsigned long long budget;
   __nv_bfloat16* out;
@@ -115,7 +116,13 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
   const int g = h / (a.Hq / a.Hkv);
   const bool shifted = head_shifted(sc, h);
   const int qt0 = 2 * pr;
-  const bool has1 = qt0 + 1 < sc.n_tiles;
+  SeqView sv;
+  if (!seq_view(sc, b, a.S, &sv)) {
+    if (threadIdx.x == 0 && pr == 0) record_error(kErrSeqOffsets, 150);
+    return;
+  }
+  if (qt0 >= sv.n_tiles) return;  // a shorter packed sequence: no work here
+  const bool has1 = qt0 + 1 < sv.n_tiles;
   const int qt_last = has1 ? qt0 + 1 : qt0;
   const bool causal = sc.causal != 0;
 
@@ -145,29 +152,29 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       tma_prefetch_desc(&tmV);
       mbar_expect_tx(bar(B_Q), has1 ? 2 * kTileB : kTileB);
       for (int t = 0; t < (has1 ? 2 : 1); ++t) {
-        const int tok = token_tile(sc, qt0 + t, shifted) * kTile;
-        tma_load_4d(sQ + t * kTileB, &tmQ, bar(B_Q), 0, h, tok, b);
-        tma_load_4d(sQ + t * kTileB + kHalf, &tmQ, bar(B_Q), 64, h, tok, b);
+        const int tok = sv.tokb + token_tile(sc, qt0 + t, shifted) * kTile;
+        tma_load_4d(sQ + t * kTileB, &tmQ, bar(B_Q), 0, h, tok, sv.bm);
+        tma_load_4d(sQ + t * kTileB + kHalf, &tmQ, bar(B_Q), 64, h, tok, sv.bm);
       }
       KvWalk w;
-      w.init(&sc, qt_last);
-      int t, j = 0;
+      w.init(&sc, qt_last, sv.len);
+      int t, lo, hi, j = 0;
       int k_issued0 = 0, k_issued1 = 0, v_issued0 = 0, v_issued1 = 0;
       bool ok = true;
-      while (ok && w.next(t)) {
+      while (ok && w.next(t, lo, hi)) {
         const int st = j & 1;
-        const int tok = token_tile(sc, t, shifted) * kTile;
+        const int tok = sv.tokb + token_tile(sc, t, shifted) * kTile;
         if (j >= 2) ok = wait_bar(bar(B_KEMPTY + st), ((j - 2) >> 1) & 1, wc, 101);
         if (!ok) break;
         mbar_expect_tx(bar(B_KFULL + st), kTileB);
-        tma_load_4d(sK + st * kTileB, &tmK, bar(B_KFULL + st), 0, g, tok, b);
-        tma_load_4d(sK + st * kTileB + kHalf, &tmK, bar(B_KFULL + st), 64, g, tok, b);
+        tma_load_4d(sK + st * kTileB, &tmK, bar(B_KFULL + st), 0, g, tok, sv.bm);
+        tma_load_4d(sK + st * kTileB + kHalf, &tmK, bar(B_KFULL + st), 64, g, tok, sv.bm);
         if (st) ++k_issued1; else ++k_issued0;
         if (j >= 2) ok = wait_bar(bar(B_VEMPTY + st), ((j - 2) >> 1) & 1, wc, 102);
         if (!ok) break;
         mbar_expect_tx(bar(B_VFULL + st), kTileB);
-        tma_load_4d(sV + st * kTileB, &tmV, bar(B_VFULL + st), 0, g, tok, b);
-        tma_load_4d(sV + st * kTileB + kHalf, &tmV, bar(B_VFULL + st), 64, g, tok, b);
+        tma_load_4d(sV + st * kTileB, &tmV, bar(B_VFULL + st), 0, g, tok, sv.bm);
+        tma_load_4d(sV + st * kTileB + kHalf, &tmV, bar(B_VFULL + st), 64, g, tok, sv.bm);
         if (st) ++v_issued1; else ++v_issued0;
         ++j;
       }
@@ -186,8 +193,8 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       const uint32_t qts[2] = {static_cast<uint32_t>(qt0), static_cast<uint32_t>(qt0 + 1)};
       bool ok = wait_bar(bar(B_Q), 0, wc, 201);
       KvWalk w;
-      w.init(&sc, qt_last);
-      int T, Tn;
+      w.init(&sc, qt_last, sv.len);
+      int T, Tn, lo, hi;
       int pv_cnt[2] = {0, 0};
       // S_t for key tile j into the S/P columns of query tile t
       auto issue_s = [&](int tq, int j) {
@@ -204,7 +211,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       auto act = [&](int tq, int T_) {
         return (tq == 0 || has1) && tile_vis(causal, static_cast<int>(qts[tq]), T_) != VIS_NONE;
       };
-      bool have = ok && w.next(T);
+      bool have = ok && w.next(T, lo, hi);
       if (have) {
         ok = wait_bar(bar(B_KFULL), 0, wc, 202);
         if (ok) {
@@ -216,7 +223,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       }
       int j = 0;
       while (ok && have) {
-        const bool has_next = w.next(Tn);
+        const bool has_next = w.next(Tn, lo, hi);
         ok = wait_bar(bar(B_VFULL + (j & 1)), (j >> 1) & 1, wc, 203);
         if (ok && has_next) ok = wait_bar(bar(B_KFULL + ((j + 1) & 1)), ((j + 1) >> 1) & 1, wc, 204);
         for (int tq = 0; tq < 2 && ok; ++tq) {
@@ -262,9 +269,9 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     bool ok = true;
     if (tq == 0 || has1) {
       KvWalk w;
-      w.init(&sc, qt_last);
-      int t;
-      while (ok && w.next(t)) {
+      w.init(&sc, qt_last, sv.len);
+      int t, lo, hi;
+      while (ok && w.next(t, lo, hi)) {
         const int vis = tile_vis(causal, qt, t);
         if (vis == VIS_NONE) continue;
         ok = __all_sync(0xffffffffu, wait_bar(bar(B_SFULL + tq), cnt & 1, wc, 301));
@@ -272,19 +279,20 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         tc_fence_after();
         float s[128];
         tmem_ld128(tS, s);
-        if (vis == VIS_DIAG) {
-#pragma unroll
-          for (int i = 0; i < 128; ++i)
-            if (i > r) s[i] = -INFINITY;
-        } else {
-          // last key tile of a ragged sequence: keys past S are zero-filled
-          // rows, masked here (on the diagonal the causal mask covers them
-          // for every stored row)
-          const int kv_valid = sc.S - token_tile(sc, t, shifted) * kTile;
-          if (kv_valid < kTile) {
+        // Keys outside this visit's range [lo, hi) -- another chunk's keys
+        // in a tile that straddles a chunk boundary, or rows past the end
+        // of the sequence -- and, on the diagonal, keys after the row.
+        {
+          const int lim = vis == VIS_DIAG ? (hi < r + 1 ? hi : r + 1) : hi;
+          if (lim < kTile) {
 #pragma unroll
             for (int i = 0; i < 128; ++i)
-              if (i >= kv_valid) s[i] = -INFINITY;
+              if (i >= lim) s[i] = -INFINITY;
+          }
+          if (lo > 0) {
+#pragma unroll
+            for (int i = 0; i < 128; ++i)
+              if (i < lo) s[i] = -INFINITY;
           }
         }
         // Row max: eight independent chains of 3-input max.
@@ -352,13 +360,13 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       ok = __all_sync(0xffffffffu, ok && cnt >= 1);
       const int tok = token_tile(sc, qt, shifted) * kTile + r;
       // Every lane takes part in the TMEM loads (warp-collective); rows past
-      // S (ragged last tile) only skip their stores.
-      const bool row_in = tok < sc.S;
+      // the end of the sequence (ragged last tile) only skip their stores.
+      const bool row_in = tok < sv.len;
+      const size_t trow = static_cast<size_t>(sv.bm) * a.S + sv.tokb + (row_in ? tok : 0);
       if (ok) {
         tc_fence_after();
         const float inv = (l_run > 0.f) ? 1.0f / l_run : 0.f;
-        __nv_bfloat16* orow =
-            a.out + ((static_cast<size_t>(b) * a.S + (row_in ? tok : 0)) * a.Hq + h) * kD;
+        __nv_bfloat16* orow = a.out + (trow * a.Hq + h) * kD;
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           float o[32];
@@ -378,7 +386,8 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         }
         const float lse = (l_run > 0.f) ? (m_run + lg2_approx(l_run)) * 0.69314718055994531f
                                         : -INFINITY;
-        if (row_in) a.lse[(static_cast<size_t>(b) * a.Hq + h) * a.S + tok] = lse;
+        if (row_in)
+          a.lse[(static_cast<size_t>(sv.bm) * a.Hq + h) * a.S + sv.tokb + tok] = lse;
       }
     }
   }

@@ -43,14 +43,17 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 constexpr unsigned long long kDefaultBudget = 1ull << 31;
 
 struct Common {
-  int B, Hq, Hkv, S, d;
+  int B, Hq, Hkv, S, d;  // tensor extents: B batch entries of S tokens (packed: 1 x total)
+  int n_seq;             // sequences (B unless packed)
+  int S_seq;             // longest sequence (S unless packed)
+  const int* cu;         // packed token offsets (device), else null
   int dtype;
   float scale;
   int tile;
 };
 
-// S rounded up to the tile of the element type's path.
-int s_pad_of(const Common& c) { return (c.S + c.tile - 1) / c.tile * c.tile; }
+// The longest sequence rounded up to the tile of the element type's path.
+int s_pad_of(const Common& c) { return (c.S_seq + c.tile - 1) / c.tile * c.tile; }
 
 lca_status check_shape(const lca_shape* sh, Common* c) {
   if (!sh) return fail(LCA_ERR_INVALID_ARG, "shape is NULL");
@@ -70,6 +73,9 @@ lca_status check_shape(const lca_shape* sh, Common* c) {
   c->Hkv = static_cast<int>(sh->Hkv);
   c->S = static_cast<int>(sh->S);
   c->d = static_cast<int>(sh->d);
+  c->n_seq = c->B;
+  c->S_seq = c->S;
+  c->cu = nullptr;
   c->dtype = sh->dtype;
   c->scale = sh->scale > 0.f ? sh->scale : 1.0f / std::sqrt(static_cast<float>(sh->d));
   if (sh->dtype == LCA_BF16) {
@@ -81,6 +87,25 @@ lca_status check_shape(const lca_shape* sh, Common* c) {
       return fail(LCA_ERR_UNSUPPORTED, "fp32 path needs d in {64, 128}");
     c->tile = 64;
   }
+  return LCA_OK;
+}
+
+// Packed variable-length batch: shape->B sequences whose tokens are
+// concatenated along one axis of shape->S tokens, sequence b holding tokens
+// [cu_seqlens[b], cu_seqlens[b+1]), none longer than max_seqlen.
+lca_status check_packed(const lca_shape* sh, const int32_t* cu_seqlens, int64_t max_seqlen,
+                        Common* c) {
+  lca_status r = check_shape(sh, c);
+  if (r != LCA_OK) return r;
+  if (!cu_seqlens) return fail(LCA_ERR_INVALID_ARG, "cu_seqlens is NULL");
+  if (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)
+    return fail(LCA_ERR_INVALID_ARG, "cu_seqlens not 4-byte aligned");
+  if (max_seqlen <= 0 || max_seqlen > sh->S)
+    return fail(LCA_ERR_INVALID_ARG, "max_seqlen must lie in [1, total tokens]");
+  c->n_seq = c->B;
+  c->B = 1;
+  c->S_seq = static_cast<int>(max_seqlen);
+  c->cu = cu_seqlens;
   return LCA_OK;
 }
 
@@ -98,22 +123,27 @@ lca_status check_ptrs(std::initializer_list<const void*> ps) {
 lca_status make_chunk_sched(const Common& c, int causal, int64_t kv_chunk, const lca_opts* o,
                             AttnSched* s) {
   std::memset(s, 0, sizeof *s);
-  s->S = c.S;
-  s->n_tiles = (c.S + c.tile - 1) / c.tile;
+  s->S = c.S_seq;
+  s->tile = c.tile;
+  s->n_tiles = (c.S_seq + c.tile - 1) / c.tile;
   s->causal = causal ? 1 : 0;
-  if (kv_chunk < 0 || kv_chunk % c.tile)
-    return fail(LCA_ERR_INVALID_ARG, "kv_chunk must be a non-negative multiple of %d", c.tile);
-  const int64_t chunk = kv_chunk == 0 ? static_cast<int64_t>(s->n_tiles) * c.tile : kv_chunk;
-  s->tiles_per_chunk = static_cast<int>(chunk / c.tile);
-  s->n_chunks = static_cast<int>((s->n_tiles + s->tiles_per_chunk - 1) / s->tiles_per_chunk);
-  if (s->n_chunks > LCA_MAX_CHUNKS)
-    return fail(LCA_ERR_INVALID_ARG, "%d chunks exceed LCA_MAX_CHUNKS", s->n_chunks);
+  s->cu_seqlens = c.cu;
+  if (kv_chunk < 0) return fail(LCA_ERR_INVALID_ARG, "kv_chunk must be >= 0");
+  const int64_t chunk = kv_chunk == 0 || kv_chunk > c.S_seq ? c.S_seq : kv_chunk;
+  s->kv_chunk = static_cast<int>(chunk);
+  const int64_t n_chunks = (c.S_seq + chunk - 1) / chunk;
+  if (n_chunks > LCA_MAX_CHUNKS)
+    return fail(LCA_ERR_INVALID_ARG, "%lld chunks exceed LCA_MAX_CHUNKS",
+                static_cast<long long>(n_chunks));
+  s->n_chunks = static_cast<int>(n_chunks);
   s->order = o ? o->order : LCA_ORDER_INORDER;
   if (s->order < 0 || s->order > 2) return fail(LCA_ERR_INVALID_ARG, "unknown chunk order");
-  int64_t qb = (o && o->q_block) ? o->q_block : chunk;
-  if (qb <= 0 || qb % c.tile)
-    return fail(LCA_ERR_INVALID_ARG, "q_block must be a positive multiple of %d", c.tile);
-  s->q_block_tiles = static_cast<int>(qb / c.tile);
+  const int64_t qb = (o && o->q_block) ? o->q_block : chunk;
+  if (qb <= 0) return fail(LCA_ERR_INVALID_ARG, "q_block must be positive");
+  s->q_block = static_cast<int>(qb > c.S_seq ? c.S_seq : qb);
+  if (s->order == LCA_ORDER_CUSTOM && c.cu)
+    return fail(LCA_ERR_INVALID_ARG,
+                "CUSTOM chunk order needs one chunk count; packed sequences have several");
   if (s->order == LCA_ORDER_CUSTOM) {
     if (!o->chunk_perm) return fail(LCA_ERR_INVALID_ARG, "CUSTOM order needs chunk_perm");
     bool seen[LCA_MAX_CHUNKS] = {};
@@ -141,12 +171,13 @@ lca_status make_s2_sched(const Common& c, int causal, int64_t group, int64_t shi
   if ((c.Hq - shift_heads) % rep)
     return fail(LCA_ERR_INVALID_ARG, "shifted heads must cover whole grouped-query groups");
   s->S = c.S;
+  s->tile = c.tile;
   s->n_tiles = c.S / c.tile;
   s->causal = causal ? 1 : 0;
   s->s2 = 1;
   s->n_chunks = 1;
-  s->tiles_per_chunk = s->n_tiles;
-  s->q_block_tiles = s->n_tiles;
+  s->kv_chunk = c.S;
+  s->q_block = c.S;
   s->group_tiles = static_cast<int>(group / c.tile);
   s->shift_tiles = static_cast<int>(group / 2 / c.tile);
   s->first_shifted_head = static_cast<int>(c.Hq - shift_heads);
@@ -265,10 +296,10 @@ unsigned long long budget_of(const lca_opts* o) {
 lca_status run_fwd(const Common& c, const AttnSched& s, const void* q, const void* k,
                    const void* v, void* out, float* lse, unsigned long long budget,
                    cudaStream_t st) {
-  const unsigned grid = static_cast<unsigned>(s.n_tiles) * c.B * c.Hq;
+  const unsigned grid = static_cast<unsigned>(s.n_tiles) * c.n_seq * c.Hq;
   if (c.dtype == LCA_BF16) {
     // one CTA per pair of 128-row query tiles
-    const unsigned grid2 = static_cast<unsigned>((s.n_tiles + 1) / 2) * c.B * c.Hq;
+    const unsigned grid2 = static_cast<unsigned>((s.n_tiles + 1) / 2) * c.n_seq * c.Hq;
     CUtensorMap mq, mk, mv;
     lca_status r;
     if ((r = make_map(&mq, q, c.B, c.S, c.Hq)) != LCA_OK) return r;
@@ -276,7 +307,7 @@ lca_status run_fwd(const Common& c, const AttnSched& s, const void* q, const voi
     if ((r = make_map(&mv, v, c.B, c.S, c.Hkv)) != LCA_OK) return r;
     if ((r = ensure_smem(attn_fwd_bf16_sm100, fwd::kSmemBytes, 0)) != LCA_OK) return r;
     fwd::Args a;
-    a.B = c.B;
+    a.B = c.n_seq;
     a.Hq = c.Hq;
     a.Hkv = c.Hkv;
     a.S = c.S;
@@ -294,7 +325,7 @@ lca_status run_fwd(const Common& c, const AttnSched& s, const void* q, const voi
   a.v = static_cast<const float*>(v);
   a.o_out = static_cast<float*>(out);
   a.lse_out = lse;
-  a.B = c.B;
+  a.B = c.n_seq;
   a.Hq = c.Hq;
   a.Hkv = c.Hkv;
   a.S = c.S;
@@ -313,10 +344,11 @@ lca_status run_fwd(const Common& c, const AttnSched& s, const void* q, const voi
 }
 
 // ---------------------------------------------------------------- backward
-// Workspace: D rows and a copy of lse, each [B][Hq][S_pad] with S_pad = S
-// rounded up to the tile (zero past S), then (bf16) the fp32 dq accumulator.
+// Workspace: D rows and a copy of lse, each [n_seq][Hq][S_pad] with S_pad
+// the longest sequence rounded up to the tile, then (bf16) the fp32 dq
+// accumulator over every token row.
 size_t ws_d_bytes(const Common& c) {
-  const size_t n = static_cast<size_t>(c.B) * c.Hq * s_pad_of(c) * sizeof(float);
+  const size_t n = static_cast<size_t>(c.n_seq) * c.Hq * s_pad_of(c) * sizeof(float);
   return (n + 255) & ~static_cast<size_t>(255);
 }
 size_t ws_bytes_of(const Common& c) {
@@ -338,14 +370,10 @@ lca_status run_bwd(const Common& c, const AttnSched& s, const void* q, const voi
   float* Drow = static_cast<float*>(ws);
   float* lse_pad = reinterpret_cast<float*>(static_cast<char*>(ws) + ws_d_bytes(c));
   const int64_t rows = static_cast<int64_t>(c.B) * c.S * c.Hq;
-  const unsigned rd_blocks = static_cast<unsigned>((rows * 32 + 255) / 256);
-  const unsigned grid = static_cast<unsigned>(s.n_tiles) * c.B * c.Hkv;
+  const int64_t pad_rows = static_cast<int64_t>(c.n_seq) * S_pad * c.Hq;
+  const unsigned rd_blocks = static_cast<unsigned>((pad_rows * 32 + 255) / 256);
+  const unsigned grid = static_cast<unsigned>(s.n_tiles) * c.n_seq * c.Hkv;
   cudaError_t e;
-  if (S_pad != c.S) {
-    // entries past S must read as zeros
-    e = cudaMemsetAsync(ws, 0, 2 * ws_d_bytes(c), st);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(padded rows)");
-  }
   lca_status r;
   if (c.dtype == LCA_BF16) {
     float* acc = reinterpret_cast<float*>(static_cast<char*>(ws) + 2 * ws_d_bytes(c));
@@ -354,7 +382,7 @@ lca_status run_bwd(const Common& c, const AttnSched& s, const void* q, const voi
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(dq accumulator)");
     bwd_rowdot<__nv_bfloat16, 128><<<rd_blocks, 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse,
-        Drow, lse_pad, c.B, c.S, S_pad, c.Hq);
+        Drow, lse_pad, c.n_seq, c.S, S_pad, c.Hq, c.cu);
     if ((r = launched("bwd_rowdot")) != LCA_OK) return r;
     CUtensorMap mq, mk, mv, mdo, mdq;
     if ((r = make_map(&mq, q, c.B, c.S, c.Hq)) != LCA_OK) return r;
@@ -365,7 +393,7 @@ lca_status run_bwd(const Common& c, const AttnSched& s, const void* q, const voi
     if ((r = check_bwd_regs()) != LCA_OK) return r;
     if ((r = ensure_smem(attn_bwd_bf16_sm100, bwd::kSmemBytes, 3)) != LCA_OK) return r;
     bwd::Args a;
-    a.B = c.B;
+    a.B = c.n_seq;
     a.Hq = c.Hq;
     a.Hkv = c.Hkv;
     a.S = c.S;
@@ -391,11 +419,12 @@ lca_status run_bwd(const Common& c, const AttnSched& s, const void* q, const voi
   if (c.d == 64)
     bwd_rowdot<float, 64><<<rd_blocks, 256, 0, st>>>(static_cast<const float*>(out),
                                                        static_cast<const float*>(dout), lse, Drow,
-                                                       lse_pad, c.B, c.S, S_pad, c.Hq);
+                                                       lse_pad, c.n_seq, c.S, S_pad, c.Hq, c.cu);
   else
     bwd_rowdot<float, 128><<<rd_blocks, 256, 0, st>>>(static_cast<const float*>(out),
                                                         static_cast<const float*>(dout), lse,
-                                                        Drow, lse_pad, c.B, c.S, S_pad, c.Hq);
+                                                        Drow, lse_pad, c.n_seq, c.S, S_pad, c.Hq,
+                                                        c.cu);
   if ((r = launched("bwd_rowdot")) != LCA_OK) return r;
   f32::Args a{};
   a.q = static_cast<const float*>(q);
@@ -408,7 +437,7 @@ lca_status run_bwd(const Common& c, const AttnSched& s, const void* q, const voi
   a.dq = static_cast<float*>(dq);
   a.dk = static_cast<float*>(dk);
   a.dv = static_cast<float*>(dv);
-  a.B = c.B;
+  a.B = c.n_seq;
   a.Hq = c.Hq;
   a.Hkv = c.Hkv;
   a.S = c.S;
@@ -459,10 +488,10 @@ lca_status lca_attn_fwd(const lca_shape* shape, const void* q, const void* k, co
 
 size_t lca_attn_bwd_workspace_size(const lca_shape* shape) {
   Common c;
-  const std::string keep = t_last_error;
-  if (check_shape(shape, &c) != LCA_OK) return 0;
+  const std::string keep = t_last_error;  // a size query leaves the error detail alone
+  const bool ok = check_shape(shape, &c) == LCA_OK;
   t_last_error = keep;
-  return ws_bytes_of(c);
+  return ok ? ws_bytes_of(c) : 0;
 }
 
 lca_status lca_attn_bwd(const lca_shape* shape, const void* q, const void* k, const void* v,
@@ -505,6 +534,44 @@ lca_status lca_s2attn_bwd(const lca_shape* shape, const void* q, const void* k, 
                  static_cast<cudaStream_t>(stream));
 }
 
+lca_status lca_attn_fwd_varlen(const lca_shape* shape, const int32_t* cu_seqlens,
+                               int64_t max_seqlen, const void* q, const void* k, const void* v,
+                               int causal, int64_t kv_chunk, const lca_opts* opts, void* out,
+                               float* lse, void* stream) {
+  Common c;
+  lca_status r = check_packed(shape, cu_seqlens, max_seqlen, &c);
+  if (r != LCA_OK) return r;
+  if ((r = check_ptrs({q, k, v, out, lse})) != LCA_OK) return r;
+  AttnSched s;
+  if ((r = make_chunk_sched(c, causal, kv_chunk, opts, &s)) != LCA_OK) return r;
+  return run_fwd(c, s, q, k, v, out, lse, budget_of(opts), static_cast<cudaStream_t>(stream));
+}
+
+size_t lca_attn_bwd_varlen_workspace_size(const lca_shape* shape, int64_t max_seqlen) {
+  Common c;
+  const std::string keep = t_last_error;
+  // the offsets are not read here; any aligned non-null stand-in passes the check
+  static const int32_t stand_in[1] = {0};
+  const bool ok = check_packed(shape, stand_in, max_seqlen, &c) == LCA_OK;
+  t_last_error = keep;
+  return ok ? ws_bytes_of(c) : 0;
+}
+
+lca_status lca_attn_bwd_varlen(const lca_shape* shape, const int32_t* cu_seqlens,
+                               int64_t max_seqlen, const void* q, const void* k, const void* v,
+                               const void* out, const float* lse, const void* dout, int causal,
+                               void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
+                               void* stream) {
+  Common c;
+  lca_status r = check_packed(shape, cu_seqlens, max_seqlen, &c);
+  if (r != LCA_OK) return r;
+  if ((r = check_ptrs({q, k, v, out, lse, dout, dq, dk, dv})) != LCA_OK) return r;
+  AttnSched s;
+  if ((r = make_chunk_sched(c, causal, 0, nullptr, &s)) != LCA_OK) return r;
+  return run_bwd(c, s, q, k, v, out, lse, dout, dq, dk, dv, workspace, ws_bytes, kDefaultBudget,
+                 static_cast<cudaStream_t>(stream));
+}
+
 lca_status lca_lse_merge(int64_t rows, int64_t d, const float* o_a, const float* lse_a,
                          const float* o_b, const float* lse_b, float* o_out, float* lse_out,
                          void* stream) {
@@ -529,7 +596,12 @@ lca_status lca_check(void* stream) {
   if (h[0]) {
     const int z[2] = {0, 0};
     cudaMemcpyToSymbol(g_err, z, sizeof z);
-    if (h[0] & 1) return fail(LCA_ERR_TIMEOUT, "a kernel wait ran out (site %d)", h[1]);
+    if (h[0] & kErrTimeout) return fail(LCA_ERR_TIMEOUT, "a kernel wait ran out (site %d)", h[1]);
+    if (h[0] & kErrSeqOffsets)
+      return fail(LCA_ERR_INVALID_ARG,
+                  "cu_seqlens out of order or range, or a sequence longer than max_seqlen "
+                  "(site %d); outputs of that call are undefined",
+                  h[1]);
     return fail(LCA_ERR_CUDA, "a kernel could not align its shared-memory layout (site %d)",
                 h[1]);
   }

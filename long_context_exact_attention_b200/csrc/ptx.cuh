@@ -12,10 +12,18 @@
 
 namespace lca {
 
-// Device error word: [0] = error bits (1 = wait timed out), [1] = site id of
-// the first timeout.  Read and cleared by lca_check().  The library is one
-// translation unit, so the definition lives here.
+// Device error word: [0] = error bits (1 = a wait timed out, 2 = a kernel
+// could not align its shared-memory layout, 4 = packed sequence offsets out
+// of order or out of range), [1] = site id of the first error.  Read and
+// cleared by lca_check().  The library is one translation unit, so the
+// definition lives here.
 __device__ int g_err[2];
+constexpr int kErrTimeout = 1, kErrSmemAlign = 2, kErrSeqOffsets = 4;
+
+__device__ __forceinline__ void record_error(int bit, int site) {
+  atomicOr(&g_err[0], bit);
+  atomicCAS(&g_err[1], 0, site);
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -64,8 +72,7 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Wa
     if (*c.abort) return false;
     if (static_cast<unsigned long long>(clock64() - t0) > c.budget) {
       *c.abort = 1;
-      atomicOr(&g_err[0], 1);
-      atomicCAS(&g_err[1], 0, site);
+      record_error(kErrTimeout, site);
       return false;
     }
   }

@@ -7,16 +7,21 @@
 // walk stays inside the query's group and each position tile maps to one
 // contiguous token tile because G/2 is a whole number of tiles.
 //
-// Ragged lengths: when S is not a multiple of the tile, the last tile is
-// partial and the last chunk may hold fewer tiles.
+// Sequences.  A batch entry is one sequence of S tokens, or -- for packed
+// variable-length batches -- sequence b holds tokens [cu[b], cu[b+1]) of one
+// packed token axis.  Every walk runs inside one sequence, with positions
+// counted from its first token.  When a sequence's length is not a multiple
+// of the tile its last tile is partial.
 //
 // Chunk order (Ring Attention with Blockwise Transformers, Summary: a query
 // block meets the key/value blocks in the order the ring delivers them, and
 // the result does not depend on it).  Keys are split into chunks of
-// `tiles_per_chunk` tiles; a query tile visits the chunks in order
+// `kv_chunk` keys, any length; a query tile visits the chunks in order
 // (in-order), ring order (query block i: chunks i, i-1, ..., i+1 mod n) or a
 // caller-given permutation, and the tiles inside a chunk in ascending order.
-// Causal chunks/tiles after the query tile are skipped.
+// A tile that straddles a chunk boundary is visited once per chunk, each
+// visit restricted to that chunk's keys [lo, hi).  Causal tiles after the
+// query tile are skipped.
 #pragma once
 
 #include <stdint.h>
@@ -26,17 +31,19 @@
 namespace lca {
 
 struct AttnSched {
-  int S;                   // sequence length in tokens
-  int n_tiles;             // ceil(S / tile); the last tile may be partial
+  int S;                   // longest sequence in tokens (every sequence when not packed)
+  int n_tiles;             // ceil(S / tile)
+  int tile;                // tokens per tile
   int causal;
   int s2;                  // 1: S2-Attn walk
-  int tiles_per_chunk;     // chunked walk
-  int n_chunks;
+  int kv_chunk;            // chunked walk: keys per chunk (>= 1)
+  int n_chunks;            // chunks of a sequence of S tokens
   int order;               // lca_order
-  int q_block_tiles;       // ring query block, in tiles
+  int q_block;             // ring query block, in tokens
   int group_tiles;         // S2: group / tile
   int shift_tiles;         // S2: (group / 2) / tile
   int first_shifted_head;  // S2: Hq - shift_heads
+  const int* cu_seqlens;   // packed sequences: n_seqs + 1 token offsets (device), else null
   uint16_t perm[LCA_MAX_CHUNKS];
 };
 
@@ -49,14 +56,43 @@ __host__ __device__ inline int token_tile(const AttnSched& s, int t, bool shifte
   return shifted ? (t + s.shift_tiles) % s.n_tiles : t;
 }
 
-// Walk of the key/value position tiles for query position tile qt.
+// Where sequence b lives in the tensors: tensor coordinates (batch index bm,
+// first token tokb) and its length.  S_tensor is the token extent of one
+// batch entry of the tensors (the packed length for packed sequences).
+struct SeqView {
+  int bm, tokb, len, n_tiles;
+};
+
+// False when packed offsets are out of order or out of range (the caller
+// records an error and does no work for the sequence).
+__host__ __device__ inline bool seq_view(const AttnSched& s, int b, int S_tensor, SeqView* v) {
+  if (!s.cu_seqlens) {
+    v->bm = b;
+    v->tokb = 0;
+    v->len = s.S;
+    v->n_tiles = s.n_tiles;
+    return true;
+  }
+  const int c0 = s.cu_seqlens[b], c1 = s.cu_seqlens[b + 1];
+  if (c0 < 0 || c1 < c0 || c1 > S_tensor || c1 - c0 > s.S) return false;
+  v->bm = 0;
+  v->tokb = c0;
+  v->len = c1 - c0;
+  v->n_tiles = (v->len + s.tile - 1) / s.tile;
+  return true;
+}
+
+// Walk of the key/value position tiles for query position tile qt of a
+// sequence of `len` tokens.
 struct KvWalk {
   const AttnSched* s;
-  int qt, ci, t, t_end, qb;
+  int qt, len, n_chunks, key_end;
+  int ci, t, t_end, c_lo, c_hi, qb;
 
-  __host__ __device__ void init(const AttnSched* sc, int qt_) {
+  __host__ __device__ void init(const AttnSched* sc, int qt_, int len_) {
     s = sc;
     qt = qt_;
+    len = len_;
     ci = 0;
     if (s->s2) {
       const int g0 = (qt / s->group_tiles) * s->group_tiles;
@@ -64,54 +100,68 @@ struct KvWalk {
       t_end = s->causal ? qt + 1 : g0 + s->group_tiles;
     } else {
       t = t_end = 0;
-      qb = qt / s->q_block_tiles;
+      n_chunks = (len + s->kv_chunk - 1) / s->kv_chunk;
+      // keys past the query tile's last row are invisible under the mask
+      key_end = len;
+      if (s->causal && (qt + 1) * s->tile < key_end) key_end = (qt + 1) * s->tile;
+      qb = static_cast<int>(static_cast<int64_t>(qt) * s->tile / s->q_block);
     }
   }
   __host__ __device__ int chunk_at(int i) const {
     if (s->order == LCA_ORDER_RING) {
-      const int n = s->n_chunks;
+      const int n = n_chunks;
       return ((qb - i) % n + n) % n;
     }
     if (s->order == LCA_ORDER_CUSTOM) return s->perm[i];
     return i;
   }
-  // Next key/value position tile; false when the walk is over.
-  __host__ __device__ bool next(int& tile) {
+  // Next visit: key/value position tile and the key range [lo, hi) of it
+  // (offsets inside the tile) that the visit covers; false when the walk is
+  // over.
+  __host__ __device__ bool next(int& tile, int& lo, int& hi) {
     if (s->s2) {
       if (t < t_end) {
         tile = t++;
+        lo = 0;
+        hi = s->tile;
         return true;
       }
       return false;
     }
     while (t >= t_end) {
-      if (ci >= s->n_chunks) return false;
+      if (ci >= n_chunks) return false;
       const int c = chunk_at(ci++);
-      t = c * s->tiles_per_chunk;
-      t_end = t + s->tiles_per_chunk;
-      if (t_end > s->n_tiles) t_end = s->n_tiles;  // last chunk may be partial
-      if (s->causal && t_end > qt + 1) t_end = qt + 1;
+      c_lo = c * s->kv_chunk;
+      c_hi = c_lo + s->kv_chunk;
+      if (c_hi > key_end) c_hi = key_end;
+      if (c_lo >= c_hi) continue;  // nothing visible in this chunk
+      t = c_lo / s->tile;
+      t_end = (c_hi - 1) / s->tile + 1;
     }
     tile = t++;
+    const int k0 = tile * s->tile;
+    lo = c_lo > k0 ? c_lo - k0 : 0;
+    hi = c_hi - k0 < s->tile ? c_hi - k0 : s->tile;
     return true;
   }
 };
 
-// Query position tiles whose walk contains key position tile kt (for the
-// backward pass, which loops over queries for a fixed key tile).
+// Query position tiles whose walk contains key position tile kt, for a
+// sequence of n_tiles tiles (the backward pass loops over queries for a
+// fixed key tile).
 struct QWalk {
   int t, t_end;
-  __host__ __device__ void init(const AttnSched* s, int kt) {
+  __host__ __device__ void init(const AttnSched* s, int kt, int n_tiles) {
     if (s->s2) {
       const int g0 = (kt / s->group_tiles) * s->group_tiles;
       t = s->causal ? kt : g0;
       t_end = g0 + s->group_tiles;
     } else {
       t = s->causal ? kt : 0;
-      t_end = s->n_tiles;
+      t_end = n_tiles;
     }
   }
-  __host__ __device__ int count() const { return t_end - t; }
+  __host__ __device__ int count() const { return t_end > t ? t_end - t : 0; }
 };
 
 }  // namespace lca

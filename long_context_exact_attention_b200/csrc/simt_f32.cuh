@@ -10,8 +10,9 @@
 // query heads of its group and the visible query tiles; dK and dV live in
 // registers, dQ is accumulated with shared-memory atomics per query tile and
 // flushed to the float32 dq output with global atomics.
-// Ragged S: rows past S of the last tile load as zeros and are not stored;
-// keys past S are masked in the forward.
+// Ragged and packed sequences: rows past the end of a sequence load as
+// zeros and are not stored; the forward masks keys outside each visit's key
+// range (which ends at the sequence's end).
 #pragma once
 
 #include "sched.cuh"
@@ -26,8 +27,9 @@ constexpr int kRowsPerWarp = kT / (kThreads / 32);
 struct Args {
   const float *q, *k, *v, *out, *lse, *dout, *D;  // lse, D: padded [B,Hq,S_pad]
   float *o_out, *lse_out, *dq, *dk, *dv;
-  int B, Hq, Hkv, S;
-  int S_pad;
+  int B, Hq, Hkv;
+  int S;      // tokens per batch entry of the tensors (packed: all sequences)
+  int S_pad;  // row length of the padded lse / D copies
   float scale;
   AttnSched sched;
 };
@@ -57,14 +59,20 @@ __global__ void __launch_bounds__(kThreads) attn_fwd_f32(const __grid_constant__
   const int bh = static_cast<int>(blockIdx.x) % BH;
   const int h = bh % a.Hq, b = bh / a.Hq;
   const int g = h / (a.Hq / a.Hkv);
+  SeqView sv;
+  if (!seq_view(sc, b, a.S, &sv)) {
+    if (threadIdx.x == 0 && qt == 0) record_error(kErrSeqOffsets, 160);
+    return;
+  }
+  if (qt >= sv.n_tiles) return;  // a shorter packed sequence: no work here
+  const size_t row0 = static_cast<size_t>(sv.bm) * a.S + sv.tokb;  // first row of the sequence
   const bool shifted = head_shifted(sc, h);
   const int qtok0 = token_tile(sc, qt, shifted) * kT;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   for (int i = threadIdx.x; i < kT * D; i += kThreads) {
     const int r = i / D, c = i % D;
-    sQ[i] = (qtok0 + r < a.S) ? a.q[((static_cast<size_t>(b) * a.S + qtok0 + r) * a.Hq + h) * D + c]
-                              : 0.f;
+    sQ[i] = (qtok0 + r < sv.len) ? a.q[((row0 + qtok0 + r) * a.Hq + h) * D + c] : 0.f;
   }
   float m[kRowsPerWarp], l[kRowsPerWarp], o[kRowsPerWarp][E];
 #pragma unroll
@@ -75,21 +83,20 @@ __global__ void __launch_bounds__(kThreads) attn_fwd_f32(const __grid_constant__
     for (int e = 0; e < E; ++e) o[rr][e] = 0.f;
   }
   KvWalk w;
-  w.init(&sc, qt);
-  int t;
-  while (w.next(t)) {
+  w.init(&sc, qt, sv.len);
+  int t, lo, hi;
+  while (w.next(t, lo, hi)) {
     const int ktok0 = token_tile(sc, t, shifted) * kT;
     __syncthreads();
     for (int i = threadIdx.x; i < kT * D; i += kThreads) {
       const int r = i / D, c = i % D;
-      const bool in = ktok0 + r < a.S;
-      const size_t src = ((static_cast<size_t>(b) * a.S + ktok0 + r) * a.Hkv + g) * D + c;
+      const bool in = ktok0 + r < sv.len;
+      const size_t src = ((row0 + (in ? ktok0 + r : 0)) * a.Hkv + g) * D + c;
       sK[r * KP + c] = in ? a.k[src] : 0.f;
       sV[r * D + c] = in ? a.v[src] : 0.f;
     }
     __syncthreads();
     const bool diag = sc.causal && t == qt;
-    const int kv_valid = a.S - ktok0;  // keys past S (ragged last tile) are masked
 #pragma unroll 1
     for (int rr = 0; rr < kRowsPerWarp; ++rr) {
       const int r = warp * kRowsPerWarp + rr;
@@ -101,8 +108,9 @@ __global__ void __launch_bounds__(kThreads) attn_fwd_f32(const __grid_constant__
       }
       s0 *= a.scale;
       s1 *= a.scale;
-      if ((diag && lane > r) || lane >= kv_valid) s0 = -INFINITY;
-      if ((diag && lane + 32 > r) || lane + 32 >= kv_valid) s1 = -INFINITY;
+      // keys outside this visit's range [lo, hi), and after the row on the diagonal
+      if ((diag && lane > r) || lane < lo || lane >= hi) s0 = -INFINITY;
+      if ((diag && lane + 32 > r) || lane + 32 < lo || lane + 32 >= hi) s1 = -INFINITY;
       const float mx = warp_max(fmaxf(s0, s1));
       const float m_new = fmaxf(m[rr], mx);
       const float alpha = (m[rr] == -INFINITY) ? 0.f : expf(m[rr] - m_new);
@@ -126,13 +134,13 @@ __global__ void __launch_bounds__(kThreads) attn_fwd_f32(const __grid_constant__
   for (int rr = 0; rr < kRowsPerWarp; ++rr) {
     const int r = warp * kRowsPerWarp + rr;
     const int tok = qtok0 + r;
-    if (tok >= a.S) continue;
+    if (tok >= sv.len) continue;
     const float inv = l[rr] > 0.f ? 1.f / l[rr] : 0.f;
-    float* orow = a.o_out + ((static_cast<size_t>(b) * a.S + tok) * a.Hq + h) * D;
+    float* orow = a.o_out + ((row0 + tok) * a.Hq + h) * D;
 #pragma unroll
     for (int e = 0; e < E; ++e) orow[lane + 32 * e] = o[rr][e] * inv;
     if (lane == 0)
-      a.lse_out[(static_cast<size_t>(b) * a.Hq + h) * a.S + tok] =
+      a.lse_out[(static_cast<size_t>(sv.bm) * a.Hq + h) * a.S + sv.tokb + tok] =
           l[rr] > 0.f ? m[rr] + logf(l[rr]) : -INFINITY;
   }
 }
@@ -155,14 +163,21 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_f32(const __grid_constant__
   const int kt = static_cast<int>(blockIdx.x) / BG;
   const int bg = static_cast<int>(blockIdx.x) % BG;
   const int g = bg % a.Hkv, b = bg / a.Hkv;
+  SeqView sv;
+  if (!seq_view(sc, b, a.S, &sv)) {
+    if (threadIdx.x == 0 && kt == 0) record_error(kErrSeqOffsets, 161);
+    return;
+  }
+  if (kt >= sv.n_tiles) return;  // a shorter packed sequence: no work here
+  const size_t row0 = static_cast<size_t>(sv.bm) * a.S + sv.tokb;
   const bool shifted = head_shifted(sc, g * rep);
   const int ktok0 = token_tile(sc, kt, shifted) * kT;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   for (int i = threadIdx.x; i < kT * D; i += kThreads) {
     const int r = i / D, c = i % D;
-    const bool in = ktok0 + r < a.S;
-    const size_t src = ((static_cast<size_t>(b) * a.S + ktok0 + r) * a.Hkv + g) * D + c;
+    const bool in = ktok0 + r < sv.len;
+    const size_t src = ((row0 + (in ? ktok0 + r : 0)) * a.Hkv + g) * D + c;
     sK[i] = in ? a.k[src] : 0.f;
     sV[i] = in ? a.v[src] : 0.f;
   }
@@ -173,7 +188,7 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_f32(const __grid_constant__
     for (int e = 0; e < E; ++e) dk[rr][e] = dv[rr][e] = 0.f;
 
   QWalk qw;
-  qw.init(&sc, kt);
+  qw.init(&sc, kt, sv.n_tiles);
   for (int hr = 0; hr < rep; ++hr) {
     const int h = g * rep + hr;
     for (int qt = qw.t; qt < qw.t_end; ++qt) {
@@ -181,8 +196,8 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_f32(const __grid_constant__
       __syncthreads();
       for (int i = threadIdx.x; i < kT * D; i += kThreads) {
         const int r = i / D, c = i % D;
-        const bool in = qtok0 + r < a.S;
-        const size_t src = ((static_cast<size_t>(b) * a.S + qtok0 + r) * a.Hq + h) * D + c;
+        const bool in = qtok0 + r < sv.len;
+        const size_t src = ((row0 + (in ? qtok0 + r : 0)) * a.Hq + h) * D + c;
         sQ[r * P + c] = in ? a.q[src] : 0.f;
         sO[r * P + c] = in ? a.dout[src] : 0.f;
         sdQ[i] = 0.f;
@@ -235,17 +250,15 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_f32(const __grid_constant__
       __syncthreads();
       for (int i = threadIdx.x; i < kT * D; i += kThreads) {
         const int r = i / D, c = i % D;
-        if (qtok0 + r < a.S)
-          atomicAdd(&a.dq[((static_cast<size_t>(b) * a.S + qtok0 + r) * a.Hq + h) * D + c],
-                    sdQ[i]);
+        if (qtok0 + r < sv.len) atomicAdd(&a.dq[((row0 + qtok0 + r) * a.Hq + h) * D + c], sdQ[i]);
       }
     }
   }
 #pragma unroll
   for (int rr = 0; rr < kRowsPerWarp; ++rr) {
     const int j = warp * kRowsPerWarp + rr;
-    if (ktok0 + j >= a.S) continue;
-    const size_t dst = ((static_cast<size_t>(b) * a.S + ktok0 + j) * a.Hkv + g) * D;
+    if (ktok0 + j >= sv.len) continue;
+    const size_t dst = ((row0 + ktok0 + j) * a.Hkv + g) * D;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
       a.dk[dst + lane + 32 * e] = dk[rr][e] * a.scale;

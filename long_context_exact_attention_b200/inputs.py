@@ -169,6 +169,32 @@ def make_inputs(w: Workload, device="cpu", with_dout: Optional[bool] = None):
     return {n: make_tensor(w, n, device) for n in names}
 
 
+def packed_lengths(n: int, max_len: int, seed: int) -> list:
+    """Seeded lengths of ``n`` packed sequences: a mix of empty, one-token,
+    tile-multiple and ragged lengths up to ``max_len`` (the recipe of the
+    packed-batch parity cases; the pages fix no length distribution).  One
+    sequence in four takes an edge value (0, 1, 128 or max_len), the rest are
+    uniform in [1, max_len]."""
+    g = torch.Generator().manual_seed(seed * 104729 + n)
+    edges = [0, 1, min(128, max_len), max_len]
+    out = []
+    for i in range(n):
+        if int(torch.randint(4, (1,), generator=g)) == 0:
+            out.append(edges[int(torch.randint(len(edges), (1,), generator=g))])
+        else:
+            out.append(int(torch.randint(1, max_len + 1, (1,), generator=g)))
+    return out
+
+
+def packed_offsets(lengths, start: int = 0) -> list:
+    """Offsets cu[0..n] of sequences of the given lengths packed from token
+    ``start`` on."""
+    cu = [start]
+    for n in lengths:
+        cu.append(cu[-1] + int(n))
+    return cu
+
+
 def chunk_permutation(n_chunks: int, seed: int) -> list:
     """Seeded random order of ``n_chunks`` KV chunks (for order-invariance
     runs)."""

@@ -22,6 +22,7 @@ STATUS = {0: "LCA_OK", 1: "LCA_ERR_INVALID_ARG", 2: "LCA_ERR_UNSUPPORTED",
           3: "LCA_ERR_CUDA", 4: "LCA_ERR_TIMEOUT", 5: "LCA_ERR_WORKSPACE"}
 SYMBOLS = ["lca_attn_fwd", "lca_attn_bwd_workspace_size", "lca_attn_bwd",
            "lca_attn_bwd_noalloc",
+           "lca_attn_fwd_varlen", "lca_attn_bwd_varlen_workspace_size", "lca_attn_bwd_varlen",
            "lca_s2attn_fwd", "lca_s2attn_bwd", "lca_lse_merge", "lca_check",
            "lca_status_string", "lca_last_error", "lca_version"]
 
@@ -62,6 +63,12 @@ def lib() -> ctypes.CDLL:
         L.lca_attn_bwd_workspace_size.restype = ctypes.c_size_t
         L.lca_attn_bwd.argtypes = [SP, P, P, P, P, P, P, I32, P, P, P, P, ctypes.c_size_t, P]
         L.lca_attn_bwd_noalloc.argtypes = [SP, P, P, P, P, P, P, I32, P, P, P, P]
+        L.lca_attn_fwd_varlen.argtypes = [SP, P, I64, P, P, P, I32, I64, ctypes.POINTER(Opts),
+                                          P, P, P]
+        L.lca_attn_bwd_varlen_workspace_size.argtypes = [SP, I64]
+        L.lca_attn_bwd_varlen_workspace_size.restype = ctypes.c_size_t
+        L.lca_attn_bwd_varlen.argtypes = [SP, P, I64, P, P, P, P, P, P, I32, P, P, P, P,
+                                          ctypes.c_size_t, P]
         L.lca_s2attn_fwd.argtypes = [SP, P, P, P, I32, I64, I64, P, P, P]
         L.lca_s2attn_bwd.argtypes = [SP, P, P, P, P, P, P, I32, I64, I64, P, P, P, P,
                                      ctypes.c_size_t, P]
@@ -70,7 +77,7 @@ def lib() -> ctypes.CDLL:
         L.lca_status_string.restype = ctypes.c_char_p
         L.lca_last_error.restype = ctypes.c_char_p
         for fn in ("lca_attn_fwd", "lca_attn_bwd", "lca_attn_bwd_noalloc", "lca_s2attn_fwd",
-                   "lca_s2attn_bwd",
+                   "lca_s2attn_bwd", "lca_attn_fwd_varlen", "lca_attn_bwd_varlen",
                    "lca_lse_merge", "lca_check"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
@@ -117,6 +124,16 @@ def _check_tensors(dtype, *ts):
             raise ValueError(f"dtype mismatch: {t.dtype} vs {dtype}")
 
 
+def _opts(order, chunk_perm, q_block, timeout_cycles):
+    """lca_opts plus the host array it points to (keep both alive)."""
+    opts = Opts(ORDERS[order], None, int(q_block), int(timeout_cycles))
+    keep = None
+    if chunk_perm is not None:
+        keep = (ctypes.c_int32 * len(chunk_perm))(*[int(x) for x in chunk_perm])
+        opts.chunk_perm = ctypes.cast(keep, ctypes.POINTER(ctypes.c_int32))
+    return opts, keep
+
+
 def attn_fwd(q, k, v, causal: bool = True, kv_chunk: int = 0, order: str = "inorder",
              chunk_perm: Optional[Sequence[int]] = None, q_block: int = 0, scale=None,
              out=None, lse=None, stream=None, timeout_cycles: int = 0):
@@ -128,15 +145,70 @@ def attn_fwd(q, k, v, causal: bool = True, kv_chunk: int = 0, order: str = "inor
     if lse is None:
         lse = torch.empty((q.shape[0], q.shape[2], q.shape[1]), device=q.device,
                           dtype=torch.float32)
-    opts = Opts(ORDERS[order], None, int(q_block), int(timeout_cycles))
-    keep = None
-    if chunk_perm is not None:
-        keep = (ctypes.c_int32 * len(chunk_perm))(*[int(x) for x in chunk_perm])
-        opts.chunk_perm = ctypes.cast(keep, ctypes.POINTER(ctypes.c_int32))
+    opts, keep = _opts(order, chunk_perm, q_block, timeout_cycles)
     _raise(lib().lca_attn_fwd(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), int(causal),
                               int(kv_chunk), ctypes.byref(opts), _ptr(out), _ptr(lse),
                               _stream(stream)))
+    del keep
     return out, lse
+
+
+def _packed_shape(q, k, cu_seqlens, scale) -> Shape:
+    """Shape of a packed batch: q [T,Hq,d], k/v [T,Hkv,d], cu_seqlens int32
+    [n+1] on the device."""
+    if q.dim() != 3 or k.dim() != 3:
+        raise ValueError("packed q is [T,Hq,d], k/v are [T,Hkv,d]")
+    if not (q.is_cuda and k.is_cuda and cu_seqlens.is_cuda):
+        raise ValueError("lca needs CUDA tensors")
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+        raise ValueError("cu_seqlens is an int32 tensor of n + 1 offsets")
+    T, Hq, d = q.shape
+    if k.shape[0] != T or k.shape[2] != d:
+        raise ValueError("k/v shape does not match q")
+    dt = {torch.bfloat16: LCA_BF16, torch.float32: LCA_FP32}.get(q.dtype)
+    if dt is None:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    return Shape(cu_seqlens.numel() - 1, Hq, k.shape[1], T, d, dt, float(scale or 0.0))
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens, max_seqlen: int, causal: bool = True,
+                    kv_chunk: int = 0, order: str = "inorder", q_block: int = 0, scale=None,
+                    out=None, lse=None, stream=None, timeout_cycles: int = 0):
+    """Forward over a packed batch of sequences (lca_attn_fwd_varlen).
+    q [T,Hq,d], k/v [T,Hkv,d]; sequence b is rows cu_seqlens[b]:cu_seqlens[b+1].
+    Returns (out [T,Hq,d], lse [Hq,T])."""
+    sh = _packed_shape(q, k, cu_seqlens, scale)
+    _check_tensors(q.dtype, q, k, v)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((q.shape[1], q.shape[0]), device=q.device, dtype=torch.float32)
+    opts, keep = _opts(order, None, q_block, timeout_cycles)
+    _raise(lib().lca_attn_fwd_varlen(ctypes.byref(sh), _ptr(cu_seqlens), int(max_seqlen),
+                                     _ptr(q), _ptr(k), _ptr(v), int(causal), int(kv_chunk),
+                                     ctypes.byref(opts), _ptr(out), _ptr(lse), _stream(stream)))
+    del keep
+    return out, lse
+
+
+def attn_bwd_varlen(q, k, v, out, lse, dout, cu_seqlens, max_seqlen: int, causal: bool = True,
+                    scale=None, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Gradients over a packed batch (lca_attn_bwd_varlen).  Returns (dq, dk, dv)."""
+    sh = _packed_shape(q, k, cu_seqlens, scale)
+    _check_tensors(q.dtype, q, k, v, out, dout)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        n = int(lib().lca_attn_bwd_varlen_workspace_size(ctypes.byref(sh), int(max_seqlen)))
+        workspace = torch.empty(max(n, 1), device=q.device, dtype=torch.uint8)
+    _raise(lib().lca_attn_bwd_varlen(ctypes.byref(sh), _ptr(cu_seqlens), int(max_seqlen),
+                                     _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                     _ptr(dout), int(causal), _ptr(dq), _ptr(dk), _ptr(dv),
+                                     _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(),
+                                     _stream(stream)))
+    return dq, dk, dv
 
 
 def workspace_size(q, k) -> int:

@@ -68,11 +68,16 @@ def test_bad_pointers_rejected():
     assert b"aligned" in lca.lib().lca_last_error()
 
 
-@pytest.mark.parametrize("kv_chunk", [100, 200, -128])
+@pytest.mark.parametrize("kv_chunk", [-1, -128])
 def test_bad_chunks_rejected(kv_chunk):
-    # a chunk must be a whole number of tiles (the last chunk of a sequence
-    # may be partial, so it need not divide S)
     assert fwd(shape(S=512), kv_chunk=kv_chunk) == 1
+
+
+def test_chunk_count_limit():
+    # any chunk length is accepted (tiles straddling a boundary are split),
+    # up to LCA_MAX_CHUNKS chunks
+    assert fwd(shape(S=1025), kv_chunk=1) == 1
+    assert b"LCA_MAX_CHUNKS" in lca.lib().lca_last_error()
 
 
 def test_bad_permutation_rejected():
@@ -111,6 +116,39 @@ def test_workspace_errors():
     args = [ctypes.byref(sh)] + [FAKE] * 6 + [1] + [FAKE] * 3
     assert L.lca_attn_bwd(*args, None, need, None) == 5
     assert L.lca_attn_bwd(*args, FAKE, need - 1, None) == 5
+
+
+def fwd_varlen(sh, cu=FAKE, max_seqlen=128, order=0, ptrs=None):
+    p = ptrs or [FAKE] * 5
+    o = lca.Opts(order, None, 0, 0)
+    return lca.lib().lca_attn_fwd_varlen(ctypes.byref(sh), cu, max_seqlen, p[0], p[1], p[2], 1,
+                                         0, ctypes.byref(o), p[3], p[4], None)
+
+
+def test_varlen_arguments_rejected():
+    sh = shape(B=3, S=1000)             # 3 packed sequences, 1000 tokens in all
+    assert fwd_varlen(sh, cu=None) == 1
+    assert fwd_varlen(sh, cu=ctypes.c_void_p(0x10002)) == 1   # not 4-byte aligned
+    assert fwd_varlen(sh, max_seqlen=0) == 1
+    assert fwd_varlen(sh, max_seqlen=1001) == 1
+    perm = (ctypes.c_int32 * 1)(0)
+    o = lca.Opts(2, ctypes.cast(perm, ctypes.POINTER(ctypes.c_int32)), 0, 0)
+    assert lca.lib().lca_attn_fwd_varlen(ctypes.byref(sh), FAKE, 128, FAKE, FAKE, FAKE, 1, 0,
+                                         ctypes.byref(o), FAKE, FAKE, None) == 1
+    assert b"CUSTOM" in lca.lib().lca_last_error()
+    assert fwd_varlen(shape(B=3, S=1000, d=64)) == 2
+
+
+def test_varlen_workspace_size():
+    L = lca.lib()
+    sh = shape(B=3, S=1000)
+    # D rows and lse copy [3, Hq, 384] each, fp32 dq accumulator [1000, Hq, 128]
+    assert L.lca_attn_bwd_varlen_workspace_size(ctypes.byref(sh), 300) == \
+        2 * 4 * 3 * 4 * 384 + 4 * 1000 * 4 * 128
+    assert L.lca_attn_bwd_varlen_workspace_size(ctypes.byref(sh), 0) == 0
+    assert L.lca_attn_bwd_varlen_workspace_size(ctypes.byref(sh), 1001) == 0
+    args = [ctypes.byref(sh), FAKE, 300] + [FAKE] * 6 + [1] + [FAKE] * 3
+    assert L.lca_attn_bwd_varlen(*args, None, 1 << 30, None) == 5
 
 
 def test_merge_arguments_rejected():

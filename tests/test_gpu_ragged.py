@@ -1,6 +1,7 @@
-"""Ragged sequence lengths: S not a multiple of the tile (the last query and
-key tiles are partial) and a last key/value chunk shorter than the others,
-forward and backward, bf16 and fp32, against the fp64 oracle in full."""
+"""Ragged tails: S not a multiple of the tile (the last query and key tiles
+are partial), a last key/value chunk shorter than the others, and chunk
+lengths that are not a multiple of the tile; forward and backward, bf16 and
+fp32, against the fp64 oracle in full."""
 
 import pytest
 import torch
@@ -64,3 +65,37 @@ def test_ragged_outputs_leave_neighbours_untouched():
     torch.cuda.synchronize()
     assert torch.isfinite(out.float()).all()
     assert torch.isnan(big[400:].float()).all()
+
+
+@pytest.mark.parametrize("S,causal,kv_chunk,order,q_block", [
+    (1000, True, 300, "ring", 0),
+    (1000, False, 300, "inorder", 0),
+    (333, True, 50, "ring", 100),
+    (130, True, 1, "ring", 0),          # one key per chunk: 130 visits per query tile
+    (640, False, 129, "custom", 0),
+])
+def test_bf16_unaligned_chunks(S, causal, kv_chunk, order, q_block):
+    """kv_chunk not a multiple of the tile: tiles straddling a chunk boundary
+    are visited once per chunk, each visit masked to its chunk's keys."""
+    w = shrink(WORKLOADS["llama2_7b_s32k"], S=S, B=1, Hq=2, Hkv=1, causal=causal, rope=False,
+               seed=91 + kv_chunk)
+    x = device_inputs(w, with_dout=False)
+    perm = chunk_permutation(-(-S // kv_chunk), 5) if order == "custom" else None
+    out, lse = lca.attn_fwd(x["q"], x["k"], x["v"], causal=causal, kv_chunk=kv_chunk,
+                            order=order, chunk_perm=perm, q_block=q_block)
+    torch.cuda.synchronize()
+    lca.check()
+    ro, rl = oracle.attention_forward(x["q"], x["k"], x["v"], causal)
+    assert_fwd_close(host(out), host(lse), ro, rl)
+
+
+@pytest.mark.parametrize("S,kv_chunk,order", [(200, 37, "ring"), (150, 64, "custom")])
+def test_fp32_unaligned_chunks(S, kv_chunk, order):
+    w = shrink(WORKLOADS["tiny_fp32_s256"], S=S, B=1, Hq=2, Hkv=2, causal=True, seed=97)
+    x = device_inputs(w, with_dout=False)
+    perm = chunk_permutation(-(-S // kv_chunk), 7) if order == "custom" else None
+    out, lse = lca.attn_fwd(x["q"], x["k"], x["v"], causal=True, kv_chunk=kv_chunk,
+                            order=order, chunk_perm=perm)
+    torch.cuda.synchronize()
+    ro, rl = oracle.attention_forward(x["q"], x["k"], x["v"], True)
+    assert_fwd_close(host(out), host(lse), ro, rl, fp32=True)
