@@ -165,8 +165,12 @@ def oracle_sample(w, seconds_target=12.0, max_rows=None):
     import oracle
     from long_context_exact_attention_b200.inputs import make_tensor
 
-    S = w.S
-    tok = (0, S)
+    tok = (0, w.S)
+    if w.packed:
+        # a packed batch: the longest sequence, as a dense problem of its own
+        i = max(range(len(w.lengths)), key=lambda j: w.lengths[j])
+        tok = (sum(w.lengths[:i]), sum(w.lengths[:i + 1]))
+    S = tok[1] - tok[0]
     q = make_tensor(w, "q", "cpu", tok)[:, :, :w.Hq // w.Hkv]
     k = make_tensor(w, "k", "cpu", tok)[:, :, :1]
     v = make_tensor(w, "v", "cpu", tok)[:, :, :1]
@@ -249,16 +253,32 @@ def main():
     torch.cuda.synchronize()
     q, k, v = x["q"], x["k"], x["v"]
     dout = x.get("dout")
+    if w.packed:
+        # one token axis: [T, H, d] views of the single batch entry
+        q, k, v = q[0], k[0], v[0]
+        dout = dout[0] if dout is not None else None
+        cu = torch.tensor([0] + list(__import__("itertools").accumulate(w.lengths)),
+                          dtype=torch.int32, device=dev)
+        max_len = max(w.lengths)
     out = torch.empty_like(q)
-    lse = torch.empty((w.B, w.Hq, w.S), device=dev, dtype=torch.float32)
+    lse = torch.empty((w.Hq, w.S) if w.packed else (w.B, w.Hq, w.S), device=dev,
+                      dtype=torch.float32)
     if w.backward:
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-        ws = torch.empty(lca.workspace_size(q, k), device=dev, dtype=torch.uint8)
+        ws = None if w.packed else torch.empty(lca.workspace_size(q, k), device=dev,
+                                               dtype=torch.uint8)
+        if w.packed:
+            ws = torch.empty(lca.varlen_workspace_size(q, k, cu, max_len), device=dev,
+                             dtype=torch.uint8)
 
     def step(ev=None):
         if ev:
             ev[0].record(stream)
-        if w.s2:
+        if w.packed:
+            lca.attn_fwd_varlen(q, k, v, cu, max_len, causal=w.causal, kv_chunk=w.kv_chunk,
+                                order=w.order, q_block=w.q_block, out=out, lse=lse,
+                                stream=stream)
+        elif w.s2:
             lca.s2attn_fwd(q, k, v, w.group, w.shift_heads, causal=w.causal, out=out, lse=lse,
                            stream=stream)
         else:
@@ -266,7 +286,10 @@ def main():
                          q_block=w.q_block, out=out, lse=lse, stream=stream)
         if ev:
             ev[1].record(stream)
-        if w.backward and w.s2:
+        if w.backward and w.packed:
+            lca.attn_bwd_varlen(q, k, v, out, lse, dout, cu, max_len, causal=w.causal, dq=dq,
+                                dk=dk, dv=dv, workspace=ws, stream=stream)
+        elif w.backward and w.s2:
             lca.s2attn_bwd(q, k, v, out, lse, dout, w.group, w.shift_heads, causal=w.causal,
                            dq=dq, dk=dk, dv=dv, workspace=ws, stream=stream)
         elif w.backward:
@@ -350,6 +373,9 @@ def main():
     if rank != 0:
         return
 
+    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v, dout) if t is not None)
+    l2_note = (f"inputs larger than L2 (q, k, v{', dout' if dout is not None else ''} "
+               f"{in_bytes / 2**20:.0f} MiB together, L2 126 MB); no flush")
     pk, pk_kind = peaks()
     sustained = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     fwd_t = statistics.median(fwd_ms)
@@ -376,8 +402,9 @@ def main():
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "S": w.S, "d": w.d,
                    "causal": w.causal, "kv_chunk": w.kv_chunk, "order": w.order,
                    "s2_group": w.group or None, "s2_shift_heads": w.shift_heads or None,
+                   "packed_lengths": list(w.lengths) or None,
                    "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (q, k, v, dout 256 MiB each); no flush"},
+                   "l2": l2_note},
         "fwd_tflops": w.fwd_flops() / (fwd_t * 1e-3) / 1e12, "fwd_ms": fwd_t,
         "bwd_tflops": (w.bwd_flops() / (bwd_t * 1e-3) / 1e12) if w.backward else None,
         "bwd_ms": bwd_t if w.backward else None,

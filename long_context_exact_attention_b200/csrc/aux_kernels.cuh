@@ -29,10 +29,19 @@ __global__ void bwd_rowdot(const T* __restrict__ out, const T* __restrict__ dout
                            const int* __restrict__ cu_seqlens) {
   const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (w >= static_cast<int64_t>(B) * S_pad * H) return;
-  const int h = static_cast<int>(w % H);
-  const int s = static_cast<int>((w / H) % S_pad);
-  const int b = static_cast<int>(w / (static_cast<int64_t>(H) * S_pad));
+  const int64_t n = static_cast<int64_t>(B) * S_pad * H;
+  if (w >= n) return;
+  int h, s, b;
+  if (n <= 0xffffffffll) {  // 32-bit index arithmetic when it fits
+    const uint32_t w32 = static_cast<uint32_t>(w), hs = static_cast<uint32_t>(H) * S_pad;
+    h = static_cast<int>(w32 % static_cast<uint32_t>(H));
+    s = static_cast<int>((w32 / static_cast<uint32_t>(H)) % static_cast<uint32_t>(S_pad));
+    b = static_cast<int>(w32 / hs);
+  } else {
+    h = static_cast<int>(w % H);
+    s = static_cast<int>((w / H) % S_pad);
+    b = static_cast<int>(w / (static_cast<int64_t>(H) * S_pad));
+  }
   int64_t r0 = static_cast<int64_t>(b) * S, l0 = (static_cast<int64_t>(b) * H + h) * S;
   int len = S;
   if (cu_seqlens) {

@@ -10,11 +10,12 @@
 //   dQ^T = K^T dS^T -> added into the fp32 dq accumulator by TMA bulk
 //                      reduce-add (scale applied later)
 // Ragged and packed sequences: the rows of the last tile past the end of a
-// sequence load whatever follows it (zeros past the tensor's end, or the
-// next packed sequence).  Their lse copy is +inf, so P and dS vanish in
-// those query columns, and key rows past the end get P = 0; their dK/dV are
-// not stored.  The dQ^T columns of such query rows are exact zeros, so their
-// reduce-adds leave the next sequence's accumulator unchanged.
+// sequence load whatever follows it on the flattened token axis (the next
+// batch entry or packed sequence, zeros past the tensor's end).  Query rows
+// there have an lse copy of +inf, so P and dS vanish in their columns and
+// their dQ^T columns are exact zeros (the reduce-adds leave the following
+// rows' accumulator unchanged); key rows there get an exponent of -inf, so
+// P = 0 and dS = 0, and their dK/dV are not stored.
 //
 // One CTA per (key tile of 128, key/value head, batch); it loops over the
 // query heads of its grouped-query group and over the query tiles that can
@@ -199,11 +200,11 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmDO);
       mbar_expect_tx(bar(B_KV), 2 * kTileB);
-      const int ktok = sv.tokb + ktok0;
-      tma_load_4d(sK, &tmK, bar(B_KV), 0, g, ktok, sv.bm);
-      tma_load_4d(sK + kHalf, &tmK, bar(B_KV), 64, g, ktok, sv.bm);
-      tma_load_4d(sV, &tmV, bar(B_KV), 0, g, ktok, sv.bm);
-      tma_load_4d(sV + kHalf, &tmV, bar(B_KV), 64, g, ktok, sv.bm);
+      const int ktok = sv.row0 + ktok0;
+      tma_load_3d(sK, &tmK, bar(B_KV), 0, g, ktok);
+      tma_load_3d(sK + kHalf, &tmK, bar(B_KV), 64, g, ktok);
+      tma_load_3d(sV, &tmV, bar(B_KV), 0, g, ktok);
+      tma_load_3d(sV + kHalf, &tmV, bar(B_KV), 64, g, ktok);
       bool ok = true;
       int issued0 = 0, issued1 = 0, o_issued = 0;
       for (int i = 0; i < nsteps && ok; ++i) {
@@ -215,8 +216,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         if (!ok) break;
         const uint32_t fb = bar(B_QFULL + st);
         mbar_expect_tx(fb, kTileB + 1024);
-        tma_load_4d(sQ + st * kTileB, &tmQ, fb, 0, h, sv.tokb + qtok0, sv.bm);
-        tma_load_4d(sQ + st * kTileB + kHalf, &tmQ, fb, 64, h, sv.tokb + qtok0, sv.bm);
+        tma_load_3d(sQ + st * kTileB, &tmQ, fb, 0, h, sv.row0 + qtok0);
+        tma_load_3d(sQ + st * kTileB + kHalf, &tmQ, fb, 64, h, sv.row0 + qtok0);
         const size_t ro = (static_cast<size_t>(b) * a.Hq + h) * a.S_pad + qtok0;
         bulk_load(sL + st * 512, a.lse + ro, 512, fb);
         bulk_load(sD + st * 512, a.Drow + ro, 512, fb);
@@ -224,8 +225,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         if (i >= 1) ok = wait_bar(bar(B_OEMPTY), (i - 1) & 1, wc, 112);
         if (!ok) break;
         mbar_expect_tx(bar(B_OFULL), kTileB);
-        tma_load_4d(sO, &tmDO, bar(B_OFULL), 0, h, sv.tokb + qtok0, sv.bm);
-        tma_load_4d(sO + kHalf, &tmDO, bar(B_OFULL), 64, h, sv.tokb + qtok0, sv.bm);
+        tma_load_3d(sO, &tmDO, bar(B_OFULL), 0, h, sv.row0 + qtok0);
+        tma_load_3d(sO + kHalf, &tmDO, bar(B_OFULL), 64, h, sv.row0 + qtok0);
         ++o_issued;
       }
       if (!ok) {
@@ -323,6 +324,9 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     const float L2E = 1.4426950408889634f;
     const uint64_t c2 = f2_pack(c, c);
     const bool key_out = ktok0 + r >= sv.len;  // key row past the sequence's end
+    // added to every exponent of this key row: -inf gives P = 0 (hence dS =
+    // 0, and the row adds nothing to dQ) for a key row past the end
+    const float kill = key_out ? -INFINITY : 0.f;
     bool ok = true;
     for (int i = 0; i < nsteps && ok; ++i) {
       const int st = i & 1;
@@ -344,7 +348,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 64; e += 2) {
           const int q0 = hq * 64 + e;
-          const uint64_t nl = f2_pack(-lse_r[e] * L2E, -lse_r[e + 1] * L2E);
+          const uint64_t nl =
+              f2_pack(fmaf(-lse_r[e], L2E, kill), fmaf(-lse_r[e + 1], L2E, kill));
           float p0, p1;
           f2_unpack(f2_fma(f2_pack(p[e], p[e + 1]), c2, nl), p0, p1);
           p0 = ex2_approx(p0);
@@ -354,12 +359,6 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
           p[e] = p0;
           p[e + 1] = p1;
           pk[e >> 1] = pack_bf16x2(p0, p1);
-        }
-        if (key_out) {
-#pragma unroll
-          for (int e = 0; e < 64; ++e) p[e] = 0.f;
-#pragma unroll
-          for (int e = 0; e < 32; ++e) pk[e] = 0u;
         }
         tmem_st32u(tmem + lad + hq * 64, pk);
       }
@@ -385,10 +384,6 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
           f2_unpack(t, t0, t1);
           dd[e >> 1] = pack_bf16x2(p[ql] * t0, p[ql + 1] * t1);
         }
-        if (key_out) {  // P = 0 there; keep dS = 0 whatever dP holds
-#pragma unroll
-          for (int e = 0; e < 16; ++e) dd[e] = 0u;
-        }
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
           const int cw = cc * 4 + v;  // 16-byte chunk within this half's 128-byte row
@@ -407,8 +402,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     // past the sequence's end (ragged last tile) only skip their stores
     if (ok) {
       tc_fence_after();
-      const size_t trow =
-          static_cast<size_t>(sv.bm) * a.S + sv.tokb + (key_out ? 0 : ktok0 + r);
+      const size_t trow = static_cast<size_t>(sv.row0) + (key_out ? 0 : ktok0 + r);
       __nv_bfloat16* row = a.dk + (trow * a.Hkv + g) * kD;
 #pragma unroll 1
       for (int cc = 2 * hq; cc < 2 * hq + 2; ++cc) {
@@ -464,8 +458,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         fence_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_reduce_add_4d(&tmDQ, sR + wq * 8192, wq * 32, h, sv.tokb + qtok0 + half * 64,
-                            sv.bm);
+          tma_reduce_add_3d(&tmDQ, sR + wq * 8192, wq * 32, h, sv.row0 + qtok0 + half * 64);
           bulk_commit();
         }
       }
@@ -478,7 +471,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     const bool row_in = ktok0 + r < sv.len;
     if (ok) {
       tc_fence_after();
-      const size_t trow = static_cast<size_t>(sv.bm) * a.S + sv.tokb + (row_in ? ktok0 + r : 0);
+      const size_t trow = static_cast<size_t>(sv.row0) + (row_in ? ktok0 + r : 0);
       __nv_bfloat16* row = a.dv + (trow * a.Hkv + g) * kD;
 #pragma unroll 1
       for (int cc = 0; cc < 4; ++cc) {

@@ -30,6 +30,8 @@
 // Each 128x128 bf16 tile is two 16 KB halves (head dims 0-63, 64-127).
 #pragma once
 
+#include <type_traits>
+
 #include "ptx.cuh"
 #include "sched.cuh"
 
@@ -83,14 +85,35 @@ __device__ __forceinline__ int tile_vis(bool causal, int Q, int T) {
   return T < Q ? VIS_FULL : (T == Q ? VIS_DIAG : VIS_NONE);
 }
 
+// One interface over the two walks: KvWalk (chunk boundaries anywhere; each
+// visit carries its key range [lo, hi)) and TileWalk (chunks of whole
+// tiles; lo and hi are left alone).
+__device__ __forceinline__ void walk_init(KvWalk& w, const AttnSched* s, int qt,
+                                          const SeqView& v) {
+  w.init(s, qt, v.len);
+}
+__device__ __forceinline__ void walk_init(TileWalk& w, const AttnSched* s, int qt,
+                                          const SeqView& v) {
+  w.init(s, qt, v.n_tiles);
+}
+__device__ __forceinline__ bool walk_next(KvWalk& w, int& t, int& lo, int& hi) {
+  return w.next(t, lo, hi);
+}
+__device__ __forceinline__ bool walk_next(TileWalk& w, int& t, int&, int&) { return w.next(t); }
+
 }  // namespace fwd
 
+// kRanged: some chunk boundary falls inside a tile, so visits carry key
+// ranges (KvWalk).  Otherwise the cheaper tile walk runs and only a ragged
+// last tile needs a key mask.
+template <bool kRanged>
 __global__ void __launch_bounds__(fwd::kThreads, 1)
     attn_fwd_bf16_sm100(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV,
                         const __grid_constant__ fwd::Args a) {
   using namespace fwd;
+  using Walk = typename std::conditional<kRanged, KvWalk, TileWalk>::type;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -100,6 +123,9 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
   auto bar = [&](int i) { return bars + 8u * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kOffBar + 8 * NUM_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + kOffBar + 8 * NUM_BARS + 8);
+  // The sequence's length, first row and lse offset, parked in shared
+  // memory (re-read where needed rather than held through the softmax loop)
+  const uint32_t seq_smem = bars + 8 * NUM_BARS + 16;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -132,6 +158,11 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       mbar_init(bar(i), cnt);
     }
     *abort_flag = 0;
+    int* si = reinterpret_cast<int*>(gbase + kOffBar + 8 * NUM_BARS + 16);
+    si[0] = sv.len;
+    si[1] = sv.row0;
+    *reinterpret_cast<long long*>(si + 2) =
+        (static_cast<long long>(sv.bm) * a.Hq + h) * a.S + sv.tokb;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -152,29 +183,29 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       tma_prefetch_desc(&tmV);
       mbar_expect_tx(bar(B_Q), has1 ? 2 * kTileB : kTileB);
       for (int t = 0; t < (has1 ? 2 : 1); ++t) {
-        const int tok = sv.tokb + token_tile(sc, qt0 + t, shifted) * kTile;
-        tma_load_4d(sQ + t * kTileB, &tmQ, bar(B_Q), 0, h, tok, sv.bm);
-        tma_load_4d(sQ + t * kTileB + kHalf, &tmQ, bar(B_Q), 64, h, tok, sv.bm);
+        const int tok = sv.row0 + token_tile(sc, qt0 + t, shifted) * kTile;
+        tma_load_3d(sQ + t * kTileB, &tmQ, bar(B_Q), 0, h, tok);
+        tma_load_3d(sQ + t * kTileB + kHalf, &tmQ, bar(B_Q), 64, h, tok);
       }
-      KvWalk w;
-      w.init(&sc, qt_last, sv.len);
-      int t, lo, hi, j = 0;
+      Walk w;
+      walk_init(w, &sc, qt_last, sv);
+      int t, lo = 0, hi = kTile, j = 0;
       int k_issued0 = 0, k_issued1 = 0, v_issued0 = 0, v_issued1 = 0;
       bool ok = true;
-      while (ok && w.next(t, lo, hi)) {
+      while (ok && walk_next(w, t, lo, hi)) {
         const int st = j & 1;
-        const int tok = sv.tokb + token_tile(sc, t, shifted) * kTile;
+        const int tok = sv.row0 + token_tile(sc, t, shifted) * kTile;
         if (j >= 2) ok = wait_bar(bar(B_KEMPTY + st), ((j - 2) >> 1) & 1, wc, 101);
         if (!ok) break;
         mbar_expect_tx(bar(B_KFULL + st), kTileB);
-        tma_load_4d(sK + st * kTileB, &tmK, bar(B_KFULL + st), 0, g, tok, sv.bm);
-        tma_load_4d(sK + st * kTileB + kHalf, &tmK, bar(B_KFULL + st), 64, g, tok, sv.bm);
+        tma_load_3d(sK + st * kTileB, &tmK, bar(B_KFULL + st), 0, g, tok);
+        tma_load_3d(sK + st * kTileB + kHalf, &tmK, bar(B_KFULL + st), 64, g, tok);
         if (st) ++k_issued1; else ++k_issued0;
         if (j >= 2) ok = wait_bar(bar(B_VEMPTY + st), ((j - 2) >> 1) & 1, wc, 102);
         if (!ok) break;
         mbar_expect_tx(bar(B_VFULL + st), kTileB);
-        tma_load_4d(sV + st * kTileB, &tmV, bar(B_VFULL + st), 0, g, tok, sv.bm);
-        tma_load_4d(sV + st * kTileB + kHalf, &tmV, bar(B_VFULL + st), 64, g, tok, sv.bm);
+        tma_load_3d(sV + st * kTileB, &tmV, bar(B_VFULL + st), 0, g, tok);
+        tma_load_3d(sV + st * kTileB + kHalf, &tmV, bar(B_VFULL + st), 64, g, tok);
         if (st) ++v_issued1; else ++v_issued0;
         ++j;
       }
@@ -192,9 +223,9 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     if (lane == 0) {
       const uint32_t qts[2] = {static_cast<uint32_t>(qt0), static_cast<uint32_t>(qt0 + 1)};
       bool ok = wait_bar(bar(B_Q), 0, wc, 201);
-      KvWalk w;
-      w.init(&sc, qt_last, sv.len);
-      int T, Tn, lo, hi;
+      Walk w;
+      walk_init(w, &sc, qt_last, sv);
+      int T, Tn, lo = 0, hi = kTile;
       int pv_cnt[2] = {0, 0};
       // S_t for key tile j into the S/P columns of query tile t
       auto issue_s = [&](int tq, int j) {
@@ -211,7 +242,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       auto act = [&](int tq, int T_) {
         return (tq == 0 || has1) && tile_vis(causal, static_cast<int>(qts[tq]), T_) != VIS_NONE;
       };
-      bool have = ok && w.next(T, lo, hi);
+      bool have = ok && walk_next(w, T, lo, hi);
       if (have) {
         ok = wait_bar(bar(B_KFULL), 0, wc, 202);
         if (ok) {
@@ -223,7 +254,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       }
       int j = 0;
       while (ok && have) {
-        const bool has_next = w.next(Tn, lo, hi);
+        const bool has_next = walk_next(w, Tn, lo, hi);
         ok = wait_bar(bar(B_VFULL + (j & 1)), (j >> 1) & 1, wc, 203);
         if (ok && has_next) ok = wait_bar(bar(B_KFULL + ((j + 1) & 1)), ((j + 1) >> 1) & 1, wc, 204);
         for (int tq = 0; tq < 2 && ok; ++tq) {
@@ -268,10 +299,10 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     int cnt = 0;
     bool ok = true;
     if (tq == 0 || has1) {
-      KvWalk w;
-      w.init(&sc, qt_last, sv.len);
-      int t, lo, hi;
-      while (ok && w.next(t, lo, hi)) {
+      Walk w;
+      walk_init(w, &sc, qt_last, sv);
+      int t, lo = 0, hi = kTile;
+      while (ok && walk_next(w, t, lo, hi)) {
         const int vis = tile_vis(causal, qt, t);
         if (vis == VIS_NONE) continue;
         ok = __all_sync(0xffffffffu, wait_bar(bar(B_SFULL + tq), cnt & 1, wc, 301));
@@ -279,10 +310,10 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         tc_fence_after();
         float s[128];
         tmem_ld128(tS, s);
-        // Keys outside this visit's range [lo, hi) -- another chunk's keys
-        // in a tile that straddles a chunk boundary, or rows past the end
-        // of the sequence -- and, on the diagonal, keys after the row.
-        {
+        if constexpr (kRanged) {
+          // Keys outside this visit's range [lo, hi) -- another chunk's keys
+          // in a tile that straddles a chunk boundary, or rows past the end
+          // of the sequence -- and, on the diagonal, keys after the row.
           const int lim = vis == VIS_DIAG ? (hi < r + 1 ? hi : r + 1) : hi;
           if (lim < kTile) {
 #pragma unroll
@@ -293,6 +324,21 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 128; ++i)
               if (i < lo) s[i] = -INFINITY;
+          }
+        } else if (vis == VIS_DIAG) {
+          // keys after the row (past the end of a ragged sequence included,
+          // for every row that is stored)
+#pragma unroll
+          for (int i = 0; i < 128; ++i)
+            if (i > r) s[i] = -INFINITY;
+        } else if (t == w.n_tiles - 1) {
+          // last key tile of a ragged sequence: rows past its end (S2-Attn
+          // sequences are whole tiles, so nothing is masked there)
+          const int kv_valid = ld_shared_volatile_s32(seq_smem) - t * kTile;
+          if (kv_valid < kTile) {
+#pragma unroll
+            for (int i = 0; i < 128; ++i)
+              if (i >= kv_valid) s[i] = -INFINITY;
           }
         }
         // Row max: eight independent chains of 3-input max.
@@ -361,8 +407,9 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       const int tok = token_tile(sc, qt, shifted) * kTile + r;
       // Every lane takes part in the TMEM loads (warp-collective); rows past
       // the end of the sequence (ragged last tile) only skip their stores.
-      const bool row_in = tok < sv.len;
-      const size_t trow = static_cast<size_t>(sv.bm) * a.S + sv.tokb + (row_in ? tok : 0);
+      const bool row_in = tok < ld_shared_volatile_s32(seq_smem);
+      const size_t trow =
+          static_cast<size_t>(ld_shared_volatile_s32(seq_smem + 4)) + (row_in ? tok : 0);
       if (ok) {
         tc_fence_after();
         const float inv = (l_run > 0.f) ? 1.0f / l_run : 0.f;
@@ -386,8 +433,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         }
         const float lse = (l_run > 0.f) ? (m_run + lg2_approx(l_run)) * 0.69314718055994531f
                                         : -INFINITY;
-        if (row_in)
-          a.lse[(static_cast<size_t>(sv.bm) * a.Hq + h) * a.S + sv.tokb + tok] = lse;
+        if (row_in) a.lse[ld_shared_volatile_s64(seq_smem + 8) + tok] = lse;
       }
     }
   }

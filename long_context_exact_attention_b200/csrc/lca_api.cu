@@ -204,19 +204,19 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [B][S][heads][128] bf16 viewed 4-D (head dim, head, token, batch); box =
-// 64 head dims x 1 head x 128 tokens x 1 batch.  Token rows past S (ragged
-// last tile) load as zeros.
+// [B][S][heads][128] bf16 viewed 3-D (head dim, head, token on the flattened
+// axis of all B*S rows); box = 64 head dims x 1 head x 128 tokens.  Rows
+// past the last token load as zeros; a ragged tile otherwise reads the
+// following batch entry's rows, which the kernels mask.
 lca_status make_map(CUtensorMap* m, const void* ptr, int64_t B, int64_t S, int64_t heads) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(LCA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-  const cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(heads), static_cast<cuuint64_t>(S),
-                              static_cast<cuuint64_t>(B)};
-  const cuuint64_t strides[3] = {128 * 2, static_cast<cuuint64_t>(heads) * 128 * 2,
-                                 static_cast<cuuint64_t>(S) * heads * 128 * 2};
-  const cuuint32_t box[4] = {64, 1, 128, 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims,
+  const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(heads),
+                              static_cast<cuuint64_t>(B * S)};
+  const cuuint64_t strides[2] = {128 * 2, static_cast<cuuint64_t>(heads) * 128 * 2};
+  const cuuint32_t box[3] = {64, 1, 128};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -224,19 +224,18 @@ lca_status make_map(CUtensorMap* m, const void* ptr, int64_t B, int64_t S, int64
   return LCA_OK;
 }
 
-// fp32 [B][S][heads][128] accumulator viewed 4-D; box = 32 head dims x 1
-// head x 64 tokens x 1 batch, no swizzle (the box's rows are 128 bytes);
-// reduce-adds of rows past S are dropped.
+// fp32 [B][S][heads][128] accumulator viewed 3-D like make_map; box = 32
+// head dims x 1 head x 64 tokens, no swizzle (the box's rows are 128 bytes);
+// reduce-adds of rows past the last token are dropped.
 lca_status make_map_acc(CUtensorMap* m, const void* ptr, int64_t B, int64_t S, int64_t heads) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(LCA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-  const cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(heads), static_cast<cuuint64_t>(S),
-                              static_cast<cuuint64_t>(B)};
-  const cuuint64_t strides[3] = {128 * 4, static_cast<cuuint64_t>(heads) * 128 * 4,
-                                 static_cast<cuuint64_t>(S) * heads * 128 * 4};
-  const cuuint32_t box[4] = {32, 1, 64, 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(ptr), dims,
+  const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(heads),
+                              static_cast<cuuint64_t>(B * S)};
+  const cuuint64_t strides[2] = {128 * 4, static_cast<cuuint64_t>(heads) * 128 * 4};
+  const cuuint32_t box[3] = {32, 1, 64};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims,
                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -305,7 +304,13 @@ lca_status run_fwd(const Common& c, const AttnSched& s, const void* q, const voi
     if ((r = make_map(&mq, q, c.B, c.S, c.Hq)) != LCA_OK) return r;
     if ((r = make_map(&mk, k, c.B, c.S, c.Hkv)) != LCA_OK) return r;
     if ((r = make_map(&mv, v, c.B, c.S, c.Hkv)) != LCA_OK) return r;
-    if ((r = ensure_smem(attn_fwd_bf16_sm100, fwd::kSmemBytes, 0)) != LCA_OK) return r;
+    // chunk boundaries inside a tile need the ranged walk
+    const bool ranged = !s.s2 && s.kv_chunk % c.tile != 0;
+    if (ranged) {
+      if ((r = ensure_smem(attn_fwd_bf16_sm100<true>, fwd::kSmemBytes, 6)) != LCA_OK) return r;
+    } else {
+      if ((r = ensure_smem(attn_fwd_bf16_sm100<false>, fwd::kSmemBytes, 0)) != LCA_OK) return r;
+    }
     fwd::Args a;
     a.B = c.n_seq;
     a.Hq = c.Hq;
@@ -316,7 +321,10 @@ lca_status run_fwd(const Common& c, const AttnSched& s, const void* q, const voi
     a.out = static_cast<__nv_bfloat16*>(out);
     a.lse = lse;
     a.sched = s;
-    attn_fwd_bf16_sm100<<<grid2, fwd::kThreads, fwd::kSmemBytes, st>>>(mq, mk, mv, a);
+    if (ranged)
+      attn_fwd_bf16_sm100<true><<<grid2, fwd::kThreads, fwd::kSmemBytes, st>>>(mq, mk, mv, a);
+    else
+      attn_fwd_bf16_sm100<false><<<grid2, fwd::kThreads, fwd::kSmemBytes, st>>>(mq, mk, mv, a);
     return launched("attn_fwd_bf16_sm100");
   }
   f32::Args a{};

@@ -57,10 +57,12 @@ __host__ __device__ inline int token_tile(const AttnSched& s, int t, bool shifte
 }
 
 // Where sequence b lives in the tensors: tensor coordinates (batch index bm,
-// first token tokb) and its length.  S_tensor is the token extent of one
-// batch entry of the tensors (the packed length for packed sequences).
+// first token tokb), its first row on the flattened token axis of all batch
+// entries (row0 = bm * S_tensor + tokb) and its length.  S_tensor is the
+// token extent of one batch entry of the tensors (the packed length for
+// packed sequences).
 struct SeqView {
-  int bm, tokb, len, n_tiles;
+  int bm, tokb, row0, len, n_tiles;
 };
 
 // False when packed offsets are out of order or out of range (the caller
@@ -69,6 +71,7 @@ __host__ __device__ inline bool seq_view(const AttnSched& s, int b, int S_tensor
   if (!s.cu_seqlens) {
     v->bm = b;
     v->tokb = 0;
+    v->row0 = b * S_tensor;
     v->len = s.S;
     v->n_tiles = s.n_tiles;
     return true;
@@ -77,6 +80,7 @@ __host__ __device__ inline bool seq_view(const AttnSched& s, int b, int S_tensor
   if (c0 < 0 || c1 < c0 || c1 > S_tensor || c1 - c0 > s.S) return false;
   v->bm = 0;
   v->tokb = c0;
+  v->row0 = c0;
   v->len = c1 - c0;
   v->n_tiles = (v->len + s.tile - 1) / s.tile;
   return true;
@@ -104,7 +108,7 @@ struct KvWalk {
       // keys past the query tile's last row are invisible under the mask
       key_end = len;
       if (s->causal && (qt + 1) * s->tile < key_end) key_end = (qt + 1) * s->tile;
-      qb = static_cast<int>(static_cast<int64_t>(qt) * s->tile / s->q_block);
+      qb = qt * s->tile / s->q_block;
     }
   }
   __host__ __device__ int chunk_at(int i) const {
@@ -142,6 +146,59 @@ struct KvWalk {
     const int k0 = tile * s->tile;
     lo = c_lo > k0 ? c_lo - k0 : 0;
     hi = c_hi - k0 < s->tile ? c_hi - k0 : s->tile;
+    return true;
+  }
+};
+
+// The same walk when every chunk is a whole number of tiles: no visit is
+// split, so it yields tiles only (the forward kernel's fast path; a ragged
+// last tile is masked there from the sequence length).  Visits the same
+// tiles in the same order as KvWalk for such chunks.
+struct TileWalk {
+  const AttnSched* s;
+  int qt, n_tiles, tpc, n_chunks, ci, t, t_end, qb;
+
+  __host__ __device__ void init(const AttnSched* sc, int qt_, int n_tiles_) {
+    s = sc;
+    qt = qt_;
+    n_tiles = n_tiles_;
+    ci = 0;
+    if (s->s2) {
+      const int g0 = (qt / s->group_tiles) * s->group_tiles;
+      t = g0;
+      t_end = s->causal ? qt + 1 : g0 + s->group_tiles;
+    } else {
+      t = t_end = 0;
+      tpc = s->kv_chunk / s->tile;
+      n_chunks = (n_tiles + tpc - 1) / tpc;
+      qb = qt * s->tile / s->q_block;
+    }
+  }
+  __host__ __device__ int chunk_at(int i) const {
+    if (s->order == LCA_ORDER_RING) {
+      const int n = n_chunks;
+      return ((qb - i) % n + n) % n;
+    }
+    if (s->order == LCA_ORDER_CUSTOM) return s->perm[i];
+    return i;
+  }
+  __host__ __device__ bool next(int& tile) {
+    if (s->s2) {
+      if (t < t_end) {
+        tile = t++;
+        return true;
+      }
+      return false;
+    }
+    while (t >= t_end) {
+      if (ci >= n_chunks) return false;
+      const int c = chunk_at(ci++);
+      t = c * tpc;
+      t_end = t + tpc;
+      if (t_end > n_tiles) t_end = n_tiles;
+      if (s->causal && t_end > qt + 1) t_end = qt + 1;
+    }
+    tile = t++;
     return true;
   }
 };

@@ -40,6 +40,8 @@ class Workload:
     Layout: q/out/dout are [B, S, Hq, d]; k/v are [B, S, Hkv, d]; lse is
     [B, Hq, S].  ``kv_chunk`` is the KV chunk length of the simulated ring;
     ``group``/``shift_heads`` select LongLoRA's shifted sparse attention.
+    ``lengths`` makes it a packed batch: B = 1, S = sum(lengths) tokens on
+    one axis, sequence i holding the next lengths[i] of them.
     """
 
     name: str
@@ -59,6 +61,7 @@ class Workload:
     group: int = 0             # S2-Attn group size (0: not S2)
     shift_heads: int = 0       # S2-Attn: trailing heads shifted by group/2
     backward: bool = True
+    lengths: tuple = ()        # packed batch: sequence lengths (sum = S)
 
     @property
     def torch_dtype(self) -> torch.dtype:
@@ -68,12 +71,18 @@ class Workload:
     def s2(self) -> bool:
         return self.group > 0
 
+    @property
+    def packed(self) -> bool:
+        return len(self.lengths) > 0
+
     def fwd_flops(self) -> float:
         """Algorithmic forward FLOPs: 4*B*Hq*S*S_vis*d with S_vis the mean
         number of visible keys per row (S for dense, S/2 for causal, G or G/2
-        for S2-Attn)."""
-        span = self.group if self.s2 else self.S
+        for S2-Attn); a packed batch sums 4*Hq*L*L_vis*d over its sequences."""
         frac = 0.5 if self.causal else 1.0
+        if self.packed:
+            return 4.0 * self.Hq * frac * self.d * float(sum(n * n for n in self.lengths))
+        span = self.group if self.s2 else self.S
         return 4.0 * self.B * self.Hq * self.S * span * frac * self.d
 
     def bwd_flops(self) -> float:
@@ -104,6 +113,35 @@ WORKLOADS = {
                  kv_chunk=4096, order="ring"),
     ]
 }
+
+
+def _packed_workload(name, n, max_len, seed, **kw):
+    lengths = tuple(packed_lengths(n, max_len, seed))
+    return Workload(name, B=1, S=sum(lengths), lengths=lengths, seed=seed, **kw)
+
+
+def packed_lengths(n: int, max_len: int, seed: int) -> list:
+    """Seeded lengths of ``n`` packed sequences: a mix of empty, one-token,
+    tile-multiple and ragged lengths up to ``max_len`` (the recipe of the
+    packed-batch cases; the pages fix no length distribution).  One sequence
+    in four takes an edge value (0, 1, 128 or max_len), the rest are uniform
+    in [1, max_len]."""
+    g = torch.Generator().manual_seed(seed * 104729 + n)
+    edges = [0, 1, min(128, max_len), max_len]
+    out = []
+    for i in range(n):
+        if int(torch.randint(4, (1,), generator=g)) == 0:
+            out.append(edges[int(torch.randint(len(edges), (1,), generator=g))])
+        else:
+            out.append(int(torch.randint(1, max_len + 1, (1,), generator=g)))
+    return out
+
+
+# Llama-3-8B attention shapes over a packed batch of documents up to 32K
+# tokens (about 128K tokens in all): the ragged, variable-length case.
+for _w in [_packed_workload("llama3_8b_gqa_packed_128k", n=8, max_len=32768, seed=6, Hq=32,
+                            Hkv=8, d=128, dtype="bf16", causal=True, std=0.5)]:
+    WORKLOADS[_w.name] = _w
 
 
 def _slab_seed(seed: int, tensor_id: int, slab: int) -> int:
@@ -167,23 +205,6 @@ def make_inputs(w: Workload, device="cpu", with_dout: Optional[bool] = None):
         with_dout = w.backward
     names = ["q", "k", "v"] + (["dout"] if with_dout else [])
     return {n: make_tensor(w, n, device) for n in names}
-
-
-def packed_lengths(n: int, max_len: int, seed: int) -> list:
-    """Seeded lengths of ``n`` packed sequences: a mix of empty, one-token,
-    tile-multiple and ragged lengths up to ``max_len`` (the recipe of the
-    packed-batch parity cases; the pages fix no length distribution).  One
-    sequence in four takes an edge value (0, 1, 128 or max_len), the rest are
-    uniform in [1, max_len]."""
-    g = torch.Generator().manual_seed(seed * 104729 + n)
-    edges = [0, 1, min(128, max_len), max_len]
-    out = []
-    for i in range(n):
-        if int(torch.randint(4, (1,), generator=g)) == 0:
-            out.append(edges[int(torch.randint(len(edges), (1,), generator=g))])
-        else:
-            out.append(int(torch.randint(1, max_len + 1, (1,), generator=g)))
-    return out
 
 
 def packed_offsets(lengths, start: int = 0) -> list:

@@ -191,6 +191,11 @@ def attn_fwd_varlen(q, k, v, cu_seqlens, max_seqlen: int, causal: bool = True,
     return out, lse
 
 
+def varlen_workspace_size(q, k, cu_seqlens, max_seqlen: int) -> int:
+    sh = _packed_shape(q, k, cu_seqlens, None)
+    return int(lib().lca_attn_bwd_varlen_workspace_size(ctypes.byref(sh), int(max_seqlen)))
+
+
 def attn_bwd_varlen(q, k, v, out, lse, dout, cu_seqlens, max_seqlen: int, causal: bool = True,
                     scale=None, dq=None, dk=None, dv=None, workspace=None, stream=None):
     """Gradients over a packed batch (lca_attn_bwd_varlen).  Returns (dq, dk, dv)."""
@@ -200,7 +205,7 @@ def attn_bwd_varlen(q, k, v, out, lse, dout, cu_seqlens, max_seqlen: int, causal
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
     if workspace is None:
-        n = int(lib().lca_attn_bwd_varlen_workspace_size(ctypes.byref(sh), int(max_seqlen)))
+        n = varlen_workspace_size(q, k, cu_seqlens, max_seqlen)
         workspace = torch.empty(max(n, 1), device=q.device, dtype=torch.uint8)
     _raise(lib().lca_attn_bwd_varlen(ctypes.byref(sh), _ptr(cu_seqlens), int(max_seqlen),
                                      _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),

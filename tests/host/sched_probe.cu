@@ -1,7 +1,8 @@
 // Host-side probe of the tile walks in sched.cuh: prints, for the schedule
 // given on the command line, every query tile's visits (key tile and the
-// key range [lo, hi) inside it), every key tile's query tile range, and the
-// position -> token tile map.  Built and run by tests/test_sched_host.py.
+// key range [lo, hi) inside it), the tile-only walk's tiles when chunks are
+// whole tiles, every key tile's query tile range, and the position -> token
+// tile map.  Built and run by tests/test_sched_host.py.
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -34,6 +35,17 @@ int main(int argc, char** argv) {
     int t, lo, hi;
     while (w.next(t, lo, hi)) printf(" %d,%d,%d", t, lo, hi);
     printf("\n");
+  }
+  // the tile-only walk, for chunks of whole tiles (S2 included)
+  if (s.s2 || s.kv_chunk % s.tile == 0) {
+    for (int qt = 0; qt < s.n_tiles; ++qt) {
+      lca::TileWalk w;
+      w.init(&s, qt, s.n_tiles);
+      printf("W %d:", qt);
+      int t;
+      while (w.next(t)) printf(" %d", t);
+      printf("\n");
+    }
   }
   for (int kt = 0; kt < s.n_tiles; ++kt) {
     lca::QWalk w;

@@ -29,18 +29,26 @@ def probe():
         args = [BIN] + [str(a) for a in (S, tile, causal, s2, kv_chunk, order, q_block, gt, st,
                                          fsh)] + [str(p) for p in perm]
         out = subprocess.run(args, capture_output=True, text=True, check=True).stdout
-        walks, qr, tok = {}, {}, {}
+        walks, qr, tok, tiles = {}, {}, {}, {}
         for line in out.splitlines():
             tag, rest = line.split(" ", 1)
             key, vals = rest.split(":")
             if tag == "Q":
                 walks[int(key)] = [tuple(int(x) for x in v.split(",")) for v in vals.split()]
+            elif tag == "W":
+                tiles[int(key)] = [int(v) for v in vals.split()]
             elif tag == "K":
                 qr[int(key)] = tuple(int(v) for v in vals.split())
             else:
                 tok[int(key)] = tuple(int(v) for v in vals.split())
+        if tiles:
+            # the tile-only walk visits the same tiles in the same order
+            assert tiles == {qt: [t for (t, _, _) in v] for qt, v in walks.items()}
+        run.tile_walks_checked += bool(tiles)
         return walks, qr, tok
-    return run
+    run.tile_walks_checked = 0
+    yield run
+    assert run.tile_walks_checked > 0
 
 
 def keys_of(visits, tile):
