@@ -21,6 +21,8 @@ bound memory:
   Large Language Models, Summary).
 * ``packed``     -- a packed batch of variable-length sequences: each
   sequence is an independent problem, so the definition applied per slice.
+* ``ffn``        -- the blockwise feedforward (gated SiLU, Llama's) computed
+  a block of token rows at a time (Ring Attention, Summary and Key points).
 * ``merge``      -- the (O, lse) combination of partial results over key
   chunks, whose order does not matter (Ring Attention, Summary).
 * ``brute``      -- pure-Python loops on tiny inputs, an independent
@@ -36,11 +38,12 @@ from .attention import (attention_forward, attention_rows, attention_backward,
 from .s2attn import s2attn_forward, s2attn_backward, s2_token_of_position
 from .merge import lse_merge
 from .packed import packed_attention_forward, packed_attention_backward
+from .ffn import ffn_forward, ffn_rows, silu
 
 __all__ = [
     "attention_forward", "attention_rows", "attention_backward",
     "attention_backward_rows",
     "chunked_attention_forward", "s2attn_forward", "s2attn_backward",
     "s2_token_of_position", "lse_merge", "packed_attention_forward",
-    "packed_attention_backward",
+    "packed_attention_backward", "ffn_forward", "ffn_rows", "silu",
 ]
