@@ -265,6 +265,40 @@ LCA_API lca_status lca_lse_merge(int64_t rows, int64_t d, const float* o_a,
                          const float* lse_b, float* o_out, float* lse_out,
                          void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Blockwise feedforward.  A host of the ring computes attention and the
+ * feedforward for its query block block by block, and the blockwise
+ * feedforward is what lowers the feedforward's activation memory (Ring
+ * Attention with Blockwise Transformers for Near-Infinite Context, Summary
+ * and Key points).  The pages print no feedforward; this is Llama's gated
+ * SiLU unit, with PyTorch's Linear weight layout:
+ *     H   = silu(x W_gate^T) * (x W_up^T),   silu(g) = g / (1 + e^-g)
+ *     out = H W_down^T
+ * x, out: [T, h] bf16; w_gate, w_up: [f, h] bf16; w_down: [h, f] bf16.
+ * The token rows are processed block_tokens at a time (0 selects
+ * LCA_FFN_BLOCK_DEFAULT; capped at T rounded up to 128), so the
+ * intermediate H exists for one block only: it lives in the caller's
+ * workspace of block_tokens * f bf16 (lca_ffn_workspace_size).  Products
+ * accumulate in float32 on the tensor cores; H is rounded to bf16.
+ * Errors: LCA_ERR_INVALID_ARG for dimensions <= 0, a block_tokens that is
+ * negative or not a multiple of 128, NULL or misaligned pointers;
+ * LCA_ERR_UNSUPPORTED unless h % 256 == 0 and f % 128 == 0 (every Llama
+ * size); LCA_ERR_WORKSPACE when the workspace is NULL or too small.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  int64_t T;  /* token rows */
+  int64_t h;  /* model width */
+  int64_t f;  /* feedforward width */
+} lca_ffn_shape;
+
+#define LCA_FFN_BLOCK_DEFAULT 8192
+
+LCA_API size_t lca_ffn_workspace_size(const lca_ffn_shape* shape, int64_t block_tokens);
+
+LCA_API lca_status lca_ffn_fwd(const lca_ffn_shape* shape, const void* x, const void* w_gate,
+                               const void* w_up, const void* w_down, int64_t block_tokens,
+                               void* out, void* workspace, size_t ws_bytes, void* stream);
+
 /* Synchronises `stream`, then reports and clears the device error word of
  * the current device: LCA_ERR_TIMEOUT if a kernel wait ran out since the
  * last check, LCA_ERR_INVALID_ARG if a kernel met invalid packed sequence

@@ -13,6 +13,7 @@
 #include "../../include/lca.h"
 #include "aux_kernels.cuh"
 #include "bwd_sm100.cuh"
+#include "ffn_sm100.cuh"
 #include "fwd_sm100.cuh"
 #include "ptx.cuh"
 #include "sched.cuh"
@@ -243,6 +244,44 @@ lca_status make_map_acc(CUtensorMap* m, const void* ptr, int64_t B, int64_t S, i
   return LCA_OK;
 }
 
+// [rows][cols] bf16 row-major viewed 2-D; box = 64 columns x 128 rows,
+// 128-byte swizzle (the K-major operand tiles of the feedforward products).
+// Rows past the extent load as zeros.
+lca_status make_map_2d(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(LCA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(LCA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return LCA_OK;
+}
+
+// Streaming multiprocessors of the current device (cached per device).
+lca_status sm_count(int* n) {
+  static std::mutex mu;
+  static int cache[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lk(mu);
+  if (dev >= 0 && dev < 64 && cache[dev]) {
+    *n = cache[dev];
+    return LCA_OK;
+  }
+  int v = 0;
+  e = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute(SM count)");
+  if (dev >= 0 && dev < 64) cache[dev] = v;
+  *n = v;
+  return LCA_OK;
+}
+
 // The backward kernel's warpgroups redistribute registers with setmaxnreg;
 // the split adds up to exactly the registers the CTA is launched with, so
 // refuse to launch a build whose register count differs.
@@ -462,6 +501,38 @@ lca_status run_bwd(const Common& c, const AttnSched& s, const void* q, const voi
   return launched("attn_bwd_f32");
 }
 
+// ---------------------------------------------------------------- feedforward
+lca_status check_ffn(const lca_ffn_shape* sh, int64_t* block) {
+  if (!sh) return fail(LCA_ERR_INVALID_ARG, "shape is NULL");
+  if (sh->T <= 0 || sh->h <= 0 || sh->f <= 0)
+    return fail(LCA_ERR_INVALID_ARG, "dimensions must be positive");
+  if (sh->T > (1ll << 31) - 1 || sh->h > (1 << 20) || sh->f > (1 << 20))
+    return fail(LCA_ERR_INVALID_ARG, "dimension too large");
+  if (sh->h % ffn::kBN || sh->f % 128)
+    return fail(LCA_ERR_UNSUPPORTED, "feedforward needs h %% 256 == 0 and f %% 128 == 0");
+  int64_t b = *block;
+  if (b < 0 || b % ffn::kBM)
+    return fail(LCA_ERR_INVALID_ARG, "block_tokens must be a non-negative multiple of 128");
+  const int64_t t_pad = (sh->T + ffn::kBM - 1) / ffn::kBM * ffn::kBM;
+  if (b == 0) b = LCA_FFN_BLOCK_DEFAULT;
+  if (b > t_pad) b = t_pad;
+  *block = b;
+  return LCA_OK;
+}
+
+template <int kEpi>
+lca_status launch_ffn_gemm(const CUtensorMap& ma, const CUtensorMap& mb0, const CUtensorMap& mb1,
+                           const ffn::Args& a, int slot, cudaStream_t st) {
+  lca_status r = ensure_smem(ffn_gemm_sm100<kEpi>, ffn::kSmemBytes, slot);
+  if (r != LCA_OK) return r;
+  int sms = 0;
+  if ((r = sm_count(&sms)) != LCA_OK) return r;
+  const int tiles = a.n_tm * a.n_tn;
+  const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
+  ffn_gemm_sm100<kEpi><<<grid, ffn::kThreads, ffn::kSmemBytes, st>>>(ma, mb0, mb1, a);
+  return launched("ffn_gemm_sm100");
+}
+
 }  // namespace
 
 extern "C" {
@@ -578,6 +649,60 @@ lca_status lca_attn_bwd_varlen(const lca_shape* shape, const int32_t* cu_seqlens
   if ((r = make_chunk_sched(c, causal, 0, nullptr, &s)) != LCA_OK) return r;
   return run_bwd(c, s, q, k, v, out, lse, dout, dq, dk, dv, workspace, ws_bytes, kDefaultBudget,
                  static_cast<cudaStream_t>(stream));
+}
+
+size_t lca_ffn_workspace_size(const lca_ffn_shape* shape, int64_t block_tokens) {
+  const std::string keep = t_last_error;  // a size query leaves the error detail alone
+  int64_t b = block_tokens;
+  const bool ok = check_ffn(shape, &b) == LCA_OK;
+  t_last_error = keep;
+  return ok ? static_cast<size_t>(b) * static_cast<size_t>(shape->f) * 2 : 0;
+}
+
+lca_status lca_ffn_fwd(const lca_ffn_shape* shape, const void* x, const void* w_gate,
+                       const void* w_up, const void* w_down, int64_t block_tokens, void* out,
+                       void* workspace, size_t ws_bytes, void* stream) {
+  int64_t block = block_tokens;
+  lca_status r = check_ffn(shape, &block);
+  if (r != LCA_OK) return r;
+  if ((r = check_ptrs({x, w_gate, w_up, w_down, out})) != LCA_OK) return r;
+  if (!workspace) return fail(LCA_ERR_WORKSPACE, "workspace is NULL");
+  const size_t need = static_cast<size_t>(block) * static_cast<size_t>(shape->f) * 2;
+  if (ws_bytes < need)
+    return fail(LCA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, need);
+  if (!aligned16(workspace)) return fail(LCA_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+  const int64_t T = shape->T, h = shape->h, f = shape->f;
+  CUtensorMap mx, mg, mu, md, mh;
+  if ((r = make_map_2d(&mx, x, T, h)) != LCA_OK) return r;
+  if ((r = make_map_2d(&mg, w_gate, f, h)) != LCA_OK) return r;
+  if ((r = make_map_2d(&mu, w_up, f, h)) != LCA_OK) return r;
+  if ((r = make_map_2d(&md, w_down, h, f)) != LCA_OK) return r;
+  if ((r = make_map_2d(&mh, workspace, block, f)) != LCA_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int64_t r0 = 0; r0 < T; r0 += block) {
+    const int rows = static_cast<int>(T - r0 < block ? T - r0 : block);
+    ffn::Args g1{};
+    g1.M = rows;
+    g1.K = static_cast<int>(h);
+    g1.n_tm = (rows + ffn::kBM - 1) / ffn::kBM;
+    g1.n_tn = static_cast<int>(f / 128);
+    g1.a_row0 = static_cast<int>(r0);
+    g1.ldo = static_cast<int>(f);
+    g1.budget = kDefaultBudget;
+    g1.out = static_cast<__nv_bfloat16*>(workspace);
+    if ((r = launch_ffn_gemm<ffn::EPI_SWIGLU>(mx, mg, mu, g1, 7, st)) != LCA_OK) return r;
+    ffn::Args g2{};
+    g2.M = rows;
+    g2.K = static_cast<int>(f);
+    g2.n_tm = g1.n_tm;
+    g2.n_tn = static_cast<int>(h / ffn::kBN);
+    g2.a_row0 = 0;
+    g2.ldo = static_cast<int>(h);
+    g2.budget = kDefaultBudget;
+    g2.out = static_cast<__nv_bfloat16*>(out) + r0 * h;
+    if ((r = launch_ffn_gemm<ffn::EPI_STORE>(mh, md, md, g2, 8, st)) != LCA_OK) return r;
+  }
+  return LCA_OK;
 }
 
 lca_status lca_lse_merge(int64_t rows, int64_t d, const float* o_a, const float* lse_a,

@@ -144,6 +144,53 @@ for _w in [_packed_workload("llama3_8b_gqa_packed_128k", n=8, max_len=32768, see
     WORKLOADS[_w.name] = _w
 
 
+@dataclasses.dataclass(frozen=True)
+class FfnWorkload:
+    """Shape and input recipe of one blockwise-feedforward workload: token
+    rows x [T, h] (standard normal, as after an RMS norm), weights w_gate,
+    w_up [f, h] and w_down [h, f] (normal with std ``w_std``, Llama's
+    initialisation), all rounded once to bf16; ``block`` token rows at a
+    time."""
+
+    name: str
+    T: int
+    h: int
+    f: int
+    block: int
+    seed: int
+    w_std: float = 0.02
+
+    def flops(self) -> float:
+        """Three products of 2*T*h*f each (gate, up, down)."""
+        return 6.0 * self.T * self.h * self.f
+
+
+FFN_WORKLOADS = {
+    w.name: w
+    for w in [
+        # the Llama-2-7B feedforward over the 32K-token sequence, 8K tokens
+        # per block
+        FfnWorkload("llama2_7b_ffn_s32k", T=32768, h=4096, f=11008, block=8192, seed=11),
+        FfnWorkload("tiny_ffn", T=300, h=256, f=384, block=128, seed=12),
+    ]
+}
+
+
+def make_ffn_inputs(w: FfnWorkload, device="cpu") -> dict:
+    """x, w_gate, w_up, w_down of workload w (one generator per tensor)."""
+    shapes = {"x": (w.T, w.h), "w_gate": (w.f, w.h), "w_up": (w.f, w.h), "w_down": (w.h, w.f)}
+    out = {}
+    for i, (name, shp) in enumerate(shapes.items()):
+        g = torch.Generator(device=device)
+        g.manual_seed(w.seed * 1_000_003 + 20 + i)
+        t = torch.randn(shp, generator=g, device=device, dtype=torch.float32)
+        if name != "x":
+            t.mul_(w.w_std)
+        out[name] = t.to(torch.bfloat16)
+        del t
+    return out
+
+
 def _slab_seed(seed: int, tensor_id: int, slab: int) -> int:
     return seed * 1_000_003 + tensor_id * 10_007 + slab
 

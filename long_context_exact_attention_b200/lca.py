@@ -23,6 +23,7 @@ STATUS = {0: "LCA_OK", 1: "LCA_ERR_INVALID_ARG", 2: "LCA_ERR_UNSUPPORTED",
 SYMBOLS = ["lca_attn_fwd", "lca_attn_bwd_workspace_size", "lca_attn_bwd",
            "lca_attn_bwd_noalloc",
            "lca_attn_fwd_varlen", "lca_attn_bwd_varlen_workspace_size", "lca_attn_bwd_varlen",
+           "lca_ffn_workspace_size", "lca_ffn_fwd",
            "lca_s2attn_fwd", "lca_s2attn_bwd", "lca_lse_merge", "lca_check",
            "lca_status_string", "lca_last_error", "lca_version"]
 
@@ -37,6 +38,10 @@ class Shape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int64), ("Hq", ctypes.c_int64), ("Hkv", ctypes.c_int64),
                 ("S", ctypes.c_int64), ("d", ctypes.c_int64), ("dtype", ctypes.c_int32),
                 ("scale", ctypes.c_float)]
+
+
+class FfnShape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("h", ctypes.c_int64), ("f", ctypes.c_int64)]
 
 
 class Opts(ctypes.Structure):
@@ -73,11 +78,15 @@ def lib() -> ctypes.CDLL:
         L.lca_s2attn_bwd.argtypes = [SP, P, P, P, P, P, P, I32, I64, I64, P, P, P, P,
                                      ctypes.c_size_t, P]
         L.lca_lse_merge.argtypes = [I64, I64, P, P, P, P, P, P, P]
+        FP = ctypes.POINTER(FfnShape)
+        L.lca_ffn_workspace_size.argtypes = [FP, I64]
+        L.lca_ffn_workspace_size.restype = ctypes.c_size_t
+        L.lca_ffn_fwd.argtypes = [FP, P, P, P, P, I64, P, P, ctypes.c_size_t, P]
         L.lca_check.argtypes = [P]
         L.lca_status_string.restype = ctypes.c_char_p
         L.lca_last_error.restype = ctypes.c_char_p
         for fn in ("lca_attn_fwd", "lca_attn_bwd", "lca_attn_bwd_noalloc", "lca_s2attn_fwd",
-                   "lca_s2attn_bwd", "lca_attn_fwd_varlen", "lca_attn_bwd_varlen",
+                   "lca_s2attn_bwd", "lca_attn_fwd_varlen", "lca_attn_bwd_varlen", "lca_ffn_fwd",
                    "lca_lse_merge", "lca_check"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
@@ -287,6 +296,33 @@ def s2attn_bwd(q, k, v, out, lse, dout, group: int, shift_heads: int, causal: bo
                                 int(shift_heads), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
                                 workspace.numel() * workspace.element_size(), _stream(stream)))
     return dq, dk, dv
+
+
+def ffn_workspace_size(T: int, h: int, f: int, block_tokens: int = 0) -> int:
+    sh = FfnShape(int(T), int(h), int(f))
+    return int(lib().lca_ffn_workspace_size(ctypes.byref(sh), int(block_tokens)))
+
+
+def ffn_fwd(x, w_gate, w_up, w_down, block_tokens: int = 0, out=None, workspace=None,
+            stream=None):
+    """Blockwise gated-SiLU feedforward (lca_ffn_fwd): x [T,h], w_gate/w_up
+    [f,h], w_down [h,f], all bf16.  Returns out [T,h]."""
+    _check_tensors(torch.bfloat16, x, w_gate, w_up, w_down)
+    if x.dim() != 2 or w_gate.dim() != 2 or w_down.dim() != 2:
+        raise ValueError("x is [T,h], w_gate/w_up are [f,h], w_down is [h,f]")
+    T, h = x.shape
+    f = w_gate.shape[0]
+    if w_gate.shape != (f, h) or w_up.shape != (f, h) or w_down.shape != (h, f):
+        raise ValueError("weight shapes do not match x")
+    sh = FfnShape(T, h, f)
+    out = torch.empty_like(x) if out is None else out
+    if workspace is None:
+        n = ffn_workspace_size(T, h, f, block_tokens)
+        workspace = torch.empty(max(n, 16), device=x.device, dtype=torch.uint8)
+    _raise(lib().lca_ffn_fwd(ctypes.byref(sh), _ptr(x), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+                             int(block_tokens), _ptr(out), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out
 
 
 def lse_merge(o_a, lse_a, o_b, lse_b, o_out=None, lse_out=None, stream=None):

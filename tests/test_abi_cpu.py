@@ -151,6 +151,28 @@ def test_varlen_workspace_size():
     assert L.lca_attn_bwd_varlen(*args, None, 1 << 30, None) == 5
 
 
+def test_ffn_arguments_rejected():
+    L = lca.lib()
+
+    def call(T=300, h=256, f=384, block=128, ws_bytes=1 << 30, ptrs=None, ws=FAKE):
+        sh = lca.FfnShape(T, h, f)
+        p = ptrs or [FAKE] * 5
+        return L.lca_ffn_fwd(ctypes.byref(sh), p[0], p[1], p[2], p[3], block, p[4], ws, ws_bytes,
+                             None)
+    assert call(T=0) == 1
+    assert call(block=100) == 1 and call(block=-128) == 1
+    assert call(h=128) == 2 and call(f=200) == 2
+    assert call(ptrs=[FAKE, None, FAKE, FAKE, FAKE]) == 1
+    assert call(ptrs=[FAKE, FAKE, FAKE, MISALIGNED, FAKE]) == 1
+    assert call(ws=None) == 5
+    assert call(ws_bytes=128 * 384 * 2 - 1) == 5
+    sh = lca.FfnShape(300, 256, 384)
+    # block rows x f bf16; 0 -> the default block, capped at T rounded up to 128
+    assert L.lca_ffn_workspace_size(ctypes.byref(sh), 128) == 128 * 384 * 2
+    assert L.lca_ffn_workspace_size(ctypes.byref(sh), 0) == 384 * 384 * 2
+    assert L.lca_ffn_workspace_size(ctypes.byref(lca.FfnShape(300, 100, 384)), 0) == 0
+
+
 def test_merge_arguments_rejected():
     L = lca.lib()
     assert L.lca_lse_merge(0, 4, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
