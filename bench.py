@@ -15,6 +15,10 @@ timing is the maximum over ranks.  Rank 0 prints one JSON line.
 --impl reference times the fp64 CPU oracle on a bounded sample of the same
 workload on this host's cores (the oracle is the only other implementation
 there is).
+
+--workload llama2_7b_ffn_s32k measures the blockwise feedforward instead
+(lca_ffn_fwd over 32768 tokens of the Llama-2-7B feedforward in blocks of
+8192): its own line, metric "blockwise feedforward TFLOP/s".
 """
 
 from __future__ import annotations
@@ -33,6 +37,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "causal attention TFLOP/s fwd+bwd (bf16, 1×B200) & fraction of dense BF16 peak"
+FFN_METRIC = "blockwise feedforward TFLOP/s (bf16, 1×B200) & fraction of dense BF16 peak"
 NOMINAL_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -199,11 +204,182 @@ def oracle_sample(w, seconds_target=12.0, max_rows=None):
     return flops(rows) / dt / 1e12, R, dt, cores, reps
 
 
+# ---------------------------------------------------------------- feedforward
+
+def ffn_oracle_sample(w, seconds_target=12.0, max_rows=None):
+    """Time the fp64 oracle on R token rows of feedforward workload w (each
+    row is independent); R doubles until one run takes >= seconds_target/4.
+    Returns (tflops, rows, seconds, cores, reps)."""
+    import oracle
+    from long_context_exact_attention_b200.inputs import make_ffn_inputs
+
+    x = make_ffn_inputs(w, "cpu")
+    xs, wg, wu, wd = (t.to(__import__("torch").float64).numpy() for t in
+                      (x["x"], x["w_gate"], x["w_up"], x["w_down"]))
+    R = 8
+    while True:
+        t0 = time.perf_counter()
+        oracle.ffn_forward(xs[:R], wg, wu, wd)
+        dt = time.perf_counter() - t0
+        if dt >= seconds_target / 4 or R >= w.T or (max_rows and R >= max_rows):
+            break
+        R *= 2
+    reps = max(1, int(round(seconds_target / max(dt, 1e-3))))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle.ffn_forward(xs[:R], wg, wu, wd)
+    dt = (time.perf_counter() - t0) / reps
+    return 6.0 * R * w.h * w.f / dt / 1e12, R, dt, len(os.sched_getaffinity(0)), reps
+
+
+def main_ffn(args, w):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    cfg = {"workload": w.name, "T": w.T, "h": w.h, "f": w.f, "block_tokens": w.block,
+           "activation": "gated SiLU (Llama)"}
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        for _ in range(args.warmup):
+            ffn_oracle_sample(w, seconds_target=2.0, max_rows=64)
+        vals, info = [], None
+        for _ in range(args.steps):
+            info = ffn_oracle_sample(w, seconds_target=5.0, max_rows=1024)
+            vals.append(info[0])
+        tf, R, dt, cores, reps = info
+        val = statistics.median(vals)
+        print(json.dumps({
+            "impl": "reference", "metric": FFN_METRIC, "value": val, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": f"fp64 oracle feedforward of {R} token rows"},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from long_context_exact_attention_b200 import lca
+    from long_context_exact_attention_b200.inputs import make_ffn_inputs
+
+    if world > 1:
+        dist.init_process_group("nccl", init_method="env://",
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.Stream(dev)
+    x = make_ffn_inputs(w, dev)
+    out = torch.empty_like(x["x"])
+    ws = torch.empty(lca.ffn_workspace_size(w.T, w.h, w.f, w.block), device=dev,
+                     dtype=torch.uint8)
+    n_blocks = -(-w.T // w.block)
+    torch.cuda.synchronize()
+
+    def step():
+        lca.ffn_fwd(x["x"], x["w_gate"], x["w_up"], x["w_down"], block_tokens=w.block, out=out,
+                    workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    stream.synchronize()
+    lca.check(stream)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    cvd = os.environ.get("CUDA_VISIBLE_DEVICES")
+    clocks = ClockSampler(cvd.split(",")[local] if cvd else str(local))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
+    stream.synchronize()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    lca.check(stream)
+    ms = [e[0].elapsed_time(e[1]) for e in evs]
+    total_ms = max_over_ranks(evs[0][0].elapsed_time(evs[-1][1]), dev)
+    value = whole_job_tflops(w.flops(), world, args.steps, total_ms)
+
+    e2e = None
+    if not args.no_e2e:
+        hx = x["x"].cpu().pin_memory()
+        hout = torch.empty_like(out, device="cpu").pin_memory()
+        with torch.cuda.stream(stream):
+            def e2e_step():
+                x["x"].copy_(hx, non_blocking=True)
+                step()
+                hout.copy_(out, non_blocking=True)
+            e2e_step()
+            stream.synchronize()
+            n_e2e = max(2, min(args.steps, 5))
+            if world > 1:
+                dist.barrier()
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            for _ in range(n_e2e):
+                e2e_step()
+            s1.record(stream)
+            s1.synchronize()
+        e_ms = max_over_ranks(s0.elapsed_time(s1), dev)
+        e2e = {"value": whole_job_tflops(w.flops(), world, n_e2e, e_ms), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": hx.numel() * hx.element_size(),
+               "d2h_bytes_per_step": hout.numel() * hout.element_size(),
+               "ms_per_step": e_ms / n_e2e}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    pk, pk_kind = peaks()
+    sustained = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    ach = w.flops() / (statistics.median(ms) * 1e-3) / 1e12
+    tr = traffic_record("ffn_gemm_sm100")
+    in_bytes = sum(t.numel() * t.element_size() for t in x.values())
+    cfg["l2"] = (f"inputs larger than L2 (x and weights {in_bytes / 2**20:.0f} MiB together, "
+                 "L2 126 MB); no flush")
+    line = {
+        "metric": FFN_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "impl": "lca", "config": cfg,
+        "frac_of_peak": {"measured_burst": value / world / pk.get("bf16_tflops", 1590.0),
+                         "measured_sustained": value / world / sustained,
+                         "nominal_2250": value / world / NOMINAL_BF16_TFLOPS},
+        "roofline": {"bound": "tensor", "kernel": "ffn_gemm_sm100", "achieved": ach,
+                     "peak": sustained, "unit": "TFLOP/s", "frac": ach / sustained,
+                     "peak_kind": f"{pk_kind} sustained bf16",
+                     "traffic": tr["dram_bytes_per_launch"] if tr else None,
+                     "frac_of_nominal_2250": ach / NOMINAL_BF16_TFLOPS,
+                     "timing": "CUDA events around the whole lca_ffn_fwd call (both products "
+                               "of every block), median over timed steps"},
+        "clocks": clk,
+        "gpu_launches": args.steps * 2 * n_blocks,
+        "e2e": e2e,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        tf, R, dt, cores, reps = ffn_oracle_sample(w)
+        line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                                "sample": f"fp64 oracle feedforward of {R} token rows, {reps} "
+                                          f"runs, {dt:.2f} s each"}
+    print(json.dumps(line), flush=True)
+
+
 # ---------------------------------------------------------------- main
 
 def main():
     args = parse()
-    from long_context_exact_attention_b200.inputs import WORKLOADS
+    from long_context_exact_attention_b200.inputs import FFN_WORKLOADS, WORKLOADS
+    if args.workload in FFN_WORKLOADS:
+        main_ffn(args, FFN_WORKLOADS[args.workload])
+        return
     w = WORKLOADS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
