@@ -1,8 +1,8 @@
 """Pins for the blockwise feedforward oracle (oracle/ffn.py), CPU only:
 pure-Python brute force on tiny inputs, invariance to the block size (the
 blockwise claim of the Ring Attention summary: blocking changes memory, not
-the result), closed forms of the gated SiLU, and planted mistakes that the
-pins must catch."""
+the result), closed forms of the gated SiLU, central finite differences of
+the backward, and planted mistakes that the pins must catch."""
 
 import math
 
@@ -101,3 +101,61 @@ def test_pins_catch_planted_mistakes(monkeypatch, mutant):
         monkeypatch.setattr(F, "ffn_forward", swapped)
     with pytest.raises(AssertionError):
         test_matches_brute(4, 5, 7)
+
+
+def _fd(fwd, tensors, do, eps=1e-6):
+    num = []
+    for t in tensors:
+        g = np.zeros_like(t)
+        for idx in np.ndindex(*t.shape):
+            old = t[idx]
+            t[idx] = old + eps
+            lp = np.sum(fwd() * do)
+            t[idx] = old - eps
+            lm = np.sum(fwd() * do)
+            t[idx] = old
+            g[idx] = (lp - lm) / (2 * eps)
+        num.append(g)
+    return num
+
+
+@pytest.mark.parametrize("block", [0, 2])
+def test_backward_finite_differences(block):
+    rng = np.random.default_rng(41 + block)
+    T, h, f = 5, 3, 4
+    x = rng.standard_normal((T, h))
+    wg, wu, wd = weights(rng, h, f, std=0.8)
+    do = rng.standard_normal((T, h))
+    got = F.ffn_backward(x, wg, wu, wd, do, block=block)
+    num = _fd(lambda: F.ffn_forward(x, wg, wu, wd), [x, wg, wu, wd], do)
+    for name, a, b in zip(("dx", "dw_gate", "dw_up", "dw_down"), got, num):
+        err = np.linalg.norm(a - b) / np.linalg.norm(b)
+        assert err <= 1e-6, (name, err)
+
+
+def test_backward_block_size_does_not_change_the_result():
+    rng = np.random.default_rng(43)
+    x = rng.standard_normal((19, 6))
+    wg, wu, wd = weights(rng, 6, 5)
+    do = rng.standard_normal((19, 6))
+    ref = F.ffn_backward(x, wg, wu, wd, do)
+    for block in (1, 4, 7):
+        for a, b in zip(F.ffn_backward(x, wg, wu, wd, do, block=block), ref):
+            np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+
+
+def test_backward_catches_a_wrong_silu_derivative(monkeypatch):
+    # the derivative of silu dropped to sigma alone must fail the pin
+    orig = F._sigmoid
+
+    def bad_backward(x, w_gate, w_up, w_down, dout, block=0):
+        x, wg, wu, wd, do = (np.asarray(t, np.float64) for t in (x, w_gate, w_up, w_down, dout))
+        g, u = x @ wg.T, x @ wu.T
+        sig = orig(g)
+        dh = do @ wd
+        dg = dh * u * sig
+        du = dh * g * sig
+        return dg @ wg + du @ wu, dg.T @ x, du.T @ x, do.T @ (g * sig * u)
+    monkeypatch.setattr(F, "ffn_backward", bad_backward)
+    with pytest.raises(AssertionError):
+        test_backward_finite_differences(0)
