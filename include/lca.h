@@ -299,6 +299,23 @@ LCA_API lca_status lca_ffn_fwd(const lca_ffn_shape* shape, const void* x, const 
                                const void* w_up, const void* w_down, int64_t block_tokens,
                                void* out, void* workspace, size_t ws_bytes, void* stream);
 
+/* lca_ffn_bwd -- gradients of sum(dout * out) of lca_ffn_fwd, block by
+ * block with the gate and up products recomputed from x:
+ *     dH = dout W_down;   dU = dH * silu(G);   dG = dH * U * silu'(G)
+ *     dx = dG W_gate + dU W_up
+ *     dw_gate += dG^T x;  dw_up += dU^T x;  dw_down += dout^T H
+ * dout: [T, h] bf16; dx: [T, h] bf16, overwritten; dw_gate, dw_up [f, h]
+ * and dw_down [h, f] are FLOAT32 and the gradients are ADDED to them (zero
+ * them first for a fresh gradient).  workspace: lca_ffn_bwd_workspace_size
+ * bytes (dH, dG, dU and H of one block, bf16).  Errors: as lca_ffn_fwd, and
+ * LCA_ERR_UNSUPPORTED unless f % 256 == 0. */
+LCA_API size_t lca_ffn_bwd_workspace_size(const lca_ffn_shape* shape, int64_t block_tokens);
+
+LCA_API lca_status lca_ffn_bwd(const lca_ffn_shape* shape, const void* x, const void* w_gate,
+                               const void* w_up, const void* w_down, const void* dout,
+                               int64_t block_tokens, void* dx, float* dw_gate, float* dw_up,
+                               float* dw_down, void* workspace, size_t ws_bytes, void* stream);
+
 /* Synchronises `stream`, then reports and clears the device error word of
  * the current device: LCA_ERR_TIMEOUT if a kernel wait ran out since the
  * last check, LCA_ERR_INVALID_ARG if a kernel met invalid packed sequence

@@ -244,15 +244,16 @@ lca_status make_map_acc(CUtensorMap* m, const void* ptr, int64_t B, int64_t S, i
   return LCA_OK;
 }
 
-// [rows][cols] bf16 row-major viewed 2-D; box = 64 columns x 128 rows,
-// 128-byte swizzle (the K-major operand tiles of the feedforward products).
-// Rows past the extent load as zeros.
-lca_status make_map_2d(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols) {
+// [rows][cols] bf16 row-major viewed 2-D; box = 64 columns x box_rows rows,
+// 128-byte swizzle: 128 rows for a K-major operand tile of the feedforward
+// products, 64 rows for an MN-major one.  Rows past the extent load as zeros.
+lca_status make_map_2d(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols,
+                       uint32_t box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(LCA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
-  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t box[2] = {64, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -303,11 +304,14 @@ lca_status check_bwd_regs() {
   return LCA_OK;
 }
 
-// Raise the dynamic shared-memory limit of a kernel once per device.
+// Raise the dynamic shared-memory limit of a kernel once per device; `slot`
+// names the kernel (one per instantiation, below kSmemSlots).
+constexpr int kSmemSlots = 16;
 template <typename K>
 lca_status ensure_smem(K kernel, size_t bytes, int slot) {
   static std::mutex mu;
-  static bool done[64][8] = {};
+  static bool done[64][kSmemSlots] = {};
+  if (slot < 0 || slot >= kSmemSlots) return fail(LCA_ERR_CUDA, "internal: bad kernel slot");
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
@@ -520,16 +524,18 @@ lca_status check_ffn(const lca_ffn_shape* sh, int64_t* block) {
   return LCA_OK;
 }
 
-template <int kEpi>
-lca_status launch_ffn_gemm(const CUtensorMap& ma, const CUtensorMap& mb0, const CUtensorMap& mb1,
-                           const ffn::Args& a, int slot, cudaStream_t st) {
-  lca_status r = ensure_smem(ffn_gemm_sm100<kEpi>, ffn::kSmemBytes, slot);
+template <int kEpi, bool kAmn, bool kBmn, bool kSplit>
+lca_status launch_ffn_gemm(const CUtensorMap& ma0, const CUtensorMap& ma1, const CUtensorMap& mb0,
+                           const CUtensorMap& mb1, const ffn::Args& a, int slot,
+                           cudaStream_t st) {
+  auto kernel = ffn_gemm_sm100<kEpi, kAmn, kBmn, kSplit>;
+  lca_status r = ensure_smem(kernel, ffn::kSmemBytes, slot);
   if (r != LCA_OK) return r;
   int sms = 0;
   if ((r = sm_count(&sms)) != LCA_OK) return r;
   const int tiles = a.n_tm * a.n_tn;
   const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
-  ffn_gemm_sm100<kEpi><<<grid, ffn::kThreads, ffn::kSmemBytes, st>>>(ma, mb0, mb1, a);
+  kernel<<<grid, ffn::kThreads, ffn::kSmemBytes, st>>>(ma0, ma1, mb0, mb1, a);
   return launched("ffn_gemm_sm100");
 }
 
@@ -686,21 +692,128 @@ lca_status lca_ffn_fwd(const lca_ffn_shape* shape, const void* x, const void* w_
     g1.K = static_cast<int>(h);
     g1.n_tm = (rows + ffn::kBM - 1) / ffn::kBM;
     g1.n_tn = static_cast<int>(f / 128);
-    g1.a_row0 = static_cast<int>(r0);
+    g1.a_off = static_cast<int>(r0);
     g1.ldo = static_cast<int>(f);
     g1.budget = kDefaultBudget;
     g1.out = static_cast<__nv_bfloat16*>(workspace);
-    if ((r = launch_ffn_gemm<ffn::EPI_SWIGLU>(mx, mg, mu, g1, 7, st)) != LCA_OK) return r;
+    if ((r = launch_ffn_gemm<ffn::EPI_SWIGLU, false, false, false>(mx, mx, mg, mu, g1, 7, st)) !=
+        LCA_OK)
+      return r;
     ffn::Args g2{};
     g2.M = rows;
     g2.K = static_cast<int>(f);
     g2.n_tm = g1.n_tm;
     g2.n_tn = static_cast<int>(h / ffn::kBN);
-    g2.a_row0 = 0;
+    g2.a_off = 0;
     g2.ldo = static_cast<int>(h);
     g2.budget = kDefaultBudget;
     g2.out = static_cast<__nv_bfloat16*>(out) + r0 * h;
-    if ((r = launch_ffn_gemm<ffn::EPI_STORE>(mh, md, md, g2, 8, st)) != LCA_OK) return r;
+    if ((r = launch_ffn_gemm<ffn::EPI_STORE, false, false, false>(mh, mh, md, md, g2, 8, st)) !=
+        LCA_OK)
+      return r;
+  }
+  return LCA_OK;
+}
+
+size_t lca_ffn_bwd_workspace_size(const lca_ffn_shape* shape, int64_t block_tokens) {
+  const std::string keep = t_last_error;
+  int64_t b = block_tokens;
+  const bool ok = check_ffn(shape, &b) == LCA_OK && shape->f % ffn::kBN == 0;
+  t_last_error = keep;
+  // dH, dG, dU and H, each [block, f] bf16
+  return ok ? 4 * static_cast<size_t>(b) * static_cast<size_t>(shape->f) * 2 : 0;
+}
+
+lca_status lca_ffn_bwd(const lca_ffn_shape* shape, const void* x, const void* w_gate,
+                       const void* w_up, const void* w_down, const void* dout,
+                       int64_t block_tokens, void* dx, float* dw_gate, float* dw_up,
+                       float* dw_down, void* workspace, size_t ws_bytes, void* stream) {
+  int64_t block = block_tokens;
+  lca_status r = check_ffn(shape, &block);
+  if (r != LCA_OK) return r;
+  if (shape->f % ffn::kBN)
+    return fail(LCA_ERR_UNSUPPORTED, "feedforward backward needs f %% 256 == 0");
+  if ((r = check_ptrs({x, w_gate, w_up, w_down, dout, dx, dw_gate, dw_up, dw_down})) != LCA_OK)
+    return r;
+  if (!workspace) return fail(LCA_ERR_WORKSPACE, "workspace is NULL");
+  const int64_t T = shape->T, h = shape->h, f = shape->f;
+  const size_t one = static_cast<size_t>(block) * static_cast<size_t>(f) * 2;
+  if (ws_bytes < 4 * one)
+    return fail(LCA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, 4 * one);
+  if (!aligned16(workspace)) return fail(LCA_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+  auto* ws = static_cast<__nv_bfloat16*>(workspace);
+  __nv_bfloat16* dH = ws;
+  __nv_bfloat16* dG = ws + block * f;
+  __nv_bfloat16* dU = ws + 2 * block * f;
+  __nv_bfloat16* H = ws + 3 * block * f;
+  // K-major views (boxes of 128 rows) and MN-major views (boxes of 64 rows)
+  CUtensorMap x_k, x_mn, do_k, do_mn, wg_k, wu_k, wg_mn, wu_mn, wd_mn, dg_k, du_k, dg_mn, du_mn,
+      h_mn;
+  if ((r = make_map_2d(&x_k, x, T, h)) != LCA_OK) return r;
+  if ((r = make_map_2d(&x_mn, x, T, h, 64)) != LCA_OK) return r;
+  if ((r = make_map_2d(&do_k, dout, T, h)) != LCA_OK) return r;
+  if ((r = make_map_2d(&do_mn, dout, T, h, 64)) != LCA_OK) return r;
+  if ((r = make_map_2d(&wg_k, w_gate, f, h)) != LCA_OK) return r;
+  if ((r = make_map_2d(&wu_k, w_up, f, h)) != LCA_OK) return r;
+  if ((r = make_map_2d(&wg_mn, w_gate, f, h, 64)) != LCA_OK) return r;
+  if ((r = make_map_2d(&wu_mn, w_up, f, h, 64)) != LCA_OK) return r;
+  if ((r = make_map_2d(&wd_mn, w_down, h, f, 64)) != LCA_OK) return r;
+  if ((r = make_map_2d(&dg_k, dG, block, f)) != LCA_OK) return r;
+  if ((r = make_map_2d(&du_k, dU, block, f)) != LCA_OK) return r;
+  if ((r = make_map_2d(&dg_mn, dG, block, f, 64)) != LCA_OK) return r;
+  if ((r = make_map_2d(&du_mn, dU, block, f, 64)) != LCA_OK) return r;
+  if ((r = make_map_2d(&h_mn, H, block, f, 64)) != LCA_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int64_t r0 = 0; r0 < T; r0 += block) {
+    const int rows = static_cast<int>(T - r0 < block ? T - r0 : block);
+    const int n_tm = (rows + ffn::kBM - 1) / ffn::kBM;
+    const int k_rows = (rows + ffn::kBK - 1) / ffn::kBK * ffn::kBK;  // whole K steps
+    ffn::Args g{};
+    g.budget = kDefaultBudget;
+    // dH = dout W_down
+    g.M = rows, g.K = static_cast<int>(h), g.n_tm = n_tm, g.n_tn = static_cast<int>(f / ffn::kBN);
+    g.a_off = static_cast<int>(r0), g.b_off = 0, g.ldo = static_cast<int>(f), g.out = dH;
+    if ((r = launch_ffn_gemm<ffn::EPI_STORE, false, true, false>(do_k, do_k, wd_mn, wd_mn, g, 9,
+                                                                 st)) != LCA_OK)
+      return r;
+    // G, U recomputed; dG, dU, H written
+    g = ffn::Args{};
+    g.budget = kDefaultBudget;
+    g.M = rows, g.K = static_cast<int>(h), g.n_tm = n_tm, g.n_tn = static_cast<int>(f / 128);
+    g.a_off = static_cast<int>(r0), g.b_off = 0, g.ldo = static_cast<int>(f);
+    g.ld_in = static_cast<int>(f), g.in = dH, g.out = dG, g.out2 = dU, g.out3 = H;
+    if ((r = launch_ffn_gemm<ffn::EPI_SWIGLU_BWD, false, false, false>(x_k, x_k, wg_k, wu_k, g,
+                                                                       10, st)) != LCA_OK)
+      return r;
+    // dX = dG W_gate + dU W_up
+    g = ffn::Args{};
+    g.budget = kDefaultBudget;
+    g.M = rows, g.K = static_cast<int>(2 * f), g.n_tm = n_tm, g.n_tn = static_cast<int>(h / ffn::kBN);
+    g.a_off = 0, g.b_off = 0, g.ldo = static_cast<int>(h);
+    g.out = static_cast<__nv_bfloat16*>(dx) + r0 * h;
+    if ((r = launch_ffn_gemm<ffn::EPI_STORE, false, true, true>(dg_k, du_k, wg_mn, wu_mn, g, 11,
+                                                                st)) != LCA_OK)
+      return r;
+    // dW_gate += dG^T x, dW_up += dU^T x
+    g = ffn::Args{};
+    g.budget = kDefaultBudget;
+    g.M = static_cast<int>(f), g.K = k_rows, g.n_tm = static_cast<int>(f / ffn::kBM);
+    g.n_tn = static_cast<int>(h / ffn::kBN);
+    g.a_off = 0, g.b_off = static_cast<int>(r0), g.ldo = static_cast<int>(h), g.out32 = dw_gate;
+    if ((r = launch_ffn_gemm<ffn::EPI_ACC32, true, true, false>(dg_mn, dg_mn, x_mn, x_mn, g, 12,
+                                                                st)) != LCA_OK)
+      return r;
+    g.out32 = dw_up;
+    if ((r = launch_ffn_gemm<ffn::EPI_ACC32, true, true, false>(du_mn, du_mn, x_mn, x_mn, g, 12,
+                                                                st)) != LCA_OK)
+      return r;
+    // dW_down += dout^T H
+    g.M = static_cast<int>(h), g.n_tm = static_cast<int>(h / ffn::kBM);
+    g.n_tn = static_cast<int>(f / ffn::kBN);
+    g.a_off = static_cast<int>(r0), g.b_off = 0, g.ldo = static_cast<int>(f), g.out32 = dw_down;
+    if ((r = launch_ffn_gemm<ffn::EPI_ACC32, true, true, false>(do_mn, do_mn, h_mn, h_mn, g, 12,
+                                                                st)) != LCA_OK)
+      return r;
   }
   return LCA_OK;
 }

@@ -23,7 +23,7 @@ STATUS = {0: "LCA_OK", 1: "LCA_ERR_INVALID_ARG", 2: "LCA_ERR_UNSUPPORTED",
 SYMBOLS = ["lca_attn_fwd", "lca_attn_bwd_workspace_size", "lca_attn_bwd",
            "lca_attn_bwd_noalloc",
            "lca_attn_fwd_varlen", "lca_attn_bwd_varlen_workspace_size", "lca_attn_bwd_varlen",
-           "lca_ffn_workspace_size", "lca_ffn_fwd",
+           "lca_ffn_workspace_size", "lca_ffn_fwd", "lca_ffn_bwd_workspace_size", "lca_ffn_bwd",
            "lca_s2attn_fwd", "lca_s2attn_bwd", "lca_lse_merge", "lca_check",
            "lca_status_string", "lca_last_error", "lca_version"]
 
@@ -82,11 +82,14 @@ def lib() -> ctypes.CDLL:
         L.lca_ffn_workspace_size.argtypes = [FP, I64]
         L.lca_ffn_workspace_size.restype = ctypes.c_size_t
         L.lca_ffn_fwd.argtypes = [FP, P, P, P, P, I64, P, P, ctypes.c_size_t, P]
+        L.lca_ffn_bwd_workspace_size.argtypes = [FP, I64]
+        L.lca_ffn_bwd_workspace_size.restype = ctypes.c_size_t
+        L.lca_ffn_bwd.argtypes = [FP, P, P, P, P, P, I64, P, P, P, P, P, ctypes.c_size_t, P]
         L.lca_check.argtypes = [P]
         L.lca_status_string.restype = ctypes.c_char_p
         L.lca_last_error.restype = ctypes.c_char_p
         for fn in ("lca_attn_fwd", "lca_attn_bwd", "lca_attn_bwd_noalloc", "lca_s2attn_fwd",
-                   "lca_s2attn_bwd", "lca_attn_fwd_varlen", "lca_attn_bwd_varlen", "lca_ffn_fwd",
+                   "lca_s2attn_bwd", "lca_attn_fwd_varlen", "lca_attn_bwd_varlen", "lca_ffn_fwd", "lca_ffn_bwd",
                    "lca_lse_merge", "lca_check"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
@@ -323,6 +326,39 @@ def ffn_fwd(x, w_gate, w_up, w_down, block_tokens: int = 0, out=None, workspace=
                              int(block_tokens), _ptr(out), _ptr(workspace),
                              workspace.numel() * workspace.element_size(), _stream(stream)))
     return out
+
+
+def ffn_bwd_workspace_size(T: int, h: int, f: int, block_tokens: int = 0) -> int:
+    sh = FfnShape(int(T), int(h), int(f))
+    return int(lib().lca_ffn_bwd_workspace_size(ctypes.byref(sh), int(block_tokens)))
+
+
+def ffn_bwd(x, w_gate, w_up, w_down, dout, block_tokens: int = 0, dx=None, dw_gate=None,
+            dw_up=None, dw_down=None, workspace=None, stream=None):
+    """Gradients of the blockwise feedforward (lca_ffn_bwd).  dx (bf16) is
+    overwritten; dw_gate, dw_up, dw_down are float32 and the gradients are
+    added to them (new zero tensors when not given).  Returns (dx, dw_gate,
+    dw_up, dw_down)."""
+    _check_tensors(torch.bfloat16, x, w_gate, w_up, w_down, dout)
+    T, h = x.shape
+    f = w_gate.shape[0]
+    if dout.shape != x.shape:
+        raise ValueError("dout must have x's shape")
+    dx = torch.empty_like(x) if dx is None else dx
+    z = lambda t: torch.zeros(t.shape, device=t.device, dtype=torch.float32)
+    dw_gate = z(w_gate) if dw_gate is None else dw_gate
+    dw_up = z(w_up) if dw_up is None else dw_up
+    dw_down = z(w_down) if dw_down is None else dw_down
+    _check_tensors(torch.float32, dw_gate, dw_up, dw_down)
+    sh = FfnShape(T, h, f)
+    if workspace is None:
+        n = ffn_bwd_workspace_size(T, h, f, block_tokens)
+        workspace = torch.empty(max(n, 16), device=x.device, dtype=torch.uint8)
+    _raise(lib().lca_ffn_bwd(ctypes.byref(sh), _ptr(x), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+                             _ptr(dout), int(block_tokens), _ptr(dx), _ptr(dw_gate), _ptr(dw_up),
+                             _ptr(dw_down), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream(stream)))
+    return dx, dw_gate, dw_up, dw_down
 
 
 def lse_merge(o_a, lse_a, o_b, lse_b, o_out=None, lse_out=None, stream=None):

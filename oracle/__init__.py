@@ -38,12 +38,12 @@ from .attention import (attention_forward, attention_rows, attention_backward,
 from .s2attn import s2attn_forward, s2attn_backward, s2_token_of_position
 from .merge import lse_merge
 from .packed import packed_attention_forward, packed_attention_backward
-from .ffn import ffn_forward, ffn_backward, ffn_rows, silu
+from .ffn import ffn_forward, ffn_backward, ffn_backward_columns, ffn_rows, silu
 
 __all__ = [
     "attention_forward", "attention_rows", "attention_backward",
     "attention_backward_rows",
     "chunked_attention_forward", "s2attn_forward", "s2attn_backward",
     "s2_token_of_position", "lse_merge", "packed_attention_forward",
-    "packed_attention_backward", "ffn_forward", "ffn_backward", "ffn_rows", "silu",
+    "packed_attention_backward", "ffn_forward", "ffn_backward", "ffn_backward_columns", "ffn_rows", "silu",
 ]

@@ -97,3 +97,20 @@ def ffn_backward(x, w_gate, w_up, w_down, dout, block: int = 0):
         dwu += du.T @ xb
         dwd += dob.T @ (s * u)
     return dx, dwg, dwu, dwd
+
+
+def ffn_backward_columns(x, w_gate, w_up, w_down, dout, cols):
+    """The weight gradients that involve feedforward columns ``cols`` only:
+    rows cols of dw_gate and dw_up, columns cols of dw_down.  Column j needs
+    g[:, j], u[:, j] and dH[:, j] over all tokens, O(T h) each, so large
+    shapes can be checked column by column.  Returns (dwg_rows, dwu_rows,
+    dwd_cols) in float64."""
+    x, wg, wu, wd, do = _f64(x), _f64(w_gate), _f64(w_up), _f64(w_down), _f64(dout)
+    cols = np.asarray(cols)
+    g, u = x @ wg[cols].T, x @ wu[cols].T          # [T, len(cols)]
+    sig = _sigmoid(g)
+    s = g * sig
+    dh = do @ wd[:, cols]
+    du = dh * s
+    dg = dh * u * sig * (1.0 + g * (1.0 - sig))
+    return dg.T @ x, du.T @ x, do.T @ (s * u)

@@ -173,6 +173,22 @@ def test_ffn_arguments_rejected():
     assert L.lca_ffn_workspace_size(ctypes.byref(lca.FfnShape(300, 100, 384)), 0) == 0
 
 
+def test_ffn_bwd_arguments_rejected():
+    L = lca.lib()
+
+    def call(T=300, h=256, f=512, block=128, ws_bytes=1 << 30, ws=FAKE):
+        sh = lca.FfnShape(T, h, f)
+        return L.lca_ffn_bwd(ctypes.byref(sh), *([FAKE] * 5), block, *([FAKE] * 4), ws,
+                             ws_bytes, None)
+    assert call(T=0) == 1
+    assert call(f=384) == 2          # the backward needs f % 256 == 0
+    assert call(ws=None) == 5
+    assert call(ws_bytes=4 * 128 * 512 * 2 - 1) == 5
+    sh = lca.FfnShape(300, 256, 512)
+    assert L.lca_ffn_bwd_workspace_size(ctypes.byref(sh), 128) == 4 * 128 * 512 * 2
+    assert L.lca_ffn_bwd_workspace_size(ctypes.byref(lca.FfnShape(300, 256, 384)), 128) == 0
+
+
 def test_merge_arguments_rejected():
     L = lca.lib()
     assert L.lca_lse_merge(0, 4, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1

@@ -87,3 +87,66 @@ def test_llama2_7b_ffn_full_size_sampled_rows():
     ref = oracle.ffn_rows(x["x"].cpu(), x["w_gate"].cpu(), x["w_up"].cpu(), x["w_down"].cpu(),
                           rows)
     check(host(out[rows]), ref)
+
+
+# ---------------------------------------------------------------- backward
+# dx and the weight gradients: relative Frobenius <= 2e-2 (the bar of the
+# attention gradients; bf16 rounding of dH, dG, dU and H, float32 sums)
+GRAD_REL = 2e-2
+
+
+def grads(x, block, dw=None):
+    g = torch.Generator(device="cuda").manual_seed(77)
+    dout = torch.randn(x["x"].shape, generator=g, device="cuda").to(torch.bfloat16)
+    kw = {} if dw is None else dict(dw_gate=dw[0], dw_up=dw[1], dw_down=dw[2])
+    res = lca.ffn_bwd(x["x"], x["w_gate"], x["w_up"], x["w_down"], dout, block_tokens=block, **kw)
+    torch.cuda.synchronize()
+    lca.check()
+    return dout, res
+
+
+@pytest.mark.parametrize("T,h,f,block", [
+    (300, 256, 512, 128),    # three blocks, the last of 44 rows (K steps past it)
+    (1000, 512, 768, 256),
+    (1, 256, 256, 0),
+])
+def test_ffn_backward_matches_oracle(T, h, f, block):
+    w, x = inputs("tiny_ffn", T=T, h=h, f=f, block=block, seed=T + f)
+    dout, got = grads(x, block)
+    ref = oracle.ffn_backward(x["x"], x["w_gate"], x["w_up"], x["w_down"], dout, block=block)
+    for name, a, b in zip(("dx", "dw_gate", "dw_up", "dw_down"), got, ref):
+        a = host(a)
+        assert np.isfinite(a).all(), name
+        assert rel_fro(a, b) <= GRAD_REL, (name, rel_fro(a, b))
+
+
+def test_ffn_backward_accumulates_and_dx_is_block_exact():
+    w, x = inputs("tiny_ffn", T=600, h=256, f=512, seed=8)
+    dout, (dx1, g1, u1, d1) = grads(x, 128)
+    # a second call adds the same gradients again
+    _, (dx2, g2, u2, d2) = grads(x, 128, dw=(g1.clone(), u1.clone(), d1.clone()))
+    for a, b in ((g2, g1), (u2, u1), (d2, d1)):
+        assert rel_fro(host(a), 2 * host(b)) < 1e-6
+    # dx rows do not depend on the blocking
+    _, (dx3, _, _, _) = grads(x, 256)
+    assert torch.equal(dx1, dx2) and torch.equal(dx1, dx3)
+
+
+def test_llama2_7b_ffn_backward_full_size_sampled():
+    """The bench configuration; dx on sampled rows, the weight gradients on
+    sampled feedforward columns (each exact in the oracle)."""
+    w = FFN_WORKLOADS["llama2_7b_ffn_s32k"]
+    x = make_ffn_inputs(w, "cuda")
+    dout, (dx, dwg, dwu, dwd) = grads(x, w.block)
+    xc = {k: v.cpu() for k, v in x.items()}
+    doc = dout.cpu()
+    rows = [0, 127, w.block - 1, w.block, w.T - 1, 12345]
+    import oracle.ffn as F
+    xs, wg, wu, wd, do = (F._f64(t) for t in (xc["x"], xc["w_gate"], xc["w_up"], xc["w_down"], doc))
+    ref_dx = F.ffn_backward(xs[rows], wg, wu, wd, do[rows])[0]
+    assert rel_fro(host(dx[rows]), ref_dx) <= GRAD_REL
+    cols = [0, 1, 4095, 5000, 11007]
+    a, b, c = oracle.ffn_backward_columns(xs, wg, wu, wd, do, cols)
+    assert rel_fro(host(dwg[cols]), a) <= GRAD_REL
+    assert rel_fro(host(dwu[cols]), b) <= GRAD_REL
+    assert rel_fro(host(dwd[:, cols]), c) <= GRAD_REL

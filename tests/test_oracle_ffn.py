@@ -159,3 +159,16 @@ def test_backward_catches_a_wrong_silu_derivative(monkeypatch):
     monkeypatch.setattr(F, "ffn_backward", bad_backward)
     with pytest.raises(AssertionError):
         test_backward_finite_differences(0)
+
+
+def test_backward_columns_match_full():
+    rng = np.random.default_rng(47)
+    x = rng.standard_normal((11, 5))
+    wg, wu, wd = weights(rng, 5, 7)
+    do = rng.standard_normal((11, 5))
+    _, dwg, dwu, dwd = F.ffn_backward(x, wg, wu, wd, do)
+    cols = [0, 3, 6]
+    a, b, c = F.ffn_backward_columns(x, wg, wu, wd, do, cols)
+    np.testing.assert_allclose(a, dwg[cols], atol=1e-13)
+    np.testing.assert_allclose(b, dwu[cols], atol=1e-13)
+    np.testing.assert_allclose(c, dwd[:, cols], atol=1e-13)
