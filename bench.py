@@ -17,8 +17,8 @@ workload on this host's cores (the oracle is the only other implementation
 there is).
 
 --workload llama2_7b_ffn_s32k measures the blockwise feedforward instead
-(lca_ffn_fwd over 32768 tokens of the Llama-2-7B feedforward in blocks of
-8192): its own line, metric "blockwise feedforward TFLOP/s".
+(lca_ffn_fwd + lca_ffn_bwd over 32768 tokens of the Llama-2-7B feedforward
+in blocks of 8192): its own line, metric "blockwise feedforward TFLOP/s".
 """
 
 from __future__ import annotations
@@ -37,7 +37,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "causal attention TFLOP/s fwd+bwd (bf16, 1×B200) & fraction of dense BF16 peak"
-FFN_METRIC = "blockwise feedforward TFLOP/s (bf16, 1×B200) & fraction of dense BF16 peak"
+FFN_METRIC = "blockwise feedforward TFLOP/s fwd+bwd (bf16, 1×B200) & fraction of dense BF16 peak"
 NOMINAL_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -216,10 +216,16 @@ def ffn_oracle_sample(w, seconds_target=12.0, max_rows=None):
     x = make_ffn_inputs(w, "cpu")
     xs, wg, wu, wd = (t.to(__import__("torch").float64).numpy() for t in
                       (x["x"], x["w_gate"], x["w_up"], x["w_down"]))
+    do = xs[::-1].copy()  # any dout of the right shape; the cost does not depend on it
+
+    def run(R):
+        oracle.ffn_forward(xs[:R], wg, wu, wd)
+        oracle.ffn_backward(xs[:R], wg, wu, wd, do[:R])
+
     R = 8
     while True:
         t0 = time.perf_counter()
-        oracle.ffn_forward(xs[:R], wg, wu, wd)
+        run(R)
         dt = time.perf_counter() - t0
         if dt >= seconds_target / 4 or R >= w.T or (max_rows and R >= max_rows):
             break
@@ -227,9 +233,10 @@ def ffn_oracle_sample(w, seconds_target=12.0, max_rows=None):
     reps = max(1, int(round(seconds_target / max(dt, 1e-3))))
     t0 = time.perf_counter()
     for _ in range(reps):
-        oracle.ffn_forward(xs[:R], wg, wu, wd)
+        run(R)
     dt = (time.perf_counter() - t0) / reps
-    return 6.0 * R * w.h * w.f / dt / 1e12, R, dt, len(os.sched_getaffinity(0)), reps
+    # the oracle's backward recomputes nothing it does not need: 6 + 12 T h f
+    return 18.0 * R * w.h * w.f / dt / 1e12, R, dt, len(os.sched_getaffinity(0)), reps
 
 
 def main_ffn(args, w):
@@ -255,7 +262,8 @@ def main_ffn(args, w):
             "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
             "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                             "sample": f"fp64 oracle feedforward of {R} token rows"},
+                             "sample": f"fp64 oracle feedforward forward + backward of {R} "
+                                       "token rows"},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}), flush=True)
         return
@@ -273,21 +281,37 @@ def main_ffn(args, w):
     stream = torch.cuda.Stream(dev)
     x = make_ffn_inputs(w, dev)
     out = torch.empty_like(x["x"])
-    ws = torch.empty(lca.ffn_workspace_size(w.T, w.h, w.f, w.block), device=dev,
+    g = torch.Generator(device=dev).manual_seed(w.seed * 1_000_003 + 30)
+    dout = torch.randn(x["x"].shape, generator=g, device=dev).to(torch.bfloat16)
+    dx = torch.empty_like(x["x"])
+    dws = [torch.zeros(x[n].shape, device=dev, dtype=torch.float32)
+           for n in ("w_gate", "w_up", "w_down")]
+    ws = torch.empty(max(lca.ffn_workspace_size(w.T, w.h, w.f, w.block),
+                         lca.ffn_bwd_workspace_size(w.T, w.h, w.f, w.block)), device=dev,
                      dtype=torch.uint8)
     n_blocks = -(-w.T // w.block)
+    fwd_flops, bwd_flops = w.flops(), w.bwd_flops()
     torch.cuda.synchronize()
 
-    def step():
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
         lca.ffn_fwd(x["x"], x["w_gate"], x["w_up"], x["w_down"], block_tokens=w.block, out=out,
                     workspace=ws, stream=stream)
+        if ev:
+            ev[1].record(stream)
+        lca.ffn_bwd(x["x"], x["w_gate"], x["w_up"], x["w_down"], dout, block_tokens=w.block,
+                    dx=dx, dw_gate=dws[0], dw_up=dws[1], dw_down=dws[2], workspace=ws,
+                    stream=stream)
+        if ev:
+            ev[2].record(stream)
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             step()
     stream.synchronize()
     lca.check(stream)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     cvd = os.environ.get("CUDA_VISIBLE_DEVICES")
     clocks = ClockSampler(cvd.split(",")[local] if cvd else str(local))
     if world > 1:
@@ -297,26 +321,29 @@ def main_ffn(args, w):
     time.sleep(0.3)
     with torch.cuda.stream(stream):
         for i in range(args.steps):
-            evs[i][0].record(stream)
-            step()
-            evs[i][1].record(stream)
+            step(evs[i])
     stream.synchronize()
     torch.cuda.synchronize()
     clk = clocks.stop()
     lca.check(stream)
-    ms = [e[0].elapsed_time(e[1]) for e in evs]
-    total_ms = max_over_ranks(evs[0][0].elapsed_time(evs[-1][1]), dev)
-    value = whole_job_tflops(w.flops(), world, args.steps, total_ms)
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    bwd_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    total_ms = max_over_ranks(evs[0][0].elapsed_time(evs[-1][2]), dev)
+    value = whole_job_tflops(fwd_flops + bwd_flops, world, args.steps, total_ms)
 
     e2e = None
     if not args.no_e2e:
         hx = x["x"].cpu().pin_memory()
+        hdo = dout.cpu().pin_memory()
         hout = torch.empty_like(out, device="cpu").pin_memory()
+        hdx = torch.empty_like(dx, device="cpu").pin_memory()
         with torch.cuda.stream(stream):
             def e2e_step():
                 x["x"].copy_(hx, non_blocking=True)
+                dout.copy_(hdo, non_blocking=True)
                 step()
                 hout.copy_(out, non_blocking=True)
+                hdx.copy_(dx, non_blocking=True)
             e2e_step()
             stream.synchronize()
             n_e2e = max(2, min(args.steps, 5))
@@ -329,9 +356,10 @@ def main_ffn(args, w):
             s1.record(stream)
             s1.synchronize()
         e_ms = max_over_ranks(s0.elapsed_time(s1), dev)
-        e2e = {"value": whole_job_tflops(w.flops(), world, n_e2e, e_ms), "unit": "TFLOP/s",
-               "h2d_bytes_per_step": hx.numel() * hx.element_size(),
-               "d2h_bytes_per_step": hout.numel() * hout.element_size(),
+        e2e = {"value": whole_job_tflops(fwd_flops + bwd_flops, world, n_e2e, e_ms),
+               "unit": "TFLOP/s",
+               "h2d_bytes_per_step": 2 * hx.numel() * hx.element_size(),
+               "d2h_bytes_per_step": 2 * hout.numel() * hout.element_size(),
                "ms_per_step": e_ms / n_e2e}
     if world > 1:
         dist.barrier()
@@ -340,9 +368,10 @@ def main_ffn(args, w):
         return
     pk, pk_kind = peaks()
     sustained = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-    ach = w.flops() / (statistics.median(ms) * 1e-3) / 1e12
-    tr = traffic_record("ffn_gemm_sm100")
-    in_bytes = sum(t.numel() * t.element_size() for t in x.values())
+    fwd_t, bwd_t = statistics.median(fwd_ms), statistics.median(bwd_ms)
+    ach = bwd_flops / (bwd_t * 1e-3) / 1e12
+    tr = traffic_record("ffn_gemm_sm100_bwd")
+    in_bytes = sum(t.numel() * t.element_size() for t in list(x.values()) + [dout])
     cfg["l2"] = (f"inputs larger than L2 (x and weights {in_bytes / 2**20:.0f} MiB together, "
                  "L2 126 MB); no flush")
     line = {
@@ -353,15 +382,18 @@ def main_ffn(args, w):
         "frac_of_peak": {"measured_burst": value / world / pk.get("bf16_tflops", 1590.0),
                          "measured_sustained": value / world / sustained,
                          "nominal_2250": value / world / NOMINAL_BF16_TFLOPS},
-        "roofline": {"bound": "tensor", "kernel": "ffn_gemm_sm100", "achieved": ach,
+        "fwd_tflops": fwd_flops / (fwd_t * 1e-3) / 1e12, "fwd_ms": fwd_t,
+        "bwd_tflops": ach, "bwd_ms": bwd_t,
+        "roofline": {"bound": "tensor", "kernel": "ffn_gemm_sm100 (lca_ffn_bwd)", "achieved": ach,
                      "peak": sustained, "unit": "TFLOP/s", "frac": ach / sustained,
                      "peak_kind": f"{pk_kind} sustained bf16",
                      "traffic": tr["dram_bytes_per_launch"] if tr else None,
                      "frac_of_nominal_2250": ach / NOMINAL_BF16_TFLOPS,
-                     "timing": "CUDA events around the whole lca_ffn_fwd call (both products "
-                               "of every block), median over timed steps"},
+                     "timing": "CUDA events around the whole lca_ffn_bwd call (six products per "
+                               "block, 16 T h f FLOPs with the recompute), median over timed "
+                               "steps"},
         "clocks": clk,
-        "gpu_launches": args.steps * 2 * n_blocks,
+        "gpu_launches": args.steps * 8 * n_blocks,
         "e2e": e2e,
     }
     if not args.no_cpu_baseline and world == 1:

@@ -161,8 +161,13 @@ class FfnWorkload:
     w_std: float = 0.02
 
     def flops(self) -> float:
-        """Three products of 2*T*h*f each (gate, up, down)."""
+        """Forward: three products of 2*T*h*f each (gate, up, down)."""
         return 6.0 * self.T * self.h * self.f
+
+    def bwd_flops(self) -> float:
+        """Backward: eight products of 2*T*h*f (dH; gate and up recomputed;
+        dx from dG and dU; three weight gradients)."""
+        return 16.0 * self.T * self.h * self.f
 
 
 FFN_WORKLOADS = {
