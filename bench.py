@@ -157,6 +157,45 @@ def whole_job_tflops(flops_per_step, world, steps, max_ms):
     return flops_per_step * world * steps / (max_ms * 1e-3) / 1e12
 
 
+def pipelined_e2e(torch, dev, sets, in_names, out_names, host_in, host_out, compute, n):
+    """Time n end-to-end steps through pinned host memory: every step uploads
+    its inputs (host_in -> set[in_names]), computes, and downloads its
+    results (set[out_names] -> host_out).  Two device sets alternate, with
+    uploads on one copy stream and downloads on another, so step i+1's upload
+    and step i-1's download overlap step i's compute (a training input
+    pipeline).  Returns the device time in ms from the first upload to the
+    last download."""
+    up, down, comp = (torch.cuda.Stream(dev) for _ in range(3))
+    ev = lambda: torch.cuda.Event()
+    in_ready, done, drained = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    start.record(up)
+    for i in range(n):
+        b = i % 2
+        S = sets[b]
+        if i >= 2:
+            up.wait_event(done[b])      # step i-2 no longer reads this set's inputs
+        with torch.cuda.stream(up):
+            for name, h in zip(in_names, host_in):
+                S[name].copy_(h, non_blocking=True)
+        in_ready[b].record(up)
+        comp.wait_event(in_ready[b])
+        if i >= 2:
+            comp.wait_event(drained[b])  # step i-2's results have left this set
+        compute(S, comp)
+        done[b].record(comp)
+        down.wait_event(done[b])
+        with torch.cuda.stream(down):
+            for h, name in zip(host_out, out_names):
+                h.copy_(S[name], non_blocking=True)
+        drained[b].record(down)
+    up.wait_event(drained[(n - 1) % 2])  # the download stream runs in order
+    end.record(up)
+    end.synchronize()
+    return start.elapsed_time(end)
+
+
 # ---------------------------------------------------------------- CPU oracle
 
 def oracle_sample(w, seconds_target=12.0, max_rows=None):
@@ -293,18 +332,22 @@ def main_ffn(args, w):
     fwd_flops, bwd_flops = w.flops(), w.bwd_flops()
     torch.cuda.synchronize()
 
-    def step(ev=None):
+    primary = {"x": x["x"], "dout": dout, "out": out, "dx": dx}
+
+    def step(ev=None, S=None, st=None):
+        S = S or primary
+        st = st or stream
         if ev:
-            ev[0].record(stream)
-        lca.ffn_fwd(x["x"], x["w_gate"], x["w_up"], x["w_down"], block_tokens=w.block, out=out,
-                    workspace=ws, stream=stream)
+            ev[0].record(st)
+        lca.ffn_fwd(S["x"], x["w_gate"], x["w_up"], x["w_down"], block_tokens=w.block,
+                    out=S["out"], workspace=ws, stream=st)
         if ev:
-            ev[1].record(stream)
-        lca.ffn_bwd(x["x"], x["w_gate"], x["w_up"], x["w_down"], dout, block_tokens=w.block,
-                    dx=dx, dw_gate=dws[0], dw_up=dws[1], dw_down=dws[2], workspace=ws,
-                    stream=stream)
+            ev[1].record(st)
+        lca.ffn_bwd(S["x"], x["w_gate"], x["w_up"], x["w_down"], S["dout"],
+                    block_tokens=w.block, dx=S["dx"], dw_gate=dws[0], dw_up=dws[1],
+                    dw_down=dws[2], workspace=ws, stream=st)
         if ev:
-            ev[2].record(stream)
+            ev[2].record(st)
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
@@ -333,34 +376,24 @@ def main_ffn(args, w):
 
     e2e = None
     if not args.no_e2e:
-        hx = x["x"].cpu().pin_memory()
-        hdo = dout.cpu().pin_memory()
-        hout = torch.empty_like(out, device="cpu").pin_memory()
-        hdx = torch.empty_like(dx, device="cpu").pin_memory()
-        with torch.cuda.stream(stream):
-            def e2e_step():
-                x["x"].copy_(hx, non_blocking=True)
-                dout.copy_(hdo, non_blocking=True)
-                step()
-                hout.copy_(out, non_blocking=True)
-                hdx.copy_(dx, non_blocking=True)
-            e2e_step()
-            stream.synchronize()
-            n_e2e = max(2, min(args.steps, 5))
-            if world > 1:
-                dist.barrier()
-            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            s0.record(stream)
-            for _ in range(n_e2e):
-                e2e_step()
-            s1.record(stream)
-            s1.synchronize()
-        e_ms = max_over_ranks(s0.elapsed_time(s1), dev)
+        in_names, out_names = ["x", "dout"], ["out", "dx"]
+        host_in = [primary[n].cpu().pin_memory() for n in in_names]
+        host_out = [torch.empty_like(primary[n], device="cpu").pin_memory() for n in out_names]
+        sets = [primary, {n: torch.empty_like(t) for n, t in primary.items()}]
+        compute = lambda S, st: step(S=S, st=st)
+        pipelined_e2e(torch, dev, sets, in_names, out_names, host_in, host_out, compute, 2)
+        n_e2e = max(3, min(args.steps, 6))
+        if world > 1:
+            dist.barrier()
+        e_ms = max_over_ranks(pipelined_e2e(torch, dev, sets, in_names, out_names, host_in,
+                                            host_out, compute, n_e2e), dev)
         e2e = {"value": whole_job_tflops(fwd_flops + bwd_flops, world, n_e2e, e_ms),
                "unit": "TFLOP/s",
-               "h2d_bytes_per_step": 2 * hx.numel() * hx.element_size(),
-               "d2h_bytes_per_step": 2 * hout.numel() * hout.element_size(),
-               "ms_per_step": e_ms / n_e2e}
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in host_in),
+               "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in host_out),
+               "ms_per_step": e_ms / n_e2e,
+               "pipelining": "two device buffer sets; uploads and downloads on their own "
+                             "streams overlap the neighbouring steps' compute"}
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -479,32 +512,38 @@ def main():
             ws = torch.empty(lca.varlen_workspace_size(q, k, cu, max_len), device=dev,
                              dtype=torch.uint8)
 
-    def step(ev=None):
+    primary = {"q": q, "k": k, "v": v, "out": out, "lse": lse}
+    if w.backward:
+        primary.update(dout=dout, dq=dq, dk=dk, dv=dv)
+
+    def step(ev=None, S=None, st=None):
+        S = S or primary
+        st = st or stream
+        q, k, v, out, lse = S["q"], S["k"], S["v"], S["out"], S["lse"]
         if ev:
-            ev[0].record(stream)
+            ev[0].record(st)
         if w.packed:
             lca.attn_fwd_varlen(q, k, v, cu, max_len, causal=w.causal, kv_chunk=w.kv_chunk,
-                                order=w.order, q_block=w.q_block, out=out, lse=lse,
-                                stream=stream)
+                                order=w.order, q_block=w.q_block, out=out, lse=lse, stream=st)
         elif w.s2:
             lca.s2attn_fwd(q, k, v, w.group, w.shift_heads, causal=w.causal, out=out, lse=lse,
-                           stream=stream)
+                           stream=st)
         else:
             lca.attn_fwd(q, k, v, causal=w.causal, kv_chunk=w.kv_chunk, order=w.order,
-                         q_block=w.q_block, out=out, lse=lse, stream=stream)
+                         q_block=w.q_block, out=out, lse=lse, stream=st)
         if ev:
-            ev[1].record(stream)
+            ev[1].record(st)
+        if w.backward:
+            g = dict(dq=S["dq"], dk=S["dk"], dv=S["dv"], workspace=ws, stream=st)
         if w.backward and w.packed:
-            lca.attn_bwd_varlen(q, k, v, out, lse, dout, cu, max_len, causal=w.causal, dq=dq,
-                                dk=dk, dv=dv, workspace=ws, stream=stream)
+            lca.attn_bwd_varlen(q, k, v, out, lse, S["dout"], cu, max_len, causal=w.causal, **g)
         elif w.backward and w.s2:
-            lca.s2attn_bwd(q, k, v, out, lse, dout, w.group, w.shift_heads, causal=w.causal,
-                           dq=dq, dk=dk, dv=dv, workspace=ws, stream=stream)
+            lca.s2attn_bwd(q, k, v, out, lse, S["dout"], w.group, w.shift_heads,
+                           causal=w.causal, **g)
         elif w.backward:
-            lca.attn_bwd(q, k, v, out, lse, dout, causal=w.causal, dq=dq, dk=dk, dv=dv,
-                         workspace=ws, stream=stream)
+            lca.attn_bwd(q, k, v, out, lse, S["dout"], causal=w.causal, **g)
         if ev:
-            ev[2].record(stream)
+            ev[2].record(st)
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
@@ -541,39 +580,24 @@ def main():
     # ---- end to end through the C ABI with pinned host buffers
     e2e = None
     if not args.no_e2e:
-        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
-        hdo = dout.cpu().pin_memory() if w.backward else None
-        res = [torch.empty_like(t, device="cpu").pin_memory()
-               for t in ([out, lse] + ([dq, dk, dv] if w.backward else []))]
-        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv) + ((hdo,) if hdo is not None else ()))
-        d2h = sum(t.numel() * t.element_size() for t in res)
-
-        def e2e_step():
-            q.copy_(hq, non_blocking=True)
-            k.copy_(hk, non_blocking=True)
-            v.copy_(hv, non_blocking=True)
-            if hdo is not None:
-                dout.copy_(hdo, non_blocking=True)
-            step()
-            for r, d in zip(res, [out, lse] + ([dq, dk, dv] if w.backward else [])):
-                r.copy_(d, non_blocking=True)
-
-        with torch.cuda.stream(stream):
-            e2e_step()
-            stream.synchronize()
-            n_e2e = max(2, min(args.steps, 5))
-            if world > 1:
-                dist.barrier()
-            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            s0.record(stream)
-            for _ in range(n_e2e):
-                e2e_step()
-            s1.record(stream)
-            s1.synchronize()
-        e_ms = max_over_ranks(s0.elapsed_time(s1), dev)
+        in_names = ["q", "k", "v"] + (["dout"] if w.backward else [])
+        out_names = ["out", "lse"] + (["dq", "dk", "dv"] if w.backward else [])
+        host_in = [primary[n].cpu().pin_memory() for n in in_names]
+        host_out = [torch.empty_like(primary[n], device="cpu").pin_memory() for n in out_names]
+        sets = [primary, {n: torch.empty_like(t) for n, t in primary.items()}]
+        compute = lambda S, st: step(S=S, st=st)
+        pipelined_e2e(torch, dev, sets, in_names, out_names, host_in, host_out, compute, 2)
+        n_e2e = max(3, min(args.steps, 6))
+        if world > 1:
+            dist.barrier()
+        e_ms = max_over_ranks(pipelined_e2e(torch, dev, sets, in_names, out_names, host_in,
+                                            host_out, compute, n_e2e), dev)
         e2e = {"value": whole_job_tflops(flops_step, world, n_e2e, e_ms), "unit": "TFLOP/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": e_ms / n_e2e}
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in host_in),
+               "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in host_out),
+               "ms_per_step": e_ms / n_e2e,
+               "pipelining": "two device buffer sets; uploads and downloads on their own "
+                             "streams overlap the neighbouring steps' compute"}
 
     if world > 1:
         dist.barrier()
