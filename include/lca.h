@@ -191,17 +191,38 @@ LCA_API lca_status lca_attn_bwd_noalloc(const lca_shape* shape, const void* q,
  *   inside the kernel, no tensor is rolled.  shift_heads == 0 gives the
  *   unshifted short attention; group == S with shift_heads == 0 is full
  *   attention.
- *   Errors: as lca_attn_fwd, plus LCA_ERR_INVALID_ARG when group does not
- *   divide S, group/2 is not a multiple of the tile, shift_heads is outside
- *   [0, Hq], or the shifted heads do not cover whole grouped-query groups.
+ *   When group/2 is a whole number of tiles (128 bf16, 64 fp32) the shift
+ *   lives in the kernels' tile coordinates and no workspace is needed.
+ *   Other even groups (LongLoRA's 100K context: S = 100000, group 25000)
+ *   need lca_s2attn_fwd_ws: the heads are rolled into its workspace, the
+ *   groups run as a packed batch, and the results are rolled back.
+ *   Errors: as lca_attn_fwd, plus LCA_ERR_INVALID_ARG when group is odd or
+ *   does not divide S, shift_heads is outside [0, Hq], or the shifted heads
+ *   do not cover whole grouped-query groups; LCA_ERR_WORKSPACE from
+ *   lca_s2attn_fwd for a group that needs a workspace.
  * ------------------------------------------------------------------------- */
 LCA_API lca_status lca_s2attn_fwd(const lca_shape* shape, const void* q, const void* k,
                           const void* v, int causal, int64_t group,
                           int64_t shift_heads, void* out, float* lse,
                           void* stream);
 
+/* lca_s2attn_fwd_ws -- lca_s2attn_fwd with a workspace of at least
+ * lca_s2attn_fwd_workspace_size bytes (0 for groups whose half is a whole
+ * number of tiles, then workspace may be NULL). */
+LCA_API size_t lca_s2attn_fwd_workspace_size(const lca_shape* shape, int64_t group,
+                                             int64_t shift_heads);
+LCA_API lca_status lca_s2attn_fwd_ws(const lca_shape* shape, const void* q, const void* k,
+                                     const void* v, int causal, int64_t group,
+                                     int64_t shift_heads, void* out, float* lse,
+                                     void* workspace, size_t ws_bytes, void* stream);
+
 /* lca_s2attn_bwd -- gradients of S2-Attn; arguments as lca_attn_bwd plus
- * group/shift_heads as lca_s2attn_fwd. */
+ * group/shift_heads as lca_s2attn_fwd.  The workspace must hold
+ * lca_s2attn_bwd_workspace_size bytes (lca_attn_bwd_workspace_size when
+ * group/2 is a whole number of tiles; more otherwise, for the rolled
+ * tensors). */
+LCA_API size_t lca_s2attn_bwd_workspace_size(const lca_shape* shape, int64_t group,
+                                             int64_t shift_heads);
 LCA_API lca_status lca_s2attn_bwd(const lca_shape* shape, const void* q, const void* k,
                           const void* v, const void* out, const float* lse,
                           const void* dout, int causal, int64_t group,

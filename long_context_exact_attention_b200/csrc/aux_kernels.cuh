@@ -7,6 +7,8 @@
 //   lse_merge    combine two partial (O, lse) results over disjoint key
 //                sets (Ring Attention with Blockwise Transformers, Summary:
 //                per-block results combine independently of order)
+//   s2_roll_*    LongLoRA's shift as a row permutation, for groups whose
+//                half is not a whole number of tiles
 #pragma once
 
 #include <cuda_bf16.h>
@@ -80,6 +82,60 @@ __global__ void bwd_rowdot(const T* __restrict__ out, const T* __restrict__ dout
     Dst[dst] = acc;
     lse_pad[dst] = lse[l0 + s];
   }
+}
+
+// S2-Attn for groups whose half is not a whole number of tiles: shifted
+// position p of a shifted head holds token (p + group/2) mod S (LongLoRA,
+// Summary).  s2_roll_rows moves whole rows between the original layout
+// [B, S, H, row] and the position layout (gather: position <- token;
+// scatter: token <- position); heads h >= first_shifted are rolled, the
+// others copied.  `vec` 16-byte words per row, one word per thread.
+template <bool kScatter>
+__global__ void s2_roll_rows(const uint4* __restrict__ src, uint4* __restrict__ dst, int B,
+                             int S, int H, int first_shifted, int half, int vec) {
+  const int64_t n = static_cast<int64_t>(B) * S * H * vec;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int w = static_cast<int>(i % vec);
+    const int64_t row = i / vec;  // (b, p, h) in the position layout
+    const int h = static_cast<int>(row % H);
+    const int64_t bp = row / H;
+    const int p = static_cast<int>(bp % S);
+    const int64_t b = bp / S;
+    const int tok = h >= first_shifted ? (p + half) % S : p;
+    const int64_t trow = ((b * S + tok) * H + h) * vec + w;
+    if (kScatter)
+      dst[trow] = src[i];
+    else
+      dst[i] = src[trow];
+  }
+}
+
+// lse between the original layout [B, H, S] and the packed position layout
+// [H, B*S] of the same roll.
+template <bool kScatter>
+__global__ void s2_roll_lse(const float* __restrict__ src, float* __restrict__ dst, int B, int S,
+                            int H, int first_shifted, int half) {
+  const int64_t n = static_cast<int64_t>(B) * S * H;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int h = static_cast<int>(i / (static_cast<int64_t>(B) * S));
+    const int64_t bp = i % (static_cast<int64_t>(B) * S);  // packed position
+    const int p = static_cast<int>(bp % S);
+    const int64_t b = bp / S;
+    const int tok = h >= first_shifted ? (p + half) % S : p;
+    const int64_t o = (b * H + h) * S + tok;
+    if (kScatter)
+      dst[o] = src[i];
+    else
+      dst[i] = src[o];
+  }
+}
+
+// cu[i] = i * len for i = 0..n (packed offsets of n equal sequences).
+__global__ void fill_offsets(int* cu, int n, int len) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i <= n; i += gridDim.x * blockDim.x)
+    cu[i] = i * len;
 }
 
 // dq(bf16) = scale * acc, 8 elements per thread.

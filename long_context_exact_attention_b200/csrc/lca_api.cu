@@ -505,6 +505,179 @@ lca_status run_bwd(const Common& c, const AttnSched& s, const void* q, const voi
   return launched("attn_bwd_f32");
 }
 
+// ---------------------------------------------------------------- S2-Attn, any group
+// Groups whose half is not a whole number of tiles cannot be remapped in
+// tile coordinates (a shifted tile would wrap around the end of the
+// sequence inside one TMA box).  Then the heads are rolled into the
+// workspace in position order (shifted heads by group/2, the others
+// copied), the groups become a packed batch of B*S/group sequences of
+// `group` tokens for the packed kernels, and results are rolled back.
+struct S2Plan {
+  bool aligned;          // group/2 is a whole number of tiles: tile remap
+  int half;              // group / 2
+  int first_q, first_kv; // first shifted query / key-value head
+  int n_seq;             // B * S / group
+  int64_t group;
+};
+
+lca_status plan_s2(const Common& c, int64_t group, int64_t shift_heads, S2Plan* p) {
+  if (group <= 0 || group % 2 || c.S % group)
+    return fail(LCA_ERR_INVALID_ARG, "group must be even and divide S");
+  if (shift_heads < 0 || shift_heads > c.Hq)
+    return fail(LCA_ERR_INVALID_ARG, "shift_heads outside [0, Hq]");
+  const int rep = c.Hq / c.Hkv;
+  if ((c.Hq - shift_heads) % rep)
+    return fail(LCA_ERR_INVALID_ARG, "shifted heads must cover whole grouped-query groups");
+  p->aligned = (group / 2) % c.tile == 0;
+  p->half = static_cast<int>(group / 2);
+  p->first_q = static_cast<int>(c.Hq - shift_heads);
+  p->first_kv = p->first_q / rep;
+  p->n_seq = static_cast<int>(static_cast<int64_t>(c.B) * c.S / group);
+  p->group = group;
+  return LCA_OK;
+}
+
+// The packed problem the rolled tensors form: one token axis of B*S rows,
+// n_seq sequences of `group` tokens.
+Common packed_of(const Common& c, const S2Plan& p, const int* cu) {
+  Common q = c;
+  q.n_seq = p.n_seq;
+  q.S = c.B * c.S;
+  q.B = 1;
+  q.S_seq = static_cast<int>(p.group);
+  q.cu = cu;
+  return q;
+}
+
+size_t align256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
+
+// Workspace regions of the rolled path, in order.
+struct S2Work {
+  size_t cu, q, kv, lse;  // bytes of the offsets, a query-side and a kv-side tensor, lse
+};
+S2Work s2_work(const Common& c, const S2Plan& p) {
+  const size_t e = c.dtype == LCA_BF16 ? 2 : 4;
+  const size_t rows = static_cast<size_t>(c.B) * c.S;
+  return {align256(static_cast<size_t>(p.n_seq + 1) * 4), align256(rows * c.Hq * c.d * e),
+          align256(rows * c.Hkv * c.d * e), align256(rows * c.Hq * 4)};
+}
+size_t s2_fwd_ws_bytes(const Common& c, const S2Plan& p) {
+  if (p.aligned) return 0;
+  const S2Work w = s2_work(c, p);
+  return w.cu + 2 * w.q + 2 * w.kv + w.lse;  // cu | q | k | v | out | lse
+}
+size_t s2_bwd_ws_bytes(const Common& c, const S2Plan& p) {
+  if (p.aligned) return ws_bytes_of(c);
+  const S2Work w = s2_work(c, p);
+  // cu | q | k | v | out | dout | lse | dq | dk | dv | the packed backward's own
+  return w.cu + 4 * w.q + 4 * w.kv + w.lse + ws_bytes_of(packed_of(c, p, nullptr));
+}
+
+template <bool kScatter>
+lca_status roll_rows(const void* src, void* dst, const Common& c, int H, int first, int half,
+                     cudaStream_t st) {
+  const int e = c.dtype == LCA_BF16 ? 2 : 4;
+  const int vec = c.d * e / 16;
+  const int64_t n = static_cast<int64_t>(c.B) * c.S * H * vec;
+  const unsigned blocks = static_cast<unsigned>(std::min<int64_t>((n + 255) / 256, 148 * 16));
+  s2_roll_rows<kScatter><<<blocks, 256, 0, st>>>(static_cast<const uint4*>(src),
+                                                 static_cast<uint4*>(dst), c.B, c.S, H, first,
+                                                 half, vec);
+  return launched("s2_roll_rows");
+}
+
+template <bool kScatter>
+lca_status roll_lse(const float* src, float* dst, const Common& c, int first, int half,
+                    cudaStream_t st) {
+  const int64_t n = static_cast<int64_t>(c.B) * c.S * c.Hq;
+  const unsigned blocks = static_cast<unsigned>(std::min<int64_t>((n + 255) / 256, 148 * 16));
+  s2_roll_lse<kScatter><<<blocks, 256, 0, st>>>(src, dst, c.B, c.S, c.Hq, first, half);
+  return launched("s2_roll_lse");
+}
+
+lca_status s2_fwd_rolled(const Common& c, const S2Plan& p, int causal, const void* q,
+                         const void* k, const void* v, void* out, float* lse, void* ws,
+                         size_t ws_bytes, cudaStream_t st) {
+  if (!ws) return fail(LCA_ERR_WORKSPACE, "workspace is NULL (group/2 is not a whole number of tiles)");
+  if (ws_bytes < s2_fwd_ws_bytes(c, p))
+    return fail(LCA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes,
+                s2_fwd_ws_bytes(c, p));
+  if (!aligned16(ws)) return fail(LCA_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+  const S2Work w = s2_work(c, p);
+  char* b = static_cast<char*>(ws);
+  int* cu = reinterpret_cast<int*>(b);
+  void* qr = b + w.cu;
+  void* kr = b + w.cu + w.q;
+  void* vr = b + w.cu + w.q + w.kv;
+  void* outr = b + w.cu + w.q + 2 * w.kv;
+  float* lser = reinterpret_cast<float*>(b + w.cu + 2 * w.q + 2 * w.kv);
+  fill_offsets<<<(p.n_seq + 256) / 256, 256, 0, st>>>(cu, p.n_seq, static_cast<int>(p.group));
+  lca_status r;
+  if ((r = launched("fill_offsets")) != LCA_OK) return r;
+  if ((r = roll_rows<false>(q, qr, c, c.Hq, p.first_q, p.half, st)) != LCA_OK) return r;
+  if ((r = roll_rows<false>(k, kr, c, c.Hkv, p.first_kv, p.half, st)) != LCA_OK) return r;
+  if ((r = roll_rows<false>(v, vr, c, c.Hkv, p.first_kv, p.half, st)) != LCA_OK) return r;
+  const Common pc = packed_of(c, p, cu);
+  AttnSched s;
+  if ((r = make_chunk_sched(pc, causal, 0, nullptr, &s)) != LCA_OK) return r;
+  if ((r = run_fwd(pc, s, qr, kr, vr, outr, lser, kDefaultBudget, st)) != LCA_OK) return r;
+  if ((r = roll_rows<true>(outr, out, c, c.Hq, p.first_q, p.half, st)) != LCA_OK) return r;
+  return roll_lse<true>(lser, lse, c, p.first_q, p.half, st);
+}
+
+lca_status s2_bwd_rolled(const Common& c, const S2Plan& p, int causal, const void* q,
+                         const void* k, const void* v, const void* out, const float* lse,
+                         const void* dout, void* dq, void* dk, void* dv, void* ws,
+                         size_t ws_bytes, cudaStream_t st) {
+  if (!ws) return fail(LCA_ERR_WORKSPACE, "workspace is NULL");
+  if (ws_bytes < s2_bwd_ws_bytes(c, p))
+    return fail(LCA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes,
+                s2_bwd_ws_bytes(c, p));
+  if (!aligned16(ws)) return fail(LCA_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+  const S2Work w = s2_work(c, p);
+  char* b = static_cast<char*>(ws);
+  size_t o = 0;
+  int* cu = reinterpret_cast<int*>(b + o);
+  o += w.cu;
+  void* qr = b + o;
+  o += w.q;
+  void* kr = b + o;
+  o += w.kv;
+  void* vr = b + o;
+  o += w.kv;
+  void* outr = b + o;
+  o += w.q;
+  void* dor = b + o;
+  o += w.q;
+  float* lser = reinterpret_cast<float*>(b + o);
+  o += w.lse;
+  void* dqr = b + o;
+  o += w.q;
+  void* dkr = b + o;
+  o += w.kv;
+  void* dvr = b + o;
+  o += w.kv;
+  void* rest = b + o;
+  fill_offsets<<<(p.n_seq + 256) / 256, 256, 0, st>>>(cu, p.n_seq, static_cast<int>(p.group));
+  lca_status r;
+  if ((r = launched("fill_offsets")) != LCA_OK) return r;
+  if ((r = roll_rows<false>(q, qr, c, c.Hq, p.first_q, p.half, st)) != LCA_OK) return r;
+  if ((r = roll_rows<false>(k, kr, c, c.Hkv, p.first_kv, p.half, st)) != LCA_OK) return r;
+  if ((r = roll_rows<false>(v, vr, c, c.Hkv, p.first_kv, p.half, st)) != LCA_OK) return r;
+  if ((r = roll_rows<false>(out, outr, c, c.Hq, p.first_q, p.half, st)) != LCA_OK) return r;
+  if ((r = roll_rows<false>(dout, dor, c, c.Hq, p.first_q, p.half, st)) != LCA_OK) return r;
+  if ((r = roll_lse<false>(lse, lser, c, p.first_q, p.half, st)) != LCA_OK) return r;
+  const Common pc = packed_of(c, p, cu);
+  AttnSched s;
+  if ((r = make_chunk_sched(pc, causal, 0, nullptr, &s)) != LCA_OK) return r;
+  if ((r = run_bwd(pc, s, qr, kr, vr, outr, lser, dor, dqr, dkr, dvr, rest, ws_bytes - o,
+                   kDefaultBudget, st)) != LCA_OK)
+    return r;
+  if ((r = roll_rows<true>(dqr, dq, c, c.Hq, p.first_q, p.half, st)) != LCA_OK) return r;
+  if ((r = roll_rows<true>(dkr, dk, c, c.Hkv, p.first_kv, p.half, st)) != LCA_OK) return r;
+  return roll_rows<true>(dvr, dv, c, c.Hkv, p.first_kv, p.half, st);
+}
+
 // ---------------------------------------------------------------- feedforward
 lca_status check_ffn(const lca_ffn_shape* sh, int64_t* block) {
   if (!sh) return fail(LCA_ERR_INVALID_ARG, "shape is NULL");
@@ -596,13 +769,46 @@ lca_status lca_attn_bwd(const lca_shape* shape, const void* q, const void* k, co
 lca_status lca_s2attn_fwd(const lca_shape* shape, const void* q, const void* k, const void* v,
                           int causal, int64_t group, int64_t shift_heads, void* out, float* lse,
                           void* stream) {
+  return lca_s2attn_fwd_ws(shape, q, k, v, causal, group, shift_heads, out, lse, nullptr, 0,
+                           stream);
+}
+
+size_t lca_s2attn_fwd_workspace_size(const lca_shape* shape, int64_t group,
+                                     int64_t shift_heads) {
+  Common c;
+  S2Plan p;
+  const std::string keep = t_last_error;
+  const bool ok = check_shape(shape, &c) == LCA_OK && plan_s2(c, group, shift_heads, &p) == LCA_OK;
+  t_last_error = keep;
+  return ok ? s2_fwd_ws_bytes(c, p) : 0;
+}
+
+size_t lca_s2attn_bwd_workspace_size(const lca_shape* shape, int64_t group,
+                                     int64_t shift_heads) {
+  Common c;
+  S2Plan p;
+  const std::string keep = t_last_error;
+  const bool ok = check_shape(shape, &c) == LCA_OK && plan_s2(c, group, shift_heads, &p) == LCA_OK;
+  t_last_error = keep;
+  return ok ? s2_bwd_ws_bytes(c, p) : 0;
+}
+
+lca_status lca_s2attn_fwd_ws(const lca_shape* shape, const void* q, const void* k,
+                             const void* v, int causal, int64_t group, int64_t shift_heads,
+                             void* out, float* lse, void* workspace, size_t ws_bytes,
+                             void* stream) {
   Common c;
   lca_status r = check_shape(shape, &c);
   if (r != LCA_OK) return r;
   if ((r = check_ptrs({q, k, v, out, lse})) != LCA_OK) return r;
+  S2Plan p;
+  if ((r = plan_s2(c, group, shift_heads, &p)) != LCA_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!p.aligned)
+    return s2_fwd_rolled(c, p, causal, q, k, v, out, lse, workspace, ws_bytes, st);
   AttnSched s;
   if ((r = make_s2_sched(c, causal, group, shift_heads, &s)) != LCA_OK) return r;
-  return run_fwd(c, s, q, k, v, out, lse, kDefaultBudget, static_cast<cudaStream_t>(stream));
+  return run_fwd(c, s, q, k, v, out, lse, kDefaultBudget, st);
 }
 
 lca_status lca_s2attn_bwd(const lca_shape* shape, const void* q, const void* k, const void* v,
@@ -613,10 +819,16 @@ lca_status lca_s2attn_bwd(const lca_shape* shape, const void* q, const void* k, 
   lca_status r = check_shape(shape, &c);
   if (r != LCA_OK) return r;
   if ((r = check_ptrs({q, k, v, out, lse, dout, dq, dk, dv})) != LCA_OK) return r;
+  S2Plan p;
+  if ((r = plan_s2(c, group, shift_heads, &p)) != LCA_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!p.aligned)
+    return s2_bwd_rolled(c, p, causal, q, k, v, out, lse, dout, dq, dk, dv, workspace, ws_bytes,
+                         st);
   AttnSched s;
   if ((r = make_s2_sched(c, causal, group, shift_heads, &s)) != LCA_OK) return r;
   return run_bwd(c, s, q, k, v, out, lse, dout, dq, dk, dv, workspace, ws_bytes, kDefaultBudget,
-                 static_cast<cudaStream_t>(stream));
+                 st);
 }
 
 lca_status lca_attn_fwd_varlen(const lca_shape* shape, const int32_t* cu_seqlens,

@@ -24,7 +24,8 @@ SYMBOLS = ["lca_attn_fwd", "lca_attn_bwd_workspace_size", "lca_attn_bwd",
            "lca_attn_bwd_noalloc",
            "lca_attn_fwd_varlen", "lca_attn_bwd_varlen_workspace_size", "lca_attn_bwd_varlen",
            "lca_ffn_workspace_size", "lca_ffn_fwd", "lca_ffn_bwd_workspace_size", "lca_ffn_bwd",
-           "lca_s2attn_fwd", "lca_s2attn_bwd", "lca_lse_merge", "lca_check",
+           "lca_s2attn_fwd", "lca_s2attn_fwd_ws", "lca_s2attn_fwd_workspace_size",
+           "lca_s2attn_bwd", "lca_s2attn_bwd_workspace_size", "lca_lse_merge", "lca_check",
            "lca_status_string", "lca_last_error", "lca_version"]
 
 
@@ -75,6 +76,10 @@ def lib() -> ctypes.CDLL:
         L.lca_attn_bwd_varlen.argtypes = [SP, P, I64, P, P, P, P, P, P, I32, P, P, P, P,
                                           ctypes.c_size_t, P]
         L.lca_s2attn_fwd.argtypes = [SP, P, P, P, I32, I64, I64, P, P, P]
+        L.lca_s2attn_fwd_ws.argtypes = [SP, P, P, P, I32, I64, I64, P, P, P, ctypes.c_size_t, P]
+        for fn in ("lca_s2attn_fwd_workspace_size", "lca_s2attn_bwd_workspace_size"):
+            getattr(L, fn).argtypes = [SP, I64, I64]
+            getattr(L, fn).restype = ctypes.c_size_t
         L.lca_s2attn_bwd.argtypes = [SP, P, P, P, P, P, P, I32, I64, I64, P, P, P, P,
                                      ctypes.c_size_t, P]
         L.lca_lse_merge.argtypes = [I64, I64, P, P, P, P, P, P, P]
@@ -89,6 +94,7 @@ def lib() -> ctypes.CDLL:
         L.lca_status_string.restype = ctypes.c_char_p
         L.lca_last_error.restype = ctypes.c_char_p
         for fn in ("lca_attn_fwd", "lca_attn_bwd", "lca_attn_bwd_noalloc", "lca_s2attn_fwd",
+                   "lca_s2attn_fwd_ws",
                    "lca_s2attn_bwd", "lca_attn_fwd_varlen", "lca_attn_bwd_varlen", "lca_ffn_fwd", "lca_ffn_bwd",
                    "lca_lse_merge", "lca_check"):
             getattr(L, fn).restype = ctypes.c_int
@@ -272,9 +278,18 @@ def attn_bwd_noalloc(q, k, v, out, lse, dout, causal: bool = True, scale=None, d
     return dq, dk, dv
 
 
+def s2attn_workspace_sizes(q, k, group: int, shift_heads: int):
+    """(forward, backward) workspace bytes of S2-Attn with this group."""
+    sh = _shape(q, k, None)
+    L = lib()
+    return (int(L.lca_s2attn_fwd_workspace_size(ctypes.byref(sh), int(group), int(shift_heads))),
+            int(L.lca_s2attn_bwd_workspace_size(ctypes.byref(sh), int(group), int(shift_heads))))
+
+
 def s2attn_fwd(q, k, v, group: int, shift_heads: int, causal: bool = True, scale=None,
-               out=None, lse=None, stream=None):
-    """LongLoRA S2-Attn forward (lca_s2attn_fwd).  Returns (out, lse)."""
+               out=None, lse=None, workspace=None, stream=None):
+    """LongLoRA S2-Attn forward (lca_s2attn_fwd_ws).  A workspace is only
+    needed when group/2 is not a whole number of tiles.  Returns (out, lse)."""
     sh = _shape(q, k, scale)
     _check_tensors(q.dtype, q, k, v)
     if out is None:
@@ -282,9 +297,13 @@ def s2attn_fwd(q, k, v, group: int, shift_heads: int, causal: bool = True, scale
     if lse is None:
         lse = torch.empty((q.shape[0], q.shape[2], q.shape[1]), device=q.device,
                           dtype=torch.float32)
-    _raise(lib().lca_s2attn_fwd(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), int(causal),
-                                int(group), int(shift_heads), _ptr(out), _ptr(lse),
-                                _stream(stream)))
+    if workspace is None:
+        n = s2attn_workspace_sizes(q, k, group, shift_heads)[0]
+        workspace = torch.empty(n, device=q.device, dtype=torch.uint8) if n else None
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _raise(lib().lca_s2attn_fwd_ws(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), int(causal),
+                                   int(group), int(shift_heads), _ptr(out), _ptr(lse),
+                                   _ptr(workspace), nbytes, _stream(stream)))
     return out, lse
 
 
@@ -293,6 +312,9 @@ def s2attn_bwd(q, k, v, out, lse, dout, group: int, shift_heads: int, causal: bo
     """LongLoRA S2-Attn backward (lca_s2attn_bwd).  Returns (dq, dk, dv)."""
     sh = _shape(q, k, scale)
     _check_tensors(q.dtype, q, k, v, out, dout)
+    if workspace is None:
+        n = s2attn_workspace_sizes(q, k, group, shift_heads)[1]
+        workspace = torch.empty(max(n, 16), device=q.device, dtype=torch.uint8)
     dq, dk, dv, workspace = _alloc_grads(q, k, v, dq, dk, dv, workspace)
     _raise(lib().lca_s2attn_bwd(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
                                 _ptr(lse), _ptr(dout), int(causal), int(group),

@@ -96,11 +96,20 @@ def test_s2_arguments_rejected():
     call = lambda g, sh_, shp=sh: L.lca_s2attn_fwd(ctypes.byref(shp), FAKE, FAKE, FAKE, 1, g,
                                                    sh_, FAKE, FAKE, None)
     assert call(384, 2) == 1          # does not divide S
-    assert call(128, 2) == 1          # half group not a multiple of the tile
+    assert call(127, 0, shape(S=127 * 8, Hq=4, Hkv=4)) == 1   # odd group
     assert call(512, 5) == 1          # more shifted heads than heads
     assert call(512, -1) == 1
     gqa = shape(S=1024, Hq=4, Hkv=2)
     assert call(512, 1, gqa) == 1     # shift boundary splits a query-head group
+    # half a group that is not a whole number of tiles needs a workspace
+    assert call(128, 2) == 5
+    assert L.lca_s2attn_fwd_workspace_size(ctypes.byref(sh), 512, 2) == 0
+    assert L.lca_s2attn_fwd_workspace_size(ctypes.byref(sh), 128, 2) > 0
+    assert L.lca_s2attn_bwd_workspace_size(ctypes.byref(sh), 512, 2) == \
+        L.lca_attn_bwd_workspace_size(ctypes.byref(sh))
+    assert L.lca_s2attn_bwd_workspace_size(ctypes.byref(sh), 128, 2) > \
+        L.lca_attn_bwd_workspace_size(ctypes.byref(sh))
+    assert L.lca_s2attn_bwd_workspace_size(ctypes.byref(sh), 384, 2) == 0
 
 
 def test_workspace_errors():
