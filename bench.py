@@ -506,11 +506,17 @@ def main():
                       dtype=torch.float32)
     if w.backward:
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-        ws = None if w.packed else torch.empty(lca.workspace_size(q, k), device=dev,
-                                               dtype=torch.uint8)
         if w.packed:
-            ws = torch.empty(lca.varlen_workspace_size(q, k, cu, max_len), device=dev,
-                             dtype=torch.uint8)
+            ws_n = lca.varlen_workspace_size(q, k, cu, max_len)
+        elif w.s2:
+            ws_n = lca.s2attn_workspace_sizes(q, k, w.group, w.shift_heads)[1]
+        else:
+            ws_n = lca.workspace_size(q, k)
+        ws = torch.empty(ws_n, device=dev, dtype=torch.uint8)
+    fws = None
+    if w.s2:
+        n = lca.s2attn_workspace_sizes(q, k, w.group, w.shift_heads)[0]
+        fws = torch.empty(n, device=dev, dtype=torch.uint8) if n else None
 
     primary = {"q": q, "k": k, "v": v, "out": out, "lse": lse}
     if w.backward:
@@ -527,7 +533,7 @@ def main():
                                 order=w.order, q_block=w.q_block, out=out, lse=lse, stream=st)
         elif w.s2:
             lca.s2attn_fwd(q, k, v, w.group, w.shift_heads, causal=w.causal, out=out, lse=lse,
-                           stream=st)
+                           workspace=fws, stream=st)
         else:
             lca.attn_fwd(q, k, v, causal=w.causal, kv_chunk=w.kv_chunk, order=w.order,
                          q_block=w.q_block, out=out, lse=lse, stream=st)

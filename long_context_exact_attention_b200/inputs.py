@@ -106,6 +106,11 @@ WORKLOADS = {
         Workload("llama2_13b_s1m", B=1, Hq=40, Hkv=40, S=1048576, d=128,
                  dtype="bf16", causal=True, seed=4, std=0.5, kv_chunk=16384,
                  q_block=16384, order="ring", backward=False),
+        # LongLoRA's 100K context: half a group (12500 tokens) is not a
+        # whole tile, so the rolled S2 path runs
+        Workload("longlora_s2_s100k", B=1, Hq=32, Hkv=32, S=100000, d=128,
+                 dtype="bf16", causal=True, seed=5, std=0.5, group=25000,
+                 shift_heads=16),
         # a quarter of the 32K layer's heads: the case ncu captures in full
         # (inputs 4 x 64 MiB, still larger than L2 together)
         Workload("llama2_7b_s32k_h8", B=1, Hq=8, Hkv=8, S=32768, d=128,

@@ -143,3 +143,40 @@ def test_llama2_13b_s1m_forward_sampled_blocks():
         rows += [r0, r0 + blk - 1] + (r0 + rng.integers(0, blk, 62)).tolist()
     rows = np.array(sorted(set(rows)))
     check_rows(x, out, lse, w, (0, 13, 26, 39), rows)
+
+
+def test_longlora_s2_s100k_sampled_rows():
+    """LongLoRA's 100K context (group 25000: half a group is not a whole
+    tile, so the rolled path runs), in the bench's launch configuration.
+    Sampled (head, position) rows: each is the oracle's full-row definition
+    over the row's group, with positions mapped to tokens by the oracle's
+    shift (position p of a shifted head holds token (p + group/2) mod S)."""
+    w = WORKLOADS["longlora_s2_s100k"]
+    x = make_inputs(w, "cuda", with_dout=False)
+    out, lse = lca.s2attn_fwd(x["q"], x["k"], x["v"], w.group, w.shift_heads, causal=True)
+    torch.cuda.synchronize()
+    lca.check()
+    S, G, half = w.S, w.group, w.group // 2
+    first = w.Hq - w.shift_heads
+    rng = np.random.default_rng(11)
+    pos = sorted(set([0, half - 1, half, G - 1, G, S - G, S - half - 1, S - half, S - 1] +
+                     rng.integers(0, S, 6).tolist()))
+    outs, refs = [], []
+    for h in (0, first - 1, first, w.Hq - 1):
+        shifted = h >= first
+        for p in pos:
+            g0 = p // G * G
+            toks = np.array([oracle.s2_token_of_position(t, S, G, shifted)
+                             for t in range(g0, g0 + G)])
+            ti = torch.as_tensor(toks, device="cuda")
+            qg = x["q"][:, ti, h:h + 1]
+            kg = x["k"][:, ti, h:h + 1]
+            vg = x["v"][:, ti, h:h + 1]
+            ro, rl = oracle.attention_rows(qg, kg, vg, True, 0, 0, [p - g0])
+            tok = int(toks[p - g0])
+            go = host(out[0, tok, h])
+            assert max_abs(go, ro[0]) <= BF16_OUT_ABS, (h, p, max_abs(go, ro[0]))
+            assert abs(float(lse[0, h, tok]) - float(rl[0])) <= BF16_LSE_ABS, (h, p)
+            outs.append(go)
+            refs.append(ro[0])
+    assert rel_fro(np.stack(outs), np.stack(refs)) <= BF16_OUT_REL
