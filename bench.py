@@ -214,6 +214,11 @@ def oracle_sample(w, seconds_target=12.0, max_rows=None):
         # a packed batch: the longest sequence, as a dense problem of its own
         i = max(range(len(w.lengths)), key=lambda j: w.lengths[j])
         tok = (sum(w.lengths[:i]), sum(w.lengths[:i + 1]))
+    elif w.s2:
+        # S2-Attn: the last group of head 0 (an unshifted head, so the
+        # group is a contiguous token range attended causally on its own)
+        assert w.shift_heads < w.Hq
+        tok = (w.S - w.group, w.S)
     S = tok[1] - tok[0]
     q = make_tensor(w, "q", "cpu", tok)[:, :, :w.Hq // w.Hkv]
     k = make_tensor(w, "k", "cpu", tok)[:, :, :1]
@@ -472,7 +477,8 @@ def main():
                        "d": w.d, "causal": w.causal},
             "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                              "sample": f"fp64 oracle fwd+bwd of the last {R} query rows of "
-                                       f"the {w.Hq // w.Hkv} query head(s) of key/value head 0"},
+                                       f"the {w.Hq // w.Hkv} query head(s) of key/value head 0"
+                                       + (" inside the last S2 group" if w.s2 else "")},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0},
         }
@@ -659,8 +665,9 @@ def main():
         line["cpu_baseline"] = {
             "value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "sample": f"fp64 oracle fwd+bwd of the last {R} query rows of the "
-                      f"{w.Hq // w.Hkv} query head(s) of key/value head 0, {reps} runs, "
-                      f"{dt:.2f} s each"}
+                      f"{w.Hq // w.Hkv} query head(s) of key/value head 0"
+                      + (" inside the last S2 group" if w.s2 else "")
+                      + f", {reps} runs, {dt:.2f} s each"}
     print(json.dumps(line), flush=True)
 
 
