@@ -63,10 +63,12 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_sha():
+def source_sha(files=None):
+    """Hash of the kernel sources `files` (names in csrc/; all of them when
+    None)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "long_context_exact_attention_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in sorted(files or os.listdir(csrc)):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
@@ -74,14 +76,15 @@ def source_sha():
 
 def traffic_record(kernel):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel sources; else None."""
+    on the current sources of that kernel (the files the record lists);
+    else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     rec = d.get(kernel)
-    if not rec or rec.get("source_sha") != source_sha():
+    if not rec or rec.get("source_sha") != source_sha(rec.get("sources")):
         return None
     return rec
 
