@@ -11,6 +11,11 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line(
         "markers", "gpu: needs a CUDA device (sm_100a) and the built library")
+    # liblca.so is a build artefact (not in version control): build it once
+    # if it is missing.  nvcc cross-compiles sm_100a without a GPU.
+    from long_context_exact_attention_b200 import build
+    if not os.path.exists(build.LIB):
+        build.build()
 
 
 def pytest_collection_modifyitems(config, items):
