@@ -441,3 +441,34 @@ def test_backward_rows_matches_full(causal):
         _, dkt, dvt = oracle.attention_backward_rows(q, k, v, do, True, 0, 0, range(12, S))
         np.testing.assert_allclose(dkt[12:], dk[0, 12:, 0], atol=1e-13)
         np.testing.assert_allclose(dvt[12:], dv[0, 12:, 0], atol=1e-13)
+
+
+# ---------------------------------------------------------------- power of the parity gates
+
+def test_lse_tolerance_catches_a_dropped_chunk():
+    """Dropping one key chunk from the merge moves lse by ln(1 - n_c/n_vis),
+    far beyond the 1e-3 lse bound (Ring Attention, Summary: every block must
+    be merged), on the bf16 workloads' 0.5-scaled inputs."""
+    rng = np.random.default_rng(71)
+    S, d, chunk = 512, 16, 64
+    q, k, v = (rand(1, S, 1, d, rng=rng, std=0.5) for _ in range(3))
+    _, ref = oracle.attention_forward(q, k, v, True)
+    n = S // chunk
+    _, dropped = oracle.chunked_attention_forward(q, k, v, True, chunk, list(range(1, n)))
+    later = slice(chunk, S)  # rows that should have seen chunk 0
+    assert np.min(np.abs(dropped[0, 0, later] - ref[0, 0, later])) > 1e-3
+
+
+def test_relative_output_gate_catches_a_zero_output():
+    """With 0.5-scaled inputs attention is near uniform and |O| shrinks like
+    1/sqrt(row), so at the 32K workload's length an all-zero output passes
+    the 2e-2 absolute bound; the per-head relative Frobenius bound of 1e-2
+    does not.  Sampled tail rows, each exact over every visible key."""
+    rng = np.random.default_rng(73)
+    S, d = 32768, 128
+    q, k, v = (rand(1, S, 1, d, rng=rng, std=0.5) for _ in range(3))
+    rows = np.sort(rng.choice(np.arange(S // 2, S), 64, replace=False))
+    ref, _ = oracle.attention_rows(q, k, v, True, 0, 0, rows)
+    zero = np.zeros_like(ref)
+    assert np.max(np.abs(zero - ref)) <= 2e-2                        # the loose gate passes
+    assert np.linalg.norm(zero - ref) / np.linalg.norm(ref) > 1e-2   # the strict gate fails it
