@@ -85,7 +85,7 @@ struct Args {
 };
 
 // Tile t -> (tm, tn): bands of kGroupM row tiles, column by column.
-__device__ __forceinline__ void tile_coords(int t, int n_tm, int n_tn, int& tm, int& tn) {
+__host__ __device__ inline void tile_coords(int t, int n_tm, int n_tn, int& tm, int& tn) {
   const int band = t / (kGroupM * n_tn);
   const int first = band * kGroupM;
   const int gm = n_tm - first < kGroupM ? n_tm - first : kGroupM;
