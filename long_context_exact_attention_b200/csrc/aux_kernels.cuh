@@ -29,58 +29,60 @@ __global__ void bwd_rowdot(const T* __restrict__ out, const T* __restrict__ dout
                            const float* __restrict__ lse, float* __restrict__ Dst,
                            float* __restrict__ lse_pad, int B, int S, int S_pad, int H,
                            const int* __restrict__ cu_seqlens) {
-  const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int64_t n = static_cast<int64_t>(B) * S_pad * H;
-  if (w >= n) return;
-  int h, s, b;
-  if (n <= 0xffffffffll) {  // 32-bit index arithmetic when it fits
-    const uint32_t w32 = static_cast<uint32_t>(w), hs = static_cast<uint32_t>(H) * S_pad;
-    h = static_cast<int>(w32 % static_cast<uint32_t>(H));
-    s = static_cast<int>((w32 / static_cast<uint32_t>(H)) % static_cast<uint32_t>(S_pad));
-    b = static_cast<int>(w32 / hs);
-  } else {
-    h = static_cast<int>(w % H);
-    s = static_cast<int>((w / H) % S_pad);
-    b = static_cast<int>(w / (static_cast<int64_t>(H) * S_pad));
-  }
-  int64_t r0 = static_cast<int64_t>(b) * S, l0 = (static_cast<int64_t>(b) * H + h) * S;
-  int len = S;
-  if (cu_seqlens) {
-    const int c0 = cu_seqlens[b], c1 = cu_seqlens[b + 1];
-    const bool valid = c0 >= 0 && c1 >= c0 && c1 <= S;
-    r0 = c0;
-    l0 = static_cast<int64_t>(h) * S + c0;
-    len = valid ? c1 - c0 : 0;
-  }
-  const int64_t dst = (static_cast<int64_t>(b) * H + h) * S_pad + s;
-  if (s >= len) {
-    if (lane == 0) {
-      Dst[dst] = 0.f;
-      lse_pad[dst] = INFINITY;
-    }
-    return;
-  }
-  const T* o = out + ((r0 + s) * H + h) * D;
-  const T* g = dout + ((r0 + s) * H + h) * D;
-  float acc = 0.f;
-#pragma unroll
-  for (int c = lane; c < D; c += 32) {
-    float ov, gv;
-    if constexpr (sizeof(T) == 2) {
-      ov = __bfloat162float(o[c]);
-      gv = __bfloat162float(g[c]);
+  const int64_t warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; w < n;
+       w += warps) {
+    int h, s, b;
+    if (n <= 0xffffffffll) {  // 32-bit index arithmetic when it fits
+      const uint32_t w32 = static_cast<uint32_t>(w), hs = static_cast<uint32_t>(H) * S_pad;
+      h = static_cast<int>(w32 % static_cast<uint32_t>(H));
+      s = static_cast<int>((w32 / static_cast<uint32_t>(H)) % static_cast<uint32_t>(S_pad));
+      b = static_cast<int>(w32 / hs);
     } else {
-      ov = o[c];
-      gv = g[c];
+      h = static_cast<int>(w % H);
+      s = static_cast<int>((w / H) % S_pad);
+      b = static_cast<int>(w / (static_cast<int64_t>(H) * S_pad));
     }
-    acc = fmaf(ov, gv, acc);
-  }
+    int64_t r0 = static_cast<int64_t>(b) * S, l0 = (static_cast<int64_t>(b) * H + h) * S;
+    int len = S;
+    if (cu_seqlens) {
+      const int c0 = cu_seqlens[b], c1 = cu_seqlens[b + 1];
+      const bool valid = c0 >= 0 && c1 >= c0 && c1 <= S;
+      r0 = c0;
+      l0 = static_cast<int64_t>(h) * S + c0;
+      len = valid ? c1 - c0 : 0;
+    }
+    const int64_t dst = (static_cast<int64_t>(b) * H + h) * S_pad + s;
+    if (s >= len) {
+      if (lane == 0) {
+        Dst[dst] = 0.f;
+        lse_pad[dst] = INFINITY;
+      }
+      continue;
+    }
+    const T* o = out + ((r0 + s) * H + h) * D;
+    const T* g = dout + ((r0 + s) * H + h) * D;
+    float acc = 0.f;
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (lane == 0) {
-    Dst[dst] = acc;
-    lse_pad[dst] = lse[l0 + s];
+    for (int c = lane; c < D; c += 32) {
+      float ov, gv;
+      if constexpr (sizeof(T) == 2) {
+        ov = __bfloat162float(o[c]);
+        gv = __bfloat162float(g[c]);
+      } else {
+        ov = o[c];
+        gv = g[c];
+      }
+      acc = fmaf(ov, gv, acc);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) {
+      Dst[dst] = acc;
+      lse_pad[dst] = lse[l0 + s];
+    }
   }
 }
 

@@ -96,8 +96,15 @@ lca_status check_shape(const lca_shape* sh, Common* c) {
 // [cu_seqlens[b], cu_seqlens[b+1]), none longer than max_seqlen.
 lca_status check_packed(const lca_shape* sh, const int32_t* cu_seqlens, int64_t max_seqlen,
                         Common* c) {
-  lca_status r = check_shape(sh, c);
+  if (!sh) return fail(LCA_ERR_INVALID_ARG, "shape is NULL");
+  // the tensors hold one batch entry of S = total tokens; B counts sequences
+  lca_shape one = *sh;
+  one.B = 1;
+  lca_status r = check_shape(&one, c);
   if (r != LCA_OK) return r;
+  if (sh->B <= 0 || sh->B > (1 << 20))
+    return fail(LCA_ERR_INVALID_ARG, "sequence count must lie in [1, 2^20]");
+  c->B = static_cast<int>(sh->B);
   if (!cu_seqlens) return fail(LCA_ERR_INVALID_ARG, "cu_seqlens is NULL");
   if (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)
     return fail(LCA_ERR_INVALID_ARG, "cu_seqlens not 4-byte aligned");
@@ -338,7 +345,11 @@ unsigned long long budget_of(const lca_opts* o) {
 lca_status run_fwd(const Common& c, const AttnSched& s, const void* q, const void* k,
                    const void* v, void* out, float* lse, unsigned long long budget,
                    cudaStream_t st) {
-  const unsigned grid = static_cast<unsigned>(s.n_tiles) * c.n_seq * c.Hq;
+  const int64_t grid64 = static_cast<int64_t>(s.n_tiles) * c.n_seq * c.Hq;
+  if (grid64 > 0x7fffffffll)
+    return fail(LCA_ERR_INVALID_ARG, "%lld query tiles exceed one launch",
+                static_cast<long long>(grid64));
+  const unsigned grid = static_cast<unsigned>(grid64);
   if (c.dtype == LCA_BF16) {
     // one CTA per pair of 128-row query tiles
     const unsigned grid2 = static_cast<unsigned>((s.n_tiles + 1) / 2) * c.n_seq * c.Hq;
@@ -422,8 +433,13 @@ lca_status run_bwd(const Common& c, const AttnSched& s, const void* q, const voi
   float* lse_pad = reinterpret_cast<float*>(static_cast<char*>(ws) + ws_d_bytes(c));
   const int64_t rows = static_cast<int64_t>(c.B) * c.S * c.Hq;
   const int64_t pad_rows = static_cast<int64_t>(c.n_seq) * S_pad * c.Hq;
-  const unsigned rd_blocks = static_cast<unsigned>((pad_rows * 32 + 255) / 256);
-  const unsigned grid = static_cast<unsigned>(s.n_tiles) * c.n_seq * c.Hkv;
+  const unsigned rd_blocks =
+      static_cast<unsigned>(std::min<int64_t>((pad_rows * 32 + 255) / 256, 148 * 64));
+  const int64_t grid64 = static_cast<int64_t>(s.n_tiles) * c.n_seq * c.Hkv;
+  if (grid64 > 0x7fffffffll)
+    return fail(LCA_ERR_INVALID_ARG, "%lld key tiles exceed one launch",
+                static_cast<long long>(grid64));
+  const unsigned grid = static_cast<unsigned>(grid64);
   cudaError_t e;
   lca_status r;
   if (c.dtype == LCA_BF16) {

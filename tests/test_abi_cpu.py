@@ -148,6 +148,16 @@ def test_varlen_arguments_rejected():
     assert fwd_varlen(shape(B=3, S=1000, d=64)) == 2
 
 
+def test_varlen_many_sequences_accepted():
+    # 2000 packed sequences over 3M tokens: sequences x tokens exceeds 2^31,
+    # which bounds only dense batches.  Validation gets past the shape to
+    # the (misaligned) output pointer, so nothing is launched.
+    sh = shape(B=2000, S=3_000_000)
+    assert fwd_varlen(sh, max_seqlen=4096,
+                      ptrs=[FAKE, FAKE, FAKE, MISALIGNED, FAKE]) == 1
+    assert b"pointer argument 3" in lca.lib().lca_last_error()
+
+
 def test_varlen_workspace_size():
     L = lca.lib()
     sh = shape(B=3, S=1000)
