@@ -23,3 +23,14 @@ def test_oracle_matches_frozen_fixture():
     o, l = oracle.s2attn_forward(inp["s2_q"], inp["s2_k"], inp["s2_v"], 4, 2, True)
     np.testing.assert_allclose(o, np.array(want["out"]), atol=1e-13)
     np.testing.assert_allclose(l, np.array(want["lse"]), atol=1e-13)
+    want = g["cases"]["packed_causal"]
+    o, l = oracle.packed_attention_forward(inp["q"][0], inp["k"][0], inp["v"][0], want["cu"], True)
+    np.testing.assert_allclose(np.nan_to_num(o, nan=0.0), np.array(want["out"]), atol=1e-13)
+    np.testing.assert_allclose(np.nan_to_num(l, nan=0.0), np.array(want["lse"]), atol=1e-13)
+    want = g["cases"]["ffn_block2"]
+    args = (inp["ffn_x"], inp["ffn_w_gate"], inp["ffn_w_up"], inp["ffn_w_down"])
+    np.testing.assert_allclose(oracle.ffn_forward(*args, block=2), np.array(want["out"]),
+                               atol=1e-13)
+    got = oracle.ffn_backward(*args, inp["ffn_dout"], block=2)
+    for name, a in zip(("dx", "dw_gate", "dw_up", "dw_down"), got):
+        np.testing.assert_allclose(a, np.array(want[name]), atol=1e-12, err_msg=name)
