@@ -86,6 +86,12 @@ __global__ void bwd_rowdot(const T* __restrict__ out, const T* __restrict__ dout
   }
 }
 
+// Token held by position p of head h under LongLoRA's shift: heads from
+// first_shifted on are rolled by half a group (LongLoRA, Summary).
+__host__ __device__ inline int s2_token(int p, int h, int first_shifted, int half, int S) {
+  return h >= first_shifted ? (p + half) % S : p;
+}
+
 // S2-Attn for groups whose half is not a whole number of tiles: shifted
 // position p of a shifted head holds token (p + group/2) mod S (LongLoRA,
 // Summary).  s2_roll_rows moves whole rows between the original layout
@@ -104,7 +110,7 @@ __global__ void s2_roll_rows(const uint4* __restrict__ src, uint4* __restrict__ 
     const int64_t bp = row / H;
     const int p = static_cast<int>(bp % S);
     const int64_t b = bp / S;
-    const int tok = h >= first_shifted ? (p + half) % S : p;
+    const int tok = s2_token(p, h, first_shifted, half, S);
     const int64_t trow = ((b * S + tok) * H + h) * vec + w;
     if (kScatter)
       dst[trow] = src[i];
@@ -125,7 +131,7 @@ __global__ void s2_roll_lse(const float* __restrict__ src, float* __restrict__ d
     const int64_t bp = i % (static_cast<int64_t>(B) * S);  // packed position
     const int p = static_cast<int>(bp % S);
     const int64_t b = bp / S;
-    const int tok = h >= first_shifted ? (p + half) % S : p;
+    const int tok = s2_token(p, h, first_shifted, half, S);
     const int64_t o = (b * H + h) * S + tok;
     if (kScatter)
       dst[o] = src[i];

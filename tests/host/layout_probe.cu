@@ -3,6 +3,7 @@
 // (sched.cuh).  Built and run by tests/test_layout_host.py.
 //   layout_probe tiles n_tm n_tn        -> "t tm tn" per tile
 //   layout_probe seq S_max tile S_tensor cu0 cu1 ...  -> "b ok tokb len n_tiles"
+//   layout_probe s2 S half H first_shifted -> "h p token" per head and position
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -10,6 +11,7 @@
 
 #include <cuda.h>
 
+#include "../../long_context_exact_attention_b200/csrc/aux_kernels.cuh"
 #include "../../long_context_exact_attention_b200/csrc/ffn_sm100.cuh"
 #include "../../long_context_exact_attention_b200/csrc/sched.cuh"
 
@@ -39,6 +41,12 @@ int main(int argc, char** argv) {
       const bool ok = lca::seq_view(s, b, S_tensor, &v);
       printf("%d %d %d %d %d\n", b, ok ? 1 : 0, v.tokb, v.len, v.n_tiles);
     }
+    return 0;
+  }
+  if (!strcmp(argv[1], "s2")) {
+    const int S = atoi(argv[2]), half = atoi(argv[3]), H = atoi(argv[4]), first = atoi(argv[5]);
+    for (int h = 0; h < H; ++h)
+      for (int p = 0; p < S; ++p) printf("%d %d %d\n", h, p, lca::s2_token(p, h, first, half, S));
     return 0;
   }
   return 2;

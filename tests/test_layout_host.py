@@ -2,7 +2,8 @@
 kernel's tile raster visits every output tile exactly once, in bands of 16
 row tiles walked column by column; and the packed-sequence view accepts
 exactly the in-order, in-range offsets no longer than the longest sequence
-(the kernels skip anything else and report it)."""
+(the kernels skip anything else and report it); and the S2 roll's position
+-> token map is the oracle's, a permutation of each head's tokens."""
 
 import os
 import subprocess
@@ -17,7 +18,8 @@ CSRC = os.path.join(HERE, "..", "long_context_exact_attention_b200", "csrc")
 
 @pytest.fixture(scope="module")
 def probe():
-    deps = [SRC] + [os.path.join(CSRC, f) for f in ("ffn_sm100.cuh", "sched.cuh", "ptx.cuh")]
+    deps = [SRC] + [os.path.join(CSRC, f) for f in ("ffn_sm100.cuh", "sched.cuh", "ptx.cuh",
+                                                     "aux_kernels.cuh")]
     if not os.path.exists(BIN) or os.path.getmtime(BIN) < max(map(os.path.getmtime, deps)):
         subprocess.run(["nvcc", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a",
                         "-x", "cu", SRC, "-o", BIN], check=True)
@@ -60,3 +62,16 @@ def test_packed_sequence_view(probe, cu, S_max, T, want):
         assert ok == w[0], (b, rows)
         if ok:
             assert (tokb, ln, nt) == w[1:], (b, rows)
+
+
+@pytest.mark.parametrize("S,G,H,shift", [(6000, 1500, 4, 2), (1200, 200, 2, 2), (400, 100, 2, 1),
+                                         (16, 4, 3, 0)])
+def test_s2_roll_map_matches_the_oracle(probe, S, G, H, shift):
+    import oracle
+    rows = probe("s2", S, G // 2, H, H - shift)
+    first = H - shift
+    for h in range(H):
+        toks = [t for hh, p, t in rows if hh == h]
+        assert sorted(toks) == list(range(S))             # a permutation of the tokens
+        want = [oracle.s2_token_of_position(p, S, G, h >= first) for p in range(S)]
+        assert toks == want
