@@ -75,3 +75,13 @@ def test_s2_roll_map_matches_the_oracle(probe, S, G, H, shift):
         assert sorted(toks) == list(range(S))             # a permutation of the tokens
         want = [oracle.s2_token_of_position(p, S, G, h >= first) for p in range(S)]
         assert toks == want
+
+
+def test_random_tile_rasters(probe):
+    import random
+    rng = random.Random(7)
+    for _ in range(20):
+        n_tm, n_tn = rng.randint(1, 60), rng.randint(1, 50)
+        rows = probe("tiles", n_tm, n_tn)
+        assert sorted((tm, tn) for _, tm, tn in rows) == \
+            [(m, n) for m in range(n_tm) for n in range(n_tn)]

@@ -140,3 +140,20 @@ def test_s2_walks(probe, causal, n, gt, st):
                                      if any(t == kt for (t, _, _) in walks[qt])]
     for t, (plain, shifted) in tok.items():
         assert plain == t and shifted == (t + st) % n
+
+
+def test_random_walks(probe):
+    """Seeded random schedules: lengths, tile sizes, chunk lengths (aligned
+    or not), orders and query blocks; every property above must hold."""
+    import random
+    rng = random.Random(2024)
+    for _ in range(40):
+        tile = rng.choice([2, 4, 8])
+        S = rng.randint(1, 70)
+        causal = rng.randint(0, 1)
+        kv_chunk = rng.choice([rng.randint(1, S), tile * rng.randint(1, 4), S])
+        order = rng.randint(0, 2)
+        n_chunks = -(-S // kv_chunk)
+        perm = tuple(rng.sample(range(n_chunks), n_chunks)) if order == 2 else ()
+        q_block = rng.choice([0, rng.randint(1, S)])
+        check_chunk_walks(probe, S, tile, causal, kv_chunk, order, q_block=q_block, perm=perm)
