@@ -32,7 +32,8 @@
 // same product, and the epilogue reads dH and writes dG, dU and H (zeros
 // for rows past M, so later products over whole 64-row K steps add
 // nothing from them); EPI_ACC32 -- adds the 256 columns into a float32
-// output.  Split K: the first half of K comes from (A0, B0), the second
+// output (two stacked outputs split at row m_split: dW_gate and dW_up come
+// from one product over [dG | dU]).  Split K: the first half of K comes from (A0, B0), the second
 // from (A1, B1).  Rows past M are computed from zero-filled rows and not
 // stored.
 #pragma once
@@ -75,13 +76,16 @@ struct Args {
   int a_off;         // A coordinate offset: rows (K-major) or K rows (MN-major)
   int b_off;         // B coordinate offset, likewise
   int ldo;           // row stride of the outputs, in elements
+  int ldo3;          // row stride of out3
   int ld_in;         // row stride of `in`
+  int m_split;       // EPI_ACC32: rows from m_split on go to out32b (M when unused)
   unsigned long long budget;
   __nv_bfloat16* out;   // C (EPI_STORE, EPI_SWIGLU), dG (EPI_SWIGLU_BWD)
   __nv_bfloat16* out2;  // dU (EPI_SWIGLU_BWD)
   __nv_bfloat16* out3;  // H (EPI_SWIGLU_BWD)
   const __nv_bfloat16* in;  // dH (EPI_SWIGLU_BWD)
-  float* out32;         // EPI_ACC32: C += A B^T
+  float* out32;         // EPI_ACC32: C += A B^T (rows below m_split)
+  float* out32b;        // EPI_ACC32: rows from m_split on, counted from m_split
 };
 
 // Tile t -> (tm, tn): bands of kGroupM row tiles, column by column.
@@ -144,6 +148,7 @@ __device__ __forceinline__ void ffn_epilogue(const ffn::Args& a, uint32_t acc, i
   } else if constexpr (kEpi == EPI_SWIGLU_BWD) {
     // rows past M (inside the block's last tile) are written as zeros
     const size_t wrow = static_cast<size_t>(row) * a.ldo;
+    const size_t hrow = static_cast<size_t>(row) * a.ldo3;
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
       float g[32], u[32];
@@ -190,7 +195,7 @@ __device__ __forceinline__ void ffn_epilogue(const ffn::Args& a, uint32_t acc, i
       }
       uint4* dg = reinterpret_cast<uint4*>(a.out + wrow + col);
       uint4* du = reinterpret_cast<uint4*>(a.out2 + wrow + col);
-      uint4* hh = reinterpret_cast<uint4*>(a.out3 + wrow + col);
+      uint4* hh = reinterpret_cast<uint4*>(a.out3 + hrow + col);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         dg[q] = make_uint4(pg[4 * q], pg[4 * q + 1], pg[4 * q + 2], pg[4 * q + 3]);
@@ -199,13 +204,16 @@ __device__ __forceinline__ void ffn_epilogue(const ffn::Args& a, uint32_t acc, i
       }
     }
   } else {  // EPI_ACC32
+    // two stacked outputs: a 128-row tile lies wholly on one side of m_split
+    float* base = row < a.m_split ? a.out32 + orow
+                                  : a.out32b + static_cast<size_t>(row - a.m_split) * a.ldo;
 #pragma unroll 1
     for (int c = 0; c < kBN / 32; ++c) {
       float v[32];
       __syncwarp();
       tmem_ld32(acc + c * 32, v);
       if (row_in) {
-        float4* dst = reinterpret_cast<float4*>(a.out32 + orow + tn * kBN + c * 32);
+        float4* dst = reinterpret_cast<float4*>(base + tn * kBN + c * 32);
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           float4 o = dst[q];

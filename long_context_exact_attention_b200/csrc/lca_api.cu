@@ -255,11 +255,11 @@ lca_status make_map_acc(CUtensorMap* m, const void* ptr, int64_t B, int64_t S, i
 // 128-byte swizzle: 128 rows for a K-major operand tile of the feedforward
 // products, 64 rows for an MN-major one.  Rows past the extent load as zeros.
 lca_status make_map_2d(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols,
-                       uint32_t box_rows = 128) {
+                       uint32_t box_rows = 128, int64_t row_stride = 0) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(LCA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_stride ? row_stride : cols) * 2};
   const cuuint32_t box[2] = {64, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
@@ -970,13 +970,12 @@ lca_status lca_ffn_bwd(const lca_ffn_shape* shape, const void* x, const void* w_
     return fail(LCA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, 4 * one);
   if (!aligned16(workspace)) return fail(LCA_ERR_INVALID_ARG, "workspace not 16-byte aligned");
   auto* ws = static_cast<__nv_bfloat16*>(workspace);
+  // dH [block, f] | [dG | dU] [block, 2f] | H [block, f]
   __nv_bfloat16* dH = ws;
-  __nv_bfloat16* dG = ws + block * f;
-  __nv_bfloat16* dU = ws + 2 * block * f;
+  __nv_bfloat16* dGU = ws + block * f;
   __nv_bfloat16* H = ws + 3 * block * f;
   // K-major views (boxes of 128 rows) and MN-major views (boxes of 64 rows)
-  CUtensorMap x_k, x_mn, do_k, do_mn, wg_k, wu_k, wg_mn, wu_mn, wd_mn, dg_k, du_k, dg_mn, du_mn,
-      h_mn;
+  CUtensorMap x_k, x_mn, do_k, do_mn, wg_k, wu_k, wg_mn, wu_mn, wd_mn, dg_k, du_k, dgu_mn, h_mn;
   if ((r = make_map_2d(&x_k, x, T, h)) != LCA_OK) return r;
   if ((r = make_map_2d(&x_mn, x, T, h, 64)) != LCA_OK) return r;
   if ((r = make_map_2d(&do_k, dout, T, h)) != LCA_OK) return r;
@@ -986,10 +985,9 @@ lca_status lca_ffn_bwd(const lca_ffn_shape* shape, const void* x, const void* w_
   if ((r = make_map_2d(&wg_mn, w_gate, f, h, 64)) != LCA_OK) return r;
   if ((r = make_map_2d(&wu_mn, w_up, f, h, 64)) != LCA_OK) return r;
   if ((r = make_map_2d(&wd_mn, w_down, h, f, 64)) != LCA_OK) return r;
-  if ((r = make_map_2d(&dg_k, dG, block, f)) != LCA_OK) return r;
-  if ((r = make_map_2d(&du_k, dU, block, f)) != LCA_OK) return r;
-  if ((r = make_map_2d(&dg_mn, dG, block, f, 64)) != LCA_OK) return r;
-  if ((r = make_map_2d(&du_mn, dU, block, f, 64)) != LCA_OK) return r;
+  if ((r = make_map_2d(&dg_k, dGU, block, f, 128, 2 * f)) != LCA_OK) return r;
+  if ((r = make_map_2d(&du_k, dGU + f, block, f, 128, 2 * f)) != LCA_OK) return r;
+  if ((r = make_map_2d(&dgu_mn, dGU, block, 2 * f, 64)) != LCA_OK) return r;
   if ((r = make_map_2d(&h_mn, H, block, f, 64)) != LCA_OK) return r;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   for (int64_t r0 = 0; r0 < T; r0 += block) {
@@ -1008,8 +1006,9 @@ lca_status lca_ffn_bwd(const lca_ffn_shape* shape, const void* x, const void* w_
     g = ffn::Args{};
     g.budget = kDefaultBudget;
     g.M = rows, g.K = static_cast<int>(h), g.n_tm = n_tm, g.n_tn = static_cast<int>(f / 128);
-    g.a_off = static_cast<int>(r0), g.b_off = 0, g.ldo = static_cast<int>(f);
-    g.ld_in = static_cast<int>(f), g.in = dH, g.out = dG, g.out2 = dU, g.out3 = H;
+    g.a_off = static_cast<int>(r0), g.b_off = 0, g.ldo = static_cast<int>(2 * f);
+    g.ldo3 = static_cast<int>(f), g.ld_in = static_cast<int>(f), g.in = dH;
+    g.out = dGU, g.out2 = dGU + f, g.out3 = H;
     if ((r = launch_ffn_gemm<ffn::EPI_SWIGLU_BWD, false, false, false>(x_k, x_k, wg_k, wu_k, g,
                                                                        10, st)) != LCA_OK)
       return r;
@@ -1022,21 +1021,19 @@ lca_status lca_ffn_bwd(const lca_ffn_shape* shape, const void* x, const void* w_
     if ((r = launch_ffn_gemm<ffn::EPI_STORE, false, true, true>(dg_k, du_k, wg_mn, wu_mn, g, 11,
                                                                 st)) != LCA_OK)
       return r;
-    // dW_gate += dG^T x, dW_up += dU^T x
+    // [dW_gate; dW_up] += [dG | dU]^T x: one product, rows split at f
     g = ffn::Args{};
     g.budget = kDefaultBudget;
-    g.M = static_cast<int>(f), g.K = k_rows, g.n_tm = static_cast<int>(f / ffn::kBM);
+    g.M = static_cast<int>(2 * f), g.K = k_rows, g.n_tm = static_cast<int>(2 * f / ffn::kBM);
     g.n_tn = static_cast<int>(h / ffn::kBN);
-    g.a_off = 0, g.b_off = static_cast<int>(r0), g.ldo = static_cast<int>(h), g.out32 = dw_gate;
-    if ((r = launch_ffn_gemm<ffn::EPI_ACC32, true, true, false>(dg_mn, dg_mn, x_mn, x_mn, g, 12,
-                                                                st)) != LCA_OK)
-      return r;
-    g.out32 = dw_up;
-    if ((r = launch_ffn_gemm<ffn::EPI_ACC32, true, true, false>(du_mn, du_mn, x_mn, x_mn, g, 12,
+    g.a_off = 0, g.b_off = static_cast<int>(r0), g.ldo = static_cast<int>(h);
+    g.m_split = static_cast<int>(f), g.out32 = dw_gate, g.out32b = dw_up;
+    if ((r = launch_ffn_gemm<ffn::EPI_ACC32, true, true, false>(dgu_mn, dgu_mn, x_mn, x_mn, g, 12,
                                                                 st)) != LCA_OK)
       return r;
     // dW_down += dout^T H
-    g.M = static_cast<int>(h), g.n_tm = static_cast<int>(h / ffn::kBM);
+    g.M = static_cast<int>(h), g.m_split = static_cast<int>(h), g.out32b = nullptr;
+    g.n_tm = static_cast<int>(h / ffn::kBM);
     g.n_tn = static_cast<int>(f / ffn::kBN);
     g.a_off = static_cast<int>(r0), g.b_off = 0, g.ldo = static_cast<int>(f), g.out32 = dw_down;
     if ((r = launch_ffn_gemm<ffn::EPI_ACC32, true, true, false>(do_mn, do_mn, h_mn, h_mn, g, 12,
