@@ -14,7 +14,8 @@ bound memory:
   analytic gradients ("Attention stays exact": Ring Attention with Blockwise
   Transformers for Near-Infinite Context, Summary; full attention with no
   approximations: sourcepulse project card of the 1M-context training
-  recipe, How It Works).
+  recipe, How It Works); and the partial result of one query block over one
+  key/value block at given positions, as a host of the ring computes it.
 * ``s2attn``     -- LongLoRA's shifted sparse attention taken literally:
   shift half the heads by half a group, split into groups, attend inside
   each group, shift back (LongLoRA: Efficient Fine-tuning of Long-Context
@@ -34,7 +35,7 @@ here is "parity unpinned".
 """
 
 from .attention import (attention_forward, attention_rows, attention_backward,
-                        attention_backward_rows, chunked_attention_forward)
+                        attention_backward_rows, block_attention, chunked_attention_forward)
 from .s2attn import s2attn_forward, s2attn_backward, s2_token_of_position
 from .merge import lse_merge
 from .packed import packed_attention_forward, packed_attention_backward
@@ -42,7 +43,7 @@ from .ffn import ffn_forward, ffn_backward, ffn_backward_columns, ffn_rows, silu
 
 __all__ = [
     "attention_forward", "attention_rows", "attention_backward",
-    "attention_backward_rows",
+    "attention_backward_rows", "block_attention",
     "chunked_attention_forward", "s2attn_forward", "s2attn_backward",
     "s2_token_of_position", "lse_merge", "packed_attention_forward",
     "packed_attention_backward", "ffn_forward", "ffn_backward", "ffn_backward_columns", "ffn_rows", "silu",

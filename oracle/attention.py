@@ -59,6 +59,11 @@ def _row_block(s_q, keys, causal, rows):
     return s
 
 
+def _row_dot_terms(p, dP):
+    """D_i = sum_j P_ij dP_ij, the row term of dS = P o (dP - D)."""
+    return np.sum(p * dP, axis=1)
+
+
 def _softmax_rows(s):
     """Return (P, lse) of each row of s (row max subtracted for range)."""
     mx = np.max(s, axis=1)
@@ -161,7 +166,7 @@ def attention_backward(q, k, v, dout, causal: bool, scale=None,
                     s = _row_block(s, kend, causal, rows)
                     p, _ = _softmax_rows(s)
                     dP = dO[r0:r1] @ V[:kend].T
-                    D = np.sum(p * dP, axis=1)
+                    D = _row_dot_terms(p, dP)
                     dS = p * (dP - D[:, None])
                     dv[b, :kend, gi] += p.T @ dO[r0:r1]
                     dq[b, r0:r1, hi] = sc * (dS @ K[:kend])
@@ -234,9 +239,46 @@ def attention_backward_rows(q, k, v, dout, causal: bool, b: int, g: int, rows,
         s = _row_block((Q @ K.T) * sc, S, causal, rows)
         p, _ = _softmax_rows(s)
         dP = dO @ V.T
-        D = np.sum(p * dP, axis=1)
+        D = _row_dot_terms(p, dP)
         dS = p * (dP - D[:, None])
         dq[:, r] = sc * (dS @ K)
         dk += sc * (dS.T @ Q)
         dv += p.T @ dO
     return dq, dk, dv
+
+
+def _position_mask(qpos, kpos):
+    """Causal visibility over absolute positions: [len(qpos), len(kpos)]."""
+    return kpos[None, :] <= qpos[:, None]
+
+
+def block_attention(q, k, v, q_pos0: int, k_pos0: int, causal: bool, scale=None):
+    """Partial attention of a query block over one key/value block, as a host
+    of the ring computes it (Ring Attention with Blockwise Transformers for
+    Near-Infinite Context, Summary: each host attends its own query block to
+    the key/value block it holds, and the per-block results are merged).
+
+    q [B, Sq, Hq, d] holds the queries at positions q_pos0 .. q_pos0+Sq-1,
+    k, v [B, Sk, Hkv, d] the keys at positions k_pos0 .. k_pos0+Sk-1 of the
+    same position axis; with ``causal`` key j is visible to query i iff
+    k_pos0 + j <= q_pos0 + i.  Returns the block's partial (out [B, Sq, Hq,
+    d], lse [B, Hq, Sq]) over the visible keys of this block only; a row
+    that sees none of them gets the empty partial (0, -inf)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Sq, Hq, d = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    rep = Hq // Hkv
+    sc = _scale(d, scale)
+    visible = _position_mask(q_pos0 + np.arange(Sq), k_pos0 + np.arange(Sk))
+    out = np.zeros((B, Sq, Hq, d))
+    lse = np.zeros((B, Hq, Sq))
+    for b in range(B):
+        for h in range(Hq):
+            g = h // rep
+            s = (q[b, :, h] @ k[b, :, g].T) * sc
+            if causal:
+                s = np.where(visible, s, -np.inf)
+            p, l = _softmax_rows(s)
+            out[b, :, h] = p @ v[b, :, g]
+            lse[b, h] = l
+    return out, lse

@@ -145,9 +145,56 @@ def test_gradient_global_identities(causal):
     # sum_j dV_j = sum_i dO_i (rows of P sum to one), summed over the query heads
     want = do.sum(axis=1).reshape(2, Hkv, rep, d).sum(axis=2)
     np.testing.assert_allclose(dv.sum(axis=1), want, atol=1e-12)
-    # D_i = sum_j P_ij dP_ij equals dO_i . O_i: checked via dq of a perturbation-free identity
+
+
+def _d_identity_holds(monkeypatch, causal):
+    """Record the rows D_i = sum_j P_ij dP_ij that the oracle's backward uses
+    and compare them with dO_i . O_i, O_i from the oracle's forward (the two
+    are equal because O_i = sum_j P_ij v_j and dP_ij = dO_i . v_j).  Returns
+    False if any row differs."""
+    B, S, d, Hq, Hkv = 2, 13, 8, 4, 2
+    rng = np.random.default_rng(77)
+    q, k, v, do = (rand(B, S, Hq, d, rng=rng), rand(B, S, Hkv, d, rng=rng),
+                   rand(B, S, Hkv, d, rng=rng), rand(B, S, Hq, d, rng=rng))
+    seen = []
+    inner = A._row_dot_terms
+
+    def record(p, dP):
+        D = inner(p, dP)
+        seen.append(np.array(D))
+        return D
+
+    monkeypatch.setattr(A, "_row_dot_terms", record)
+    oracle.attention_backward(q, k, v, do, causal, row_block=S)  # one row block per head
+    monkeypatch.setattr(A, "_row_dot_terms", inner)
     out, _ = oracle.attention_forward(q, k, v, causal)
-    assert np.isfinite(out).all()
+    rep = Hq // Hkv
+    # the backward visits batch entries, then key/value heads, then their query heads
+    order = [(b, g * rep + r) for b in range(B) for g in range(Hkv) for r in range(rep)]
+    assert len(seen) == len(order)
+    return all(np.allclose(D, np.sum(do[b, :, h] * out[b, :, h], axis=1), rtol=0, atol=1e-12)
+               for D, (b, h) in zip(seen, order))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_d_rows_equal_dout_dot_out(monkeypatch, causal):
+    """D_i = sum_j P_ij dP_ij (as the backward computes it) equals dO_i . O_i."""
+    assert _d_identity_holds(monkeypatch, causal)
+
+
+def test_d_identity_catches_rows_taken_from_the_wrong_row(monkeypatch):
+    """A planted mistake in the oracle -- D of row i taken from row i - 1 --
+    breaks the identity, and the backward's gradients too."""
+    S, d = 9, 4
+    q, k, v, do = rand(1, S, 1, d), rand(1, S, 1, d), rand(1, S, 1, d), rand(1, S, 1, d)
+    good = oracle.attention_backward(q, k, v, do, True)
+    orig = A._row_dot_terms
+    monkeypatch.setattr(A, "_row_dot_terms", lambda p, dP: np.roll(orig(p, dP), 1))
+    assert not _d_identity_holds(monkeypatch, True)
+    monkeypatch.setattr(A, "_row_dot_terms", lambda p, dP: np.roll(orig(p, dP), 1))
+    bad = oracle.attention_backward(q, k, v, do, True)
+    assert np.abs(bad[0] - good[0]).max() > 1e-3  # dQ moves; dV does not depend on D
+    np.testing.assert_allclose(bad[2], good[2], atol=1e-14)
 
 
 def test_backward_kv_head_subset_matches_full():
@@ -472,3 +519,72 @@ def test_relative_output_gate_catches_a_zero_output():
     zero = np.zeros_like(ref)
     assert np.max(np.abs(zero - ref)) <= 2e-2                        # the loose gate passes
     assert np.linalg.norm(zero - ref) / np.linalg.norm(ref) > 1e-2   # the strict gate fails it
+
+
+# ---------------------------------------------------------------- blocks
+
+@pytest.mark.parametrize("q_pos0,k_pos0,Sq,Sk", [(0, 0, 6, 6), (5, 2, 4, 7), (2, 9, 5, 3),
+                                                 (3, 3, 4, 2), (0, 6, 3, 4)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_block_matches_brute_with_positions(q_pos0, k_pos0, Sq, Sk, causal):
+    """A query block at q_pos0 against a key block at k_pos0, against the
+    pure-Python loops with the mask stated over absolute positions (rows
+    that see no key of the block give (0, -inf))."""
+    rng = np.random.default_rng(q_pos0 * 31 + k_pos0)
+    d = 4
+    q, k, v = rand(1, Sq, 2, d, rng=rng), rand(1, Sk, 1, d, rng=rng), rand(1, Sk, 1, d, rng=rng)
+    out, lse = oracle.block_attention(q, k, v, q_pos0, k_pos0, causal)
+    vis = (lambda i, j: k_pos0 + j <= q_pos0 + i) if causal else (lambda i, j: True)
+    for h in range(2):
+        bo, bl = brute.attend(as_lists(q[0, :, h]), as_lists(k[0, :, 0]), as_lists(v[0, :, 0]),
+                              vis, 1 / math.sqrt(d))
+        np.testing.assert_allclose(out[0, :, h], bo, atol=1e-12)
+        np.testing.assert_array_equal(np.isinf(lse[0, h]), np.isinf(bl))
+        fin = np.isfinite(bl)
+        np.testing.assert_allclose(lse[0, h][fin], np.asarray(bl)[fin], atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_block_at_equal_positions_is_full_attention(causal):
+    q, k, v = rand(2, 11, 4, 3), rand(2, 11, 2, 3), rand(2, 11, 2, 3)
+    bo, bl = oracle.block_attention(q, k, v, 7, 7, causal)
+    fo, fl = oracle.attention_forward(q, k, v, causal)
+    np.testing.assert_allclose(bo, fo, atol=1e-13)
+    np.testing.assert_allclose(bl, fl, atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("cuts", [(0, 5, 12, 20), (0, 1, 2, 20), (0, 13, 20)])
+def test_merged_blocks_are_the_whole_row(causal, cuts):
+    """Splitting the keys of a sequence into blocks, attending a query block
+    to each at its own position and merging the partials in any order gives
+    the rows of full attention (Ring Attention, Summary)."""
+    S, d = 20, 5
+    rng = np.random.default_rng(len(cuts))
+    q, k, v = rand(1, S, 2, d, rng=rng), rand(1, S, 2, d, rng=rng), rand(1, S, 2, d, rng=rng)
+    fo, fl = oracle.attention_forward(q, k, v, causal)
+    r0, r1 = 4, 17  # the query block
+    parts = [oracle.block_attention(q[:, r0:r1], k[:, a:b], v[:, a:b], r0, a, causal)
+             for a, b in zip(cuts[:-1], cuts[1:])]
+    for order in (range(len(parts)), reversed(range(len(parts)))):
+        o = np.zeros((1, r1 - r0, 2, d))
+        l = np.full((1, 2, r1 - r0), -np.inf)
+        for i in order:
+            po, pl = parts[i]
+            o_t, l_t = lse_merge(o.transpose(0, 2, 1, 3), l, po.transpose(0, 2, 1, 3), pl)
+            o, l = o_t.transpose(0, 2, 1, 3), l_t
+        np.testing.assert_allclose(o, fo[:, r0:r1], atol=1e-12)
+        np.testing.assert_allclose(l, fl[:, :, r0:r1], atol=1e-12)
+
+
+def test_block_pins_catch_a_mask_off_by_one(monkeypatch):
+    """Planted in the oracle: the block mask uses < instead of <= (the
+    diagonal key dropped); the brute-force pin catches it."""
+    q, k, v = rand(1, 6, 1, 3), rand(1, 6, 1, 3), rand(1, 6, 1, 3)
+    bo, _ = brute.attend(as_lists(q[0, :, 0]), as_lists(k[0, :, 0]), as_lists(v[0, :, 0]),
+                         brute.full_visible(True), 1 / math.sqrt(3))
+    good = oracle.block_attention(q, k, v, 0, 0, True)
+    monkeypatch.setattr(A, "_position_mask", lambda qp, kp: kp[None, :] < qp[:, None])
+    bad = oracle.block_attention(q, k, v, 0, 0, True)
+    assert np.abs(good[0][0, :, 0] - np.asarray(bo)).max() < 1e-12
+    assert np.abs(bad[0][0, :, 0] - np.asarray(bo)).max() > 1e-3
