@@ -33,8 +33,11 @@
  * Ownership and memory
  *   The caller allocates every device buffer (inputs, outputs, workspace)
  *   and keeps it alive until the stream work completes.  Pointers are device
- *   pointers aligned to 16 bytes.  The library allocates no device memory;
- *   it keeps no state between calls except one device error word per device.
+ *   pointers aligned to 16 bytes.  The library allocates no device memory.
+ *   Its device image holds two pieces of state that outlive a call: one
+ *   error word per device (read and cleared by lca_check), and the fixed
+ *   scratch array of lca_attn_bwd_noalloc (LCA_NOALLOC_SCRATCH_BYTES per
+ *   device, loaded with the library and kept until the process exits).
  *
  * Errors
  *   Argument errors are returned synchronously, before anything is launched.
@@ -273,6 +276,107 @@ LCA_API lca_status lca_attn_bwd_varlen(const lca_shape* shape, const int32_t* cu
                                        void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Blocks: one step of a sequence-parallel ring.  Each host keeps its block of
+ * query rows, the key/value blocks travel from host to host, and every host
+ * attends its queries to each key/value block as it arrives, overlapping the
+ * transfer of the next block with the computation (Ring Attention with
+ * Blockwise Transformers for Near-Infinite Context, Summary and Key points);
+ * the per-block partial results combine into the exact answer whatever the
+ * order of arrival.  These calls are the per-host steps; the transfer
+ * between hosts is the caller's (the package's ring driver uses NCCL).
+ *
+ * Shape: B batch entries; a query block of Sq rows (q, dout, out, dq
+ * [B, Sq, Hq, d]; lse [B, Hq, Sq]) and a key/value block of Sk rows (k, v
+ * [B, Sk, Hkv, d]; dk_acc, dv_acc [B, Sk, Hkv, d] float32).  Query row i
+ * sits at position q_pos0 + i and key j at k_pos0 + j of one position
+ * axis; with `causal`, key j is visible to query i iff
+ * k_pos0 + j <= q_pos0 + i.  bf16 only (LCA_ERR_UNSUPPORTED otherwise).
+ * When the diagonal crosses the blocks (some but not all keys visible to
+ * some query), q_pos0 - k_pos0 must be a multiple of 128 (the tile);
+ * blocks wholly before or wholly after each other have no such rule.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  int64_t B, Hq, Hkv;
+  int64_t Sq;     /* query rows of the block */
+  int64_t Sk;     /* key/value rows of the block */
+  int64_t d;      /* 128 */
+  int32_t dtype;  /* LCA_BF16 */
+  float scale;    /* softmax scale; 0 selects 1/sqrt(d) */
+} lca_block_shape;
+
+/* lca_attn_fwd_block -- attend the query block to one key/value block and
+ * fold the result into a running one:
+ *   partial (O_b, lse_b) over the visible keys of this block (a row that
+ *   sees none has the empty partial (0, -inf));
+ *   accumulate != 0: (o_acc, lse_acc) <- merge((o_acc, lse_acc), (O_b, lse_b))
+ *     with lse = M + ln(e^(lse_acc - M) + e^(lse_b - M)), M the larger,
+ *     o = e^(lse_acc - lse) o_acc + e^(lse_b - lse) O_b;
+ *   accumulate == 0: (o_acc, lse_acc) <- (O_b, lse_b) (the first block).
+ * o_acc: [B, Sq, Hq, d] float32, the running output, normalised (NULL is
+ * allowed only with accumulate == 0 and out given); lse_acc: [B, Hq, Sq]
+ * float32, natural log, in/out.  out (nullable): the merged output rounded
+ * to bf16 (after the last block it is the attention output).  Both are
+ * caller-owned device buffers; lse_acc/o_acc are read only when
+ * accumulating.  A causal block that no query sees adds nothing and
+ * launches nothing when accumulating.
+ * Errors: as lca_attn_fwd, plus LCA_ERR_INVALID_ARG for negative
+ * positions, misaligned diagonal offsets (above), o_acc and out both NULL,
+ * or accumulate without o_acc. */
+LCA_API lca_status lca_attn_fwd_block(const lca_block_shape* shape, const void* q,
+                                      const void* k, const void* v, int causal, int64_t q_pos0,
+                                      int64_t k_pos0, int accumulate, float* o_acc,
+                                      float* lse_acc, void* out, void* stream);
+
+/* Workspace of the block backward for one query block: D rows and a
+ * padded lse copy ([B, Hq, Sq rounded up to 128] float32 each) and a
+ * float32 dq accumulator [B, Sq, Hq, d].  0 for an invalid shape. */
+LCA_API size_t lca_attn_bwd_block_workspace_size(const lca_block_shape* shape);
+
+/* lca_attn_bwd_block_prep -- start the backward of a query block: zero the
+ * workspace's dq accumulator and compute D_i = dout_i . out_i from the
+ * block's FINAL out and lse (over every key of the sequence).  Only Sq of
+ * the shape is read (Sk may be anything valid). */
+LCA_API lca_status lca_attn_bwd_block_prep(const lca_block_shape* shape, const void* out,
+                                           const float* lse, const void* dout, void* workspace,
+                                           size_t ws_bytes, void* stream);
+
+/* lca_attn_bwd_block -- add one key/value block's share of the gradients
+ * of sum(dout * out): P_ij = exp(scale s_ij - lse_i) recomputed with the
+ * final lse, dV_j += sum_i P_ij dO_i, dK_j += scale sum_i dS_ij q_i into
+ * the block's accumulators, and dQ_i += scale sum_j dS_ij k_j into the
+ * workspace (prepared by lca_attn_bwd_block_prep; blocks may come in any
+ * order).  Either dk_acc and dv_acc ([B, Sk, Hkv, d] float32: this block's
+ * share is ADDED to them when accumulate_kv != 0, else written over them;
+ * the ring's accumulators travel with the key/value block) or dk and dv
+ * (bf16, overwritten with this block's share alone) are given, the other
+ * pair NULL.
+ * Errors: as lca_attn_bwd, plus the block rules above, and
+ * LCA_ERR_INVALID_ARG unless exactly one pair is given. */
+LCA_API lca_status lca_attn_bwd_block(const lca_block_shape* shape, const void* q,
+                                      const void* k, const void* v, const void* dout,
+                                      int causal, int64_t q_pos0, int64_t k_pos0,
+                                      void* workspace, size_t ws_bytes, float* dk_acc,
+                                      float* dv_acc, int accumulate_kv, void* dk, void* dv,
+                                      void* stream);
+
+/* lca_attn_bwd_block_dq -- finish the query block: dq (bf16, [B, Sq, Hq,
+ * d]) from the workspace's accumulator. */
+LCA_API lca_status lca_attn_bwd_block_dq(const lca_block_shape* shape, const void* workspace,
+                                         size_t ws_bytes, void* dq, void* stream);
+
+/* lca_cast_f32_bf16 -- dst[i] = bf16(src[i]) (round to nearest even) for n
+ * elements: turns a running float32 block result (o_acc, dk_acc, dv_acc)
+ * into the bf16 output.  Device pointers, 16-byte aligned.  Errors:
+ * LCA_ERR_INVALID_ARG for n <= 0 or NULL/misaligned pointers. */
+LCA_API lca_status lca_cast_f32_bf16(int64_t n, const float* src, void* dst, void* stream);
+
+/* lca_accumulate_f32 -- dst[i] += src[i] for n float32 elements: folds a
+ * ring step's partial key/value gradients into the accumulators that
+ * arrived with the block.  Device pointers, 16-byte aligned, not
+ * overlapping.  Errors: as lca_cast_f32_bf16. */
+LCA_API lca_status lca_accumulate_f32(int64_t n, const float* src, float* dst, void* stream);
+
+/* ---------------------------------------------------------------------------
  * lca_lse_merge -- combine two partial attention results over disjoint key
  * sets (Ring Attention, Summary: per-block results combine independently of
  * order):  lse = M + ln(e^(lse_a-M) + e^(lse_b-M)), M = max(lse_a, lse_b);
@@ -337,10 +441,68 @@ LCA_API lca_status lca_ffn_bwd(const lca_ffn_shape* shape, const void* x, const 
                                int64_t block_tokens, void* dx, float* dw_gate, float* dw_up,
                                float* dw_down, void* workspace, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Blockwise Transformer sweep: a host "computes attention and feedforward
+ * for its query block block by block" (Ring Attention with Blockwise
+ * Transformers for Near-Infinite Context, Summary), and the blockwise
+ * feedforward keeps the feedforward's intermediate to one block (Key
+ * points).  For each block of q_block query rows in turn: the exact
+ * attention of those rows over the keys they see (all keys before the
+ * block's last row when causal), then the gated-SiLU feedforward
+ * (lca_ffn_fwd's unit) of the block's attention output rows, x =
+ * attn_out viewed [S, h] with h = Hq * d.  One sequence (B = 1);
+ * bf16, d = 128.
+ *   q, attn_out: [S, Hq, d]; k, v: [S, Hkv, d]; lse: [Hq, S] float32;
+ *   w_gate, w_up: [f, h]; w_down: [h, f]; out: [S, h] bf16.
+ * The attention output of the sweep is the input of its feedforward (no
+ * output projection, residual or normalisation in between: those are not
+ * part of this library).  Errors: LCA_ERR_INVALID_ARG for dimensions <= 0,
+ * q_block not a multiple of 128, NULL or misaligned pointers;
+ * LCA_ERR_UNSUPPORTED unless d == 128, h % 256 == 0 and f % 128 == 0 (f %
+ * 256 == 0 for the backward); LCA_ERR_WORKSPACE for a missing or small
+ * workspace.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  int64_t S;        /* tokens of the sequence */
+  int64_t Hq, Hkv;  /* attention heads; the feedforward width is h = Hq * d */
+  int64_t d;        /* head dimension, 128 */
+  int64_t f;        /* feedforward width */
+  int64_t q_block;  /* query rows per block, a multiple of 128; 0 selects
+                       LCA_FFN_BLOCK_DEFAULT */
+  float scale;      /* softmax scale; 0 selects 1/sqrt(d) */
+} lca_bpt_shape;
+
+/* Workspace of lca_bpt_fwd: the lse and the feedforward intermediate of one
+ * block.  0 for an invalid shape. */
+LCA_API size_t lca_bpt_fwd_workspace_size(const lca_bpt_shape* shape);
+LCA_API lca_status lca_bpt_fwd(const lca_bpt_shape* shape, const void* q, const void* k,
+                               const void* v, int causal, const void* w_gate, const void* w_up,
+                               const void* w_down, void* attn_out, float* lse, void* out,
+                               void* workspace, size_t ws_bytes, void* stream);
+
+/* lca_bpt_bwd -- gradients of sum(dout * out) of lca_bpt_fwd, block by
+ * block: the feedforward backward of the block's rows (weight gradients
+ * ADDED to the float32 dw_gate, dw_up, dw_down, as lca_ffn_bwd), whose input
+ * gradient is the dout of the block's attention rows; their attention
+ * backward recomputes P from lse (dq of the block's rows; dk, dv over every
+ * block are summed in float32 inside the workspace and written as bf16 at
+ * the end).  attn_out and lse are lca_bpt_fwd's.  dq: [S, Hq, d]; dk, dv:
+ * [S, Hkv, d], bf16, overwritten. */
+LCA_API size_t lca_bpt_bwd_workspace_size(const lca_bpt_shape* shape);
+LCA_API lca_status lca_bpt_bwd(const lca_bpt_shape* shape, const void* q, const void* k,
+                               const void* v, int causal, const void* w_gate, const void* w_up,
+                               const void* w_down, const void* attn_out, const float* lse,
+                               const void* dout, void* dq, void* dk, void* dv, float* dw_gate,
+                               float* dw_up, float* dw_down, void* workspace, size_t ws_bytes,
+                               void* stream);
+
 /* Synchronises `stream`, then reports and clears the device error word of
  * the current device: LCA_ERR_TIMEOUT if a kernel wait ran out since the
- * last check, LCA_ERR_INVALID_ARG if a kernel met invalid packed sequence
- * offsets, LCA_ERR_CUDA if the stream holds a CUDA error, else LCA_OK. */
+ * last check, or if a CTA gave up waiting (about one second) for its own
+ * copies or MMAs in flight before it freed its tensor memory (the detail
+ * text of lca_last_error says which); LCA_ERR_INVALID_ARG if a kernel met
+ * invalid packed sequence offsets, LCA_ERR_CUDA if the stream holds a CUDA
+ * error, else LCA_OK. */
 LCA_API lca_status lca_check(void* stream);
 
 /* Static description of a status code. */

@@ -8,6 +8,13 @@ library's backward entry point.  Every step runs in the CUDA library.
     from long_context_exact_attention_b200.autograd import attention, s2_attention, feedforward
     out = attention(q, k, v, causal=True, kv_chunk=4096, order="ring")
     out.float().sum().backward()
+
+Errors inside a kernel (a wait that ran out, invalid packed offsets) are
+recorded in the library's device error word, not raised by these calls,
+because reading it synchronises the stream.  Call ``lca.check()`` at a point
+where a synchronisation is acceptable (for example once per training step);
+it raises if any kernel since the last check reported an error, and the
+results of that step must then be discarded.
 """
 
 from __future__ import annotations

@@ -4,6 +4,8 @@
 //                dS = P o (dP - D) in the backward pass, plus a copy of lse,
 //                both into per-sequence rows padded to whole tiles
 //   dq_finalize  dq = scale * dq_acc, float32 accumulator -> bf16
+//   cast_f32_bf16  float32 -> bf16 (a blockwise result's last step)
+//   accumulate_f32 dst += src (ring steps' partial key/value gradients)
 //   lse_merge    combine two partial (O, lse) results over disjoint key
 //                sets (Ring Attention with Blockwise Transformers, Summary:
 //                per-block results combine independently of order)
@@ -160,6 +162,46 @@ __global__ void dq_finalize(const float* __restrict__ acc, __nv_bfloat16* __rest
     r[3] = __floats2bfloat162_rn(b.z * scale, b.w * scale);
     reinterpret_cast<uint4*>(dq)[i] = *reinterpret_cast<uint4*>(r);
   }
+}
+
+// dst(bf16) = src(float32), n elements, rounded to nearest even: 8 per
+// thread (both pointers 16-byte aligned), then the n % 8 tail elements.
+__global__ void cast_f32_bf16(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst,
+                              int64_t n) {
+  const int64_t n8 = n / 8;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (int64_t i = tid; i < n8; i += stride) {
+    const float4 a = reinterpret_cast<const float4*>(src)[2 * i];
+    const float4 b = reinterpret_cast<const float4*>(src)[2 * i + 1];
+    __nv_bfloat162 r[4];
+    r[0] = __floats2bfloat162_rn(a.x, a.y);
+    r[1] = __floats2bfloat162_rn(a.z, a.w);
+    r[2] = __floats2bfloat162_rn(b.x, b.y);
+    r[3] = __floats2bfloat162_rn(b.z, b.w);
+    reinterpret_cast<uint4*>(dst)[i] = *reinterpret_cast<uint4*>(r);
+  }
+  if (tid < n - n8 * 8) dst[n8 * 8 + tid] = __float2bfloat16_rn(src[n8 * 8 + tid]);
+}
+
+// dst += src, n float32 elements: 4 per thread (both pointers 16-byte
+// aligned), then the n % 4 tail (a ring step's partial key/value gradients
+// folded into the accumulators that travel with the block).
+__global__ void accumulate_f32(const float* __restrict__ src, float* __restrict__ dst,
+                               int64_t n) {
+  const int64_t n4 = n / 4;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (int64_t i = tid; i < n4; i += stride) {
+    const float4 a = reinterpret_cast<const float4*>(src)[i];
+    float4 b = reinterpret_cast<float4*>(dst)[i];
+    b.x += a.x;
+    b.y += a.y;
+    b.z += a.z;
+    b.w += a.w;
+    reinterpret_cast<float4*>(dst)[i] = b;
+  }
+  if (tid < n - n4 * 4) dst[n4 * 4 + tid] += src[n4 * 4 + tid];
 }
 
 // (O, lse) merge, one warp per row.  Every lane reads the row's two lse

@@ -20,6 +20,14 @@
 // One CTA per (key tile of 128, key/value head, batch); it loops over the
 // query heads of its grouped-query group and over the query tiles that can
 // see the key tile, so dK/dV of a key tile finish inside one CTA.
+//
+// Block calls: the key tiles belong to a key/value block that may start
+// elsewhere on the position axis than the query block (a sequence-parallel
+// ring; Ring Attention with Blockwise Transformers, Summary), with its own
+// length and a shifted causal diagonal (AttnSched::diag).  With kAccKV the
+// CTA writes its dK/dV in float32, added to what the buffers hold when
+// acc_add is set (the ring carries such accumulators with the key/value
+// block from host to host), instead of storing bf16.
 // Roles (16 warps, four warpgroups):
 //   warpgroup 0  warp 0: TMA producer (K, V once; Q + lse/D rows through a
 //                2-stage ring, dO single-staged); warp 1: TMEM owner, lane 0
@@ -103,8 +111,11 @@ struct Args {
   unsigned long long budget;
   const float* lse;      // [B,Hq,S_pad], +inf past each sequence's end
   const float* Drow;     // [B,Hq,S_pad], zero past each sequence's end
-  __nv_bfloat16* dk;
+  __nv_bfloat16* dk;     // bf16 outputs (kAccKV false)
   __nv_bfloat16* dv;
+  float* dk_acc;         // float32 accumulators, [B, S_kv, Hkv, 128] (kAccKV true)
+  float* dv_acc;
+  int acc_add;           // kAccKV: add to dk_acc/dv_acc (else overwrite them)
   AttnSched sched;
 };
 
@@ -119,6 +130,7 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
+template <bool kAccKV>
 __global__ void __launch_bounds__(bwd::kThreads, 1)
     attn_bwd_bf16_sm100(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
@@ -154,8 +166,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
   // Head-major order (the CTAs in flight update one or two heads' dq rows,
   // which stay in L2), longest causal work first within a head: key tile 0
   // sees every query tile.
-  const int kt = static_cast<int>(blockIdx.x) % sc.n_tiles;
-  const int bg = static_cast<int>(blockIdx.x) / sc.n_tiles;
+  const int kt = static_cast<int>(blockIdx.x) % sc.n_kv_tiles;
+  const int bg = static_cast<int>(blockIdx.x) / sc.n_kv_tiles;
   const int g = bg % a.Hkv;
   const int b = bg / a.Hkv;
   SeqView sv;
@@ -163,7 +175,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     if (threadIdx.x == 0 && kt == 0) record_error(kErrSeqOffsets, 151);
     return;
   }
-  if (kt >= sv.n_tiles) return;  // a shorter packed sequence: no work here
+  if (kt >= sv.kv_n_tiles) return;  // a shorter packed sequence: no work here
   const bool shifted = head_shifted(sc, g * rep);
   const int ktok0 = token_tile(sc, kt, shifted) * kTile;
   QWalk qw;
@@ -200,7 +212,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmDO);
       mbar_expect_tx(bar(B_KV), 2 * kTileB);
-      const int ktok = sv.row0 + ktok0;
+      const int ktok = sv.kv_row0 + ktok0;
       tma_load_3d(sK, &tmK, bar(B_KV), 0, g, ktok);
       tma_load_3d(sK + kHalf, &tmK, bar(B_KV), 64, g, ktok);
       tma_load_3d(sV, &tmV, bar(B_KV), 0, g, ktok);
@@ -230,10 +242,10 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         ++o_issued;
       }
       if (!ok) {
-        drain_bar(bar(B_KV), 0, a.budget);
-        if (issued0) drain_bar(bar(B_QFULL), (issued0 - 1) & 1, a.budget);
-        if (issued1) drain_bar(bar(B_QFULL + 1), (issued1 - 1) & 1, a.budget);
-        if (o_issued) drain_bar(bar(B_OFULL), (o_issued - 1) & 1, a.budget);
+        drain_bar(bar(B_KV), 0, 171);
+        if (issued0) drain_bar(bar(B_QFULL), (issued0 - 1) & 1, 172);
+        if (issued1) drain_bar(bar(B_QFULL + 1), (issued1 - 1) & 1, 173);
+        if (o_issued) drain_bar(bar(B_OFULL), (o_issued - 1) & 1, 174);
       }
     } else if (warp == 1 && lane == 0) {
       // =================================================== MMA issuer
@@ -311,7 +323,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       }
       tc_commit(bar(B_DONE));
       tc_commit(bar(B_DRAIN));
-      drain_bar(bar(B_DRAIN), 0, a.budget);
+      drain_bar(bar(B_DRAIN), 0, 175);
     }
   } else if (wg <= 2) {
     regs_inc<kRegsWork>();
@@ -323,7 +335,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     const float c = a.scale_log2;
     const float L2E = 1.4426950408889634f;
     const uint64_t c2 = f2_pack(c, c);
-    const bool key_out = ktok0 + r >= sv.len;  // key row past the sequence's end
+    const bool key_out = ktok0 + r >= sv.kv_len;  // key row past the sequence's end
     // added to every exponent of this key row: -inf gives P = 0 (hence dS =
     // 0, and the row adds nothing to dQ) for a key row past the end
     const float kill = key_out ? -INFINITY : 0.f;
@@ -338,7 +350,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const bool diag = sc.causal && qt == kt;
+      const bool diag = sc.causal && qt + sc.diag == kt;
       // ---- P^T = exp2(S^T c - lse log2e) for queries [64hq, 64hq+64),
       // written back as bf16 over columns [64hq, 64hq+32) of S^T
       float p[64];
@@ -402,14 +414,29 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     // past the sequence's end (ragged last tile) only skip their stores
     if (ok) {
       tc_fence_after();
-      const size_t trow = static_cast<size_t>(sv.row0) + (key_out ? 0 : ktok0 + r);
+      const size_t trow = static_cast<size_t>(sv.kv_row0) + (key_out ? 0 : ktok0 + r);
       __nv_bfloat16* row = a.dk + (trow * a.Hkv + g) * kD;
+      float* arow = a.dk_acc + (trow * a.Hkv + g) * kD;
 #pragma unroll 1
       for (int cc = 2 * hq; cc < 2 * hq + 2; ++cc) {
         float o[32];
         __syncwarp();
-        tmem_ld32(tmem + lad + 384 + cc * 32, o);
-        if (!key_out) {
+        if (nsteps > 0) {
+          tmem_ld32(tmem + lad + 384 + cc * 32, o);
+        } else {  // a block call's key tile that no query sees: no gradient
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0.f;
+        }
+        if (kAccKV && !key_out) {
+          float4* dst = reinterpret_cast<float4*>(arow + cc * 32);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const float4 x = a.acc_add ? dst[v] : make_float4(0.f, 0.f, 0.f, 0.f);
+            dst[v] = make_float4(fmaf(o[4 * v], a.scale, x.x), fmaf(o[4 * v + 1], a.scale, x.y),
+                                 fmaf(o[4 * v + 2], a.scale, x.z),
+                                 fmaf(o[4 * v + 3], a.scale, x.w));
+          }
+        } else if (!key_out) {
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
             uint4 pk;
@@ -468,17 +495,31 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     // ---- dV -> bf16
     if (ok) ok = wait_bar(bar(B_DONE), 0, wc, 412);
     ok = __all_sync(0xffffffffu, ok);
-    const bool row_in = ktok0 + r < sv.len;
+    const bool row_in = ktok0 + r < sv.kv_len;
     if (ok) {
       tc_fence_after();
-      const size_t trow = static_cast<size_t>(sv.row0) + (row_in ? ktok0 + r : 0);
+      const size_t trow = static_cast<size_t>(sv.kv_row0) + (row_in ? ktok0 + r : 0);
       __nv_bfloat16* row = a.dv + (trow * a.Hkv + g) * kD;
+      float* arow = a.dv_acc + (trow * a.Hkv + g) * kD;
 #pragma unroll 1
       for (int cc = 0; cc < 4; ++cc) {
         float o[32];
         __syncwarp();
-        tmem_ld32(tmem + lad + 256 + cc * 32, o);
-        if (row_in) {
+        if (nsteps > 0) {
+          tmem_ld32(tmem + lad + 256 + cc * 32, o);
+        } else {  // a block call's key tile that no query sees: no gradient
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0.f;
+        }
+        if (kAccKV && row_in) {
+          float4* dst = reinterpret_cast<float4*>(arow + cc * 32);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const float4 x = a.acc_add ? dst[v] : make_float4(0.f, 0.f, 0.f, 0.f);
+            dst[v] = make_float4(o[4 * v] + x.x, o[4 * v + 1] + x.y, o[4 * v + 2] + x.z,
+                                 o[4 * v + 3] + x.w);
+          }
+        } else if (row_in) {
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
             uint4 pk;

@@ -24,8 +24,11 @@
 //     2-5: epilogue, one output row per thread (its TMEM lane);
 //   * two 256-column fp32 accumulators in TMEM (all 512 columns), so the
 //     epilogue of one tile runs while the next tile's products accumulate;
-//   * tiles are visited in bands of 16 row tiles, column by column, so the
-//     tiles in flight share their A rows and B columns in L2.
+//   * tiles are visited in bands of group_m row tiles, column by column, so
+//     the tiles in flight share their A rows and B columns in L2 (the host
+//     picks the band per product: a whole block of rows when the weights are
+//     the large operand, so each weight column is read once per block; one
+//     row tile when B is small enough to stay in L2 whole).
 // Epilogues: EPI_STORE -- 256 columns as bf16; EPI_SWIGLU -- the B stage
 // holds 128 rows of W_gate then 128 rows of W_up for the same columns and
 // the epilogue writes silu(gate) * up (128 columns); EPI_SWIGLU_BWD -- the
@@ -48,7 +51,7 @@ constexpr int kBM = 128;
 constexpr int kBN = 256;
 constexpr int kBK = 64;
 constexpr int kStages = 4;
-constexpr int kGroupM = 16;
+constexpr int kGroupM = 16;  // default band height (row tiles)
 constexpr int kThreads = 192;
 constexpr uint32_t kAStage = kBM * kBK * 2;  // 16 KB
 constexpr uint32_t kBHalf = 128 * kBK * 2;   // 16 KB
@@ -78,7 +81,9 @@ struct Args {
   int ldo;           // row stride of the outputs, in elements
   int ldo3;          // row stride of out3
   int ld_in;         // row stride of `in`
-  int m_split;       // EPI_ACC32: rows from m_split on go to out32b (M when unused)
+  int m_split;       // EPI_ACC32: rows from m_split on go to out32b (ignored when
+                     // out32b is null)
+  int group_m;       // band height of the tile raster in row tiles (>= 1)
   unsigned long long budget;
   __nv_bfloat16* out;   // C (EPI_STORE, EPI_SWIGLU), dG (EPI_SWIGLU_BWD)
   __nv_bfloat16* out2;  // dU (EPI_SWIGLU_BWD)
@@ -88,12 +93,13 @@ struct Args {
   float* out32b;        // EPI_ACC32: rows from m_split on, counted from m_split
 };
 
-// Tile t -> (tm, tn): bands of kGroupM row tiles, column by column.
-__host__ __device__ inline void tile_coords(int t, int n_tm, int n_tn, int& tm, int& tn) {
-  const int band = t / (kGroupM * n_tn);
-  const int first = band * kGroupM;
-  const int gm = n_tm - first < kGroupM ? n_tm - first : kGroupM;
-  const int t_in = t - band * kGroupM * n_tn;
+// Tile t -> (tm, tn): bands of group_m row tiles, column by column.
+__host__ __device__ inline void tile_coords(int t, int n_tm, int n_tn, int group_m, int& tm,
+                                            int& tn) {
+  const int band = t / (group_m * n_tn);
+  const int first = band * group_m;
+  const int gm = n_tm - first < group_m ? n_tm - first : group_m;
+  const int t_in = t - band * group_m * n_tn;
   tm = first + t_in % gm;
   tn = t_in / gm;
 }
@@ -204,9 +210,12 @@ __device__ __forceinline__ void ffn_epilogue(const ffn::Args& a, uint32_t acc, i
       }
     }
   } else {  // EPI_ACC32
-    // two stacked outputs: a 128-row tile lies wholly on one side of m_split
-    float* base = row < a.m_split ? a.out32 + orow
-                                  : a.out32b + static_cast<size_t>(row - a.m_split) * a.ldo;
+    // two stacked outputs: a 128-row tile lies wholly on one side of m_split.
+    // Without a second output (out32b null) every row goes to out32, whatever
+    // m_split holds.
+    float* base = (row < a.m_split || a.out32b == nullptr)
+                      ? a.out32 + orow
+                      : a.out32b + static_cast<size_t>(row - a.m_split) * a.ldo;
 #pragma unroll 1
     for (int c = 0; c < kBN / 32; ++c) {
       float v[32];
@@ -285,7 +294,7 @@ __global__ void __launch_bounds__(ffn::kThreads, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
         int tm, tn;
-        tile_coords(t, a.n_tm, a.n_tn, tm, tn);
+        tile_coords(t, a.n_tm, a.n_tn, a.group_m, tm, tn);
         const int m0 = tm * kBM;
         // first B row/column of the tile: 256 output columns, or 128 gate +
         // 128 up rows for the same 128 columns
@@ -323,7 +332,7 @@ __global__ void __launch_bounds__(ffn::kThreads, 1)
       if (!ok) {
         // let the copies already issued land before the CTA exits
         for (int s = 0; s < kStages; ++s)
-          if (issued[s]) drain_bar(bar(B_FULL + s), (issued[s] - 1) & 1, a.budget);
+          if (issued[s]) drain_bar(bar(B_FULL + s), (issued[s] - 1) & 1, 181);
       }
     }
   } else if (warp == 1) {
@@ -360,7 +369,7 @@ __global__ void __launch_bounds__(ffn::kThreads, 1)
       }
       // wait for every product this thread issued before TMEM is freed
       tc_commit(bar(B_DRAIN));
-      drain_bar(bar(B_DRAIN), 0, a.budget);
+      drain_bar(bar(B_DRAIN), 0, 182);
     }
   } else {
     // =================================================== epilogue
@@ -373,7 +382,7 @@ __global__ void __launch_bounds__(ffn::kThreads, 1)
       if (!__all_sync(0xffffffffu, wait_bar(bar(B_ACCFULL + b), (li >> 1) & 1, wc, 621))) break;
       tc_fence_after();
       int tm, tn;
-      tile_coords(t, a.n_tm, a.n_tn, tm, tn);
+      tile_coords(t, a.n_tm, a.n_tn, a.group_m, tm, tn);
       ffn_epilogue<kEpi>(a, tmem + lad + b * kBN, tm * kBM + r, tn);
       // this accumulator may be overwritten by the tile after next
       tc_fence_before();

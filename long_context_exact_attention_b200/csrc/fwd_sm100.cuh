@@ -24,6 +24,19 @@
 // issues S_t for the next key tile right behind the PV that reads P_t from
 // the same columns; the tensor pipe runs one thread's MMAs in order.
 //
+// Block calls (kBlock) attend a query block to a key/value block that
+// starts elsewhere on the position axis, for a sequence-parallel ring (Ring
+// Attention with Blockwise Transformers, Summary: each host keeps its query
+// block, the key/value blocks travel, and the per-block results combine
+// whatever their order).  The epilogue then folds this block's partial
+// (O_b, lse_b) into a running float32 (O, lse) held in global memory with
+// the log-sum-exp merge
+//   lse = L + log(e^(lse_old - L) + e^(lse_b - L)),  L = max of the two,
+//   O   = e^(lse_old - lse) O_old + e^(lse_b - lse) O_b,
+// an empty partial being (0, -inf), and may also write the merged O as
+// bf16.  In log2 units with this block's running (m, l): lse_b = m + log2 l
+// and e^(lse_b - lse) O_b = 2^(m - lse) * (O l), the unnormalised TMEM sum.
+//
 // TMEM columns: S/P tile 0 [0,128) | S/P tile 1 [128,256) | O tile 0
 // [256,384) | O tile 1 [384,512).
 // Shared memory (1024-aligned, 128-byte swizzle): Q0 | Q1 | K x2 | V x2.
@@ -70,19 +83,23 @@ constexpr uint32_t kIdescO = idesc_bf16_f32(128, 128, false, true);    // P V (V
 
 struct Args {
   int B, Hq, Hkv;
-  int S;  // tokens per batch entry of the tensors (packed: all sequences)
+  int S;  // tokens per batch entry of the query tensors (packed: all sequences)
   float scale_log2;
   unsigned long long budget;
-  __nv_bfloat16* out;
-  float* lse;
+  __nv_bfloat16* out;  // block calls: may be null
+  float* lse;          // block calls: the running lse, read when accumulating
+  float* o_acc;        // block calls: running O, [B, S, Hq, 128] float32, or null
+  int accumulate;      // block calls: fold into (o_acc, lse) instead of overwriting
   AttnSched sched;
 };
 
-// Visibility of key/value position tile T to query position tile Q.
+// Visibility of key/value position tile T to query position tile Q, whose
+// diagonal key tile is Q + diag.
 enum { VIS_NONE = 0, VIS_FULL = 1, VIS_DIAG = 2 };
-__device__ __forceinline__ int tile_vis(bool causal, int Q, int T) {
+__device__ __forceinline__ int tile_vis(bool causal, int diag, int Q, int T) {
   if (!causal) return VIS_FULL;
-  return T < Q ? VIS_FULL : (T == Q ? VIS_DIAG : VIS_NONE);
+  const int D = Q + diag;
+  return T < D ? VIS_FULL : (T == D ? VIS_DIAG : VIS_NONE);
 }
 
 // One interface over the two walks: KvWalk (chunk boundaries anywhere; each
@@ -90,11 +107,11 @@ __device__ __forceinline__ int tile_vis(bool causal, int Q, int T) {
 // tiles; lo and hi are left alone).
 __device__ __forceinline__ void walk_init(KvWalk& w, const AttnSched* s, int qt,
                                           const SeqView& v) {
-  w.init(s, qt, v.len);
+  w.init(s, qt, v.kv_len);
 }
 __device__ __forceinline__ void walk_init(TileWalk& w, const AttnSched* s, int qt,
                                           const SeqView& v) {
-  w.init(s, qt, v.n_tiles);
+  w.init(s, qt, v.kv_n_tiles);
 }
 __device__ __forceinline__ bool walk_next(KvWalk& w, int& t, int& lo, int& hi) {
   return w.next(t, lo, hi);
@@ -103,11 +120,82 @@ __device__ __forceinline__ bool walk_next(TileWalk& w, int& t, int&, int&) { ret
 
 }  // namespace fwd
 
+// Epilogue of a block call for one query row (one thread): fold this
+// block's partial (TMEM O, running m and l in log2 units) into the running
+// float32 (o_acc, lse) and/or write the merged row as bf16.  Every lane of
+// the warp calls it (the TMEM loads are warp-collective).
+__device__ __forceinline__ void fwd_block_epilogue(const fwd::Args& a, uint32_t tO, int cnt,
+                                                float m_run, float l_run, bool row_in,
+                                                size_t trow, int h, size_t li) {
+  using namespace fwd;
+  const float L2E = 1.4426950408889634f;
+  // log2-domain lse of this block's partial and of the running result
+  const float lb = (cnt >= 1 && l_run > 0.f) ? m_run + lg2_approx(l_run) : -INFINITY;
+  const float lold = (a.accumulate && row_in) ? a.lse[li] * L2E : -INFINITY;
+  const float mx = fmaxf(lb, lold);
+  float ln = -INFINITY, w_old = 0.f, w_b = 0.f;
+  if (mx != -INFINITY) {
+    ln = mx + lg2_approx(ex2_approx(lold - mx) + ex2_approx(lb - mx));
+    w_old = (lold == -INFINITY) ? 0.f : ex2_approx(lold - ln);
+    w_b = (lb == -INFINITY) ? 0.f : ex2_approx(m_run - ln);
+  }
+  float* arow = a.o_acc ? a.o_acc + (trow * a.Hq + h) * kD : nullptr;
+  __nv_bfloat16* orow = a.out ? a.out + (trow * a.Hq + h) * kD : nullptr;
+#pragma unroll 1
+  for (int q4 = 0; q4 < 4; ++q4) {
+    float o[32];
+    __syncwarp();
+    if (cnt >= 1) {
+      tmem_ld32(tO + q4 * 32, o);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] = 0.f;
+    }
+    if (row_in) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] *= w_b;
+      if (a.accumulate && w_old != 0.f) {
+        const float4* src = reinterpret_cast<const float4*>(arow + q4 * 32);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const float4 x = src[v];
+          o[4 * v + 0] = fmaf(w_old, x.x, o[4 * v + 0]);
+          o[4 * v + 1] = fmaf(w_old, x.y, o[4 * v + 1]);
+          o[4 * v + 2] = fmaf(w_old, x.z, o[4 * v + 2]);
+          o[4 * v + 3] = fmaf(w_old, x.w, o[4 * v + 3]);
+        }
+      }
+      if (arow) {
+        float4* dst = reinterpret_cast<float4*>(arow + q4 * 32);
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          dst[v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+      }
+      if (orow) {
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          uint4 pk;
+          pk.x = pack_bf16x2(o[v * 8 + 0], o[v * 8 + 1]);
+          pk.y = pack_bf16x2(o[v * 8 + 2], o[v * 8 + 3]);
+          pk.z = pack_bf16x2(o[v * 8 + 4], o[v * 8 + 5]);
+          pk.w = pack_bf16x2(o[v * 8 + 6], o[v * 8 + 7]);
+          *reinterpret_cast<uint4*>(orow + q4 * 32 + v * 8) = pk;
+        }
+      }
+    }
+  }
+  if (row_in) a.lse[li] = ln * 0.69314718055994531f;
+}
+
 // kRanged: some chunk boundary falls inside a tile, so visits carry key
 // ranges (KvWalk).  Otherwise the cheaper tile walk runs and only a ragged
-// last tile needs a key mask.
-template <bool kRanged>
-__global__ void __launch_bounds__(fwd::kThreads, 1)
+// last tile needs a key mask.  kBlock: a block call (merging epilogue).
+// Register cap: 200 per thread (10 warps x 200 fit the register file at one
+// CTA per SM, which shared memory fixes anyway).  The ranged and block
+// instantiations need a few registers more than the plain one's 168, which
+// the default cap for 320 threads did not give them (they spilled).
+template <bool kRanged, bool kBlock>
+__global__ void __maxnreg__(200)
     attn_fwd_bf16_sm100(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV,
@@ -123,8 +211,9 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
   auto bar = [&](int i) { return bars + 8u * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kOffBar + 8 * NUM_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + kOffBar + 8 * NUM_BARS + 8);
-  // The sequence's length, first row and lse offset, parked in shared
-  // memory (re-read where needed rather than held through the softmax loop)
+  // The sequence's length, first row, lse offset and key count, parked in
+  // shared memory (re-read where needed rather than held through the
+  // softmax loop): [0] len, [4] row0, [8] lse offset (64-bit), [16] kv_len
   const uint32_t seq_smem = bars + 8 * NUM_BARS + 16;
 
   const int warp = threadIdx.x >> 5;
@@ -163,6 +252,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     si[1] = sv.row0;
     *reinterpret_cast<long long*>(si + 2) =
         (static_cast<long long>(sv.bm) * a.Hq + h) * a.S + sv.tokb;
+    si[4] = sv.kv_len;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -194,7 +284,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       bool ok = true;
       while (ok && walk_next(w, t, lo, hi)) {
         const int st = j & 1;
-        const int tok = sv.row0 + token_tile(sc, t, shifted) * kTile;
+        const int tok = sv.kv_row0 + token_tile(sc, t, shifted) * kTile;
         if (j >= 2) ok = wait_bar(bar(B_KEMPTY + st), ((j - 2) >> 1) & 1, wc, 101);
         if (!ok) break;
         mbar_expect_tx(bar(B_KFULL + st), kTileB);
@@ -211,11 +301,11 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       }
       if (!ok) {
         // Unwind: let the copies already issued land before the CTA exits.
-        drain_bar(bar(B_Q), 0, a.budget);
-        if (k_issued0) drain_bar(bar(B_KFULL), (k_issued0 - 1) & 1, a.budget);
-        if (k_issued1) drain_bar(bar(B_KFULL + 1), (k_issued1 - 1) & 1, a.budget);
-        if (v_issued0) drain_bar(bar(B_VFULL), (v_issued0 - 1) & 1, a.budget);
-        if (v_issued1) drain_bar(bar(B_VFULL + 1), (v_issued1 - 1) & 1, a.budget);
+        drain_bar(bar(B_Q), 0, 161);
+        if (k_issued0) drain_bar(bar(B_KFULL), (k_issued0 - 1) & 1, 162);
+        if (k_issued1) drain_bar(bar(B_KFULL + 1), (k_issued1 - 1) & 1, 163);
+        if (v_issued0) drain_bar(bar(B_VFULL), (v_issued0 - 1) & 1, 164);
+        if (v_issued1) drain_bar(bar(B_VFULL + 1), (v_issued1 - 1) & 1, 165);
       }
     }
   } else if (warp == 1) {
@@ -240,7 +330,8 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         tc_commit(bar(B_SFULL + tq));
       };
       auto act = [&](int tq, int T_) {
-        return (tq == 0 || has1) && tile_vis(causal, static_cast<int>(qts[tq]), T_) != VIS_NONE;
+        return (tq == 0 || has1) &&
+               tile_vis(causal, kBlock ? sc.diag : 0, static_cast<int>(qts[tq]), T_) != VIS_NONE;
       };
       bool have = ok && walk_next(w, T, lo, hi);
       if (have) {
@@ -283,7 +374,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       }
       // Drain: wait for every MMA this thread issued before TMEM is freed.
       tc_commit(bar(B_DRAIN));
-      drain_bar(bar(B_DRAIN), 0, a.budget);
+      drain_bar(bar(B_DRAIN), 0, 166);
     }
   } else {
     // =================================================== softmax warpgroups
@@ -303,7 +394,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       walk_init(w, &sc, qt_last, sv);
       int t, lo = 0, hi = kTile;
       while (ok && walk_next(w, t, lo, hi)) {
-        const int vis = tile_vis(causal, qt, t);
+        const int vis = tile_vis(causal, kBlock ? sc.diag : 0, qt, t);
         if (vis == VIS_NONE) continue;
         ok = __all_sync(0xffffffffu, wait_bar(bar(B_SFULL + tq), cnt & 1, wc, 301));
         if (!ok) break;
@@ -327,14 +418,28 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
           }
         } else if (vis == VIS_DIAG) {
           // keys after the row (past the end of a ragged sequence included,
-          // for every row that is stored)
+          // for every row that is stored when queries and keys are one
+          // sequence; a block call's key block can end inside the diagonal
+          // tile before the query rows do)
+          if constexpr (kBlock) {
+            int lim = r + 1;
+            if (t == w.n_tiles - 1) {
+              const int kv_valid = ld_shared_volatile_s32(seq_smem + 16) - t * kTile;
+              lim = kv_valid < lim ? kv_valid : lim;
+            }
 #pragma unroll
-          for (int i = 0; i < 128; ++i)
-            if (i > r) s[i] = -INFINITY;
+            for (int i = 0; i < 128; ++i)
+              if (i >= lim) s[i] = -INFINITY;
+          } else {
+#pragma unroll
+            for (int i = 0; i < 128; ++i)
+              if (i > r) s[i] = -INFINITY;
+          }
         } else if (t == w.n_tiles - 1) {
           // last key tile of a ragged sequence: rows past its end (S2-Attn
           // sequences are whole tiles, so nothing is masked there)
-          const int kv_valid = ld_shared_volatile_s32(seq_smem) - t * kTile;
+          // (the key count: the sequence's length unless this is a block call)
+          const int kv_valid = ld_shared_volatile_s32(seq_smem + (kBlock ? 16 : 0)) - t * kTile;
           if (kv_valid < kTile) {
 #pragma unroll
             for (int i = 0; i < 128; ++i)
@@ -403,14 +508,24 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       }
       // ---- epilogue: O / l -> bf16 out, lse = ln(2) * (m + log2 l)
       if (ok && cnt >= 1) ok = wait_bar(bar(B_OREADY + tq), (cnt - 1) & 1, wc, 303);
-      ok = __all_sync(0xffffffffu, ok && cnt >= 1);
+      if constexpr (kBlock) {
+        // a query tile before the key block's first diagonal sees no key: its
+        // partial is empty (0, -inf) and still merges
+        ok = __all_sync(0xffffffffu, ok);
+      } else {
+        ok = __all_sync(0xffffffffu, ok && cnt >= 1);
+      }
       const int tok = token_tile(sc, qt, shifted) * kTile + r;
       // Every lane takes part in the TMEM loads (warp-collective); rows past
       // the end of the sequence (ragged last tile) only skip their stores.
       const bool row_in = tok < ld_shared_volatile_s32(seq_smem);
       const size_t trow =
           static_cast<size_t>(ld_shared_volatile_s32(seq_smem + 4)) + (row_in ? tok : 0);
-      if (ok) {
+      if (kBlock && ok) {
+        tc_fence_after();
+        fwd_block_epilogue(a, tO, cnt, m_run, l_run, row_in, trow, h,
+                           static_cast<size_t>(ld_shared_volatile_s64(seq_smem + 8)) + tok);
+      } else if (ok) {
         tc_fence_after();
         const float inv = (l_run > 0.f) ? 1.0f / l_run : 0.f;
         __nv_bfloat16* orow = a.out + (trow * a.Hq + h) * kD;

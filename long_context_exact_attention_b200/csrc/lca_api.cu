@@ -45,6 +45,7 @@ constexpr unsigned long long kDefaultBudget = 1ull << 31;
 
 struct Common {
   int B, Hq, Hkv, S, d;  // tensor extents: B batch entries of S tokens (packed: 1 x total)
+  int S_kv;              // key/value tokens per batch entry (block calls; else S)
   int n_seq;             // sequences (B unless packed)
   int S_seq;             // longest sequence (S unless packed)
   const int* cu;         // packed token offsets (device), else null
@@ -73,6 +74,7 @@ lca_status check_shape(const lca_shape* sh, Common* c) {
   c->Hq = static_cast<int>(sh->Hq);
   c->Hkv = static_cast<int>(sh->Hkv);
   c->S = static_cast<int>(sh->S);
+  c->S_kv = c->S;
   c->d = static_cast<int>(sh->d);
   c->n_seq = c->B;
   c->S_seq = c->S;
@@ -134,6 +136,8 @@ lca_status make_chunk_sched(const Common& c, int causal, int64_t kv_chunk, const
   s->S = c.S_seq;
   s->tile = c.tile;
   s->n_tiles = (c.S_seq + c.tile - 1) / c.tile;
+  s->S_kv = s->S;
+  s->n_kv_tiles = s->n_tiles;
   s->causal = causal ? 1 : 0;
   s->cu_seqlens = c.cu;
   if (kv_chunk < 0) return fail(LCA_ERR_INVALID_ARG, "kv_chunk must be >= 0");
@@ -181,6 +185,8 @@ lca_status make_s2_sched(const Common& c, int causal, int64_t group, int64_t shi
   s->S = c.S;
   s->tile = c.tile;
   s->n_tiles = c.S / c.tile;
+  s->S_kv = s->S;
+  s->n_kv_tiles = s->n_tiles;
   s->causal = causal ? 1 : 0;
   s->s2 = 1;
   s->n_chunks = 1;
@@ -293,13 +299,14 @@ lca_status sm_count(int* n) {
 // The backward kernel's warpgroups redistribute registers with setmaxnreg;
 // the split adds up to exactly the registers the CTA is launched with, so
 // refuse to launch a build whose register count differs.
+template <bool kAccKV>
 lca_status check_bwd_regs() {
   static int regs = -1;
   static std::mutex mu;
   std::lock_guard<std::mutex> lk(mu);
   if (regs < 0) {
     cudaFuncAttributes attr{};
-    const cudaError_t e = cudaFuncGetAttributes(&attr, attn_bwd_bf16_sm100);
+    const cudaError_t e = cudaFuncGetAttributes(&attr, attn_bwd_bf16_sm100<kAccKV>);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes(backward)");
     regs = attr.numRegs;
   }
@@ -313,7 +320,7 @@ lca_status check_bwd_regs() {
 
 // Raise the dynamic shared-memory limit of a kernel once per device; `slot`
 // names the kernel (one per instantiation, below kSmemSlots).
-constexpr int kSmemSlots = 16;
+constexpr int kSmemSlots = 24;
 template <typename K>
 lca_status ensure_smem(K kernel, size_t bytes, int slot) {
   static std::mutex mu;
@@ -342,9 +349,17 @@ unsigned long long budget_of(const lca_opts* o) {
 }
 
 // ---------------------------------------------------------------- forward
+// Block calls pass o_acc (may be null when out is given) and `accumulate`;
+// `block` selects the merging epilogue.
+struct FwdBlock {
+  bool block = false;
+  float* o_acc = nullptr;
+  int accumulate = 0;
+};
+
 lca_status run_fwd(const Common& c, const AttnSched& s, const void* q, const void* k,
                    const void* v, void* out, float* lse, unsigned long long budget,
-                   cudaStream_t st) {
+                   cudaStream_t st, const FwdBlock& fb = FwdBlock()) {
   const int64_t grid64 = static_cast<int64_t>(s.n_tiles) * c.n_seq * c.Hq;
   if (grid64 > 0x7fffffffll)
     return fail(LCA_ERR_INVALID_ARG, "%lld query tiles exceed one launch",
@@ -356,14 +371,24 @@ lca_status run_fwd(const Common& c, const AttnSched& s, const void* q, const voi
     CUtensorMap mq, mk, mv;
     lca_status r;
     if ((r = make_map(&mq, q, c.B, c.S, c.Hq)) != LCA_OK) return r;
-    if ((r = make_map(&mk, k, c.B, c.S, c.Hkv)) != LCA_OK) return r;
-    if ((r = make_map(&mv, v, c.B, c.S, c.Hkv)) != LCA_OK) return r;
+    if ((r = make_map(&mk, k, c.B, c.S_kv, c.Hkv)) != LCA_OK) return r;
+    if ((r = make_map(&mv, v, c.B, c.S_kv, c.Hkv)) != LCA_OK) return r;
     // chunk boundaries inside a tile need the ranged walk
     const bool ranged = !s.s2 && s.kv_chunk % c.tile != 0;
-    if (ranged) {
-      if ((r = ensure_smem(attn_fwd_bf16_sm100<true>, fwd::kSmemBytes, 6)) != LCA_OK) return r;
+    if (fb.block) {
+      if (ranged) {
+        if ((r = ensure_smem(attn_fwd_bf16_sm100<true, true>, fwd::kSmemBytes, 14)) != LCA_OK)
+          return r;
+      } else {
+        if ((r = ensure_smem(attn_fwd_bf16_sm100<false, true>, fwd::kSmemBytes, 13)) != LCA_OK)
+          return r;
+      }
+    } else if (ranged) {
+      if ((r = ensure_smem(attn_fwd_bf16_sm100<true, false>, fwd::kSmemBytes, 6)) != LCA_OK)
+        return r;
     } else {
-      if ((r = ensure_smem(attn_fwd_bf16_sm100<false>, fwd::kSmemBytes, 0)) != LCA_OK) return r;
+      if ((r = ensure_smem(attn_fwd_bf16_sm100<false, false>, fwd::kSmemBytes, 0)) != LCA_OK)
+        return r;
     }
     fwd::Args a;
     a.B = c.n_seq;
@@ -374,11 +399,21 @@ lca_status run_fwd(const Common& c, const AttnSched& s, const void* q, const voi
     a.budget = budget;
     a.out = static_cast<__nv_bfloat16*>(out);
     a.lse = lse;
+    a.o_acc = fb.o_acc;
+    a.accumulate = fb.accumulate;
     a.sched = s;
-    if (ranged)
-      attn_fwd_bf16_sm100<true><<<grid2, fwd::kThreads, fwd::kSmemBytes, st>>>(mq, mk, mv, a);
+    if (fb.block && ranged)
+      attn_fwd_bf16_sm100<true, true><<<grid2, fwd::kThreads, fwd::kSmemBytes, st>>>(mq, mk, mv,
+                                                                                      a);
+    else if (fb.block)
+      attn_fwd_bf16_sm100<false, true><<<grid2, fwd::kThreads, fwd::kSmemBytes, st>>>(mq, mk, mv,
+                                                                                       a);
+    else if (ranged)
+      attn_fwd_bf16_sm100<true, false><<<grid2, fwd::kThreads, fwd::kSmemBytes, st>>>(mq, mk, mv,
+                                                                                       a);
     else
-      attn_fwd_bf16_sm100<false><<<grid2, fwd::kThreads, fwd::kSmemBytes, st>>>(mq, mk, mv, a);
+      attn_fwd_bf16_sm100<false, false><<<grid2, fwd::kThreads, fwd::kSmemBytes, st>>>(mq, mk,
+                                                                                        mv, a);
     return launched("attn_fwd_bf16_sm100");
   }
   f32::Args a{};
@@ -419,15 +454,110 @@ size_t ws_bytes_of(const Common& c) {
   return n;
 }
 
-lca_status run_bwd(const Common& c, const AttnSched& s, const void* q, const void* k,
-                   const void* v, const void* out, const float* lse, const void* dout, void* dq,
-                   void* dk, void* dv, void* ws, size_t ws_bytes, unsigned long long budget,
-                   cudaStream_t st) {
+// bf16 backward in three phases over the workspace (D | lse copy | dq
+// accumulator): prep (zero the accumulator, D rows and the padded lse copy),
+// main (the tensor-core kernel: dK/dV of every key tile, dQ added into the
+// accumulator), dq (scale and round the accumulator).  lca_attn_bwd runs
+// all three; block calls run prep once per query block, main once per key
+// block, and dq at the end.
+lca_status bwd_prep(const Common& c, const void* out, const float* lse, const void* dout,
+                    void* ws, cudaStream_t st) {
+  const int S_pad = s_pad_of(c);
+  float* Drow = static_cast<float*>(ws);
+  float* lse_pad = reinterpret_cast<float*>(static_cast<char*>(ws) + ws_d_bytes(c));
+  float* acc = reinterpret_cast<float*>(static_cast<char*>(ws) + 2 * ws_d_bytes(c));
+  const int64_t rows = static_cast<int64_t>(c.B) * c.S * c.Hq;
+  const int64_t pad_rows = static_cast<int64_t>(c.n_seq) * S_pad * c.Hq;
+  const unsigned rd_blocks =
+      static_cast<unsigned>(std::min<int64_t>((pad_rows * 32 + 255) / 256, 148 * 64));
+  const cudaError_t e =
+      cudaMemsetAsync(acc, 0, static_cast<size_t>(rows) * c.d * sizeof(float), st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(dq accumulator)");
+  bwd_rowdot<__nv_bfloat16, 128><<<rd_blocks, 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse, Drow,
+      lse_pad, c.n_seq, c.S, S_pad, c.Hq, c.cu);
+  return launched("bwd_rowdot");
+}
+
+// dk/dv (bf16, overwritten) or dk_acc/dv_acc (float32, added to when
+// acc_add, else overwritten): exactly one pair is non-null.
+lca_status bwd_main(const Common& c, const AttnSched& s, const void* q, const void* k,
+                    const void* v, const void* dout, void* ws, void* dk, void* dv, float* dk_acc,
+                    float* dv_acc, int acc_add, unsigned long long budget, cudaStream_t st) {
+  const int S_pad = s_pad_of(c);
+  float* Drow = static_cast<float*>(ws);
+  float* lse_pad = reinterpret_cast<float*>(static_cast<char*>(ws) + ws_d_bytes(c));
+  float* acc = reinterpret_cast<float*>(static_cast<char*>(ws) + 2 * ws_d_bytes(c));
+  const int64_t grid64 = static_cast<int64_t>(s.n_kv_tiles) * c.n_seq * c.Hkv;
+  if (grid64 > 0x7fffffffll)
+    return fail(LCA_ERR_INVALID_ARG, "%lld key tiles exceed one launch",
+                static_cast<long long>(grid64));
+  const unsigned grid = static_cast<unsigned>(grid64);
+  const bool acc_kv = dk_acc != nullptr;
+  lca_status r;
+  CUtensorMap mq, mk, mv, mdo, mdq;
+  if ((r = make_map(&mq, q, c.B, c.S, c.Hq)) != LCA_OK) return r;
+  if ((r = make_map(&mk, k, c.B, c.S_kv, c.Hkv)) != LCA_OK) return r;
+  if ((r = make_map(&mv, v, c.B, c.S_kv, c.Hkv)) != LCA_OK) return r;
+  if ((r = make_map(&mdo, dout, c.B, c.S, c.Hq)) != LCA_OK) return r;
+  if ((r = make_map_acc(&mdq, acc, c.B, c.S, c.Hq)) != LCA_OK) return r;
+  if (acc_kv) {
+    if ((r = check_bwd_regs<true>()) != LCA_OK) return r;
+    if ((r = ensure_smem(attn_bwd_bf16_sm100<true>, bwd::kSmemBytes, 15)) != LCA_OK) return r;
+  } else {
+    if ((r = check_bwd_regs<false>()) != LCA_OK) return r;
+    if ((r = ensure_smem(attn_bwd_bf16_sm100<false>, bwd::kSmemBytes, 3)) != LCA_OK) return r;
+  }
+  bwd::Args a;
+  a.B = c.n_seq;
+  a.Hq = c.Hq;
+  a.Hkv = c.Hkv;
+  a.S = c.S;
+  a.S_pad = S_pad;
+  a.scale = c.scale;
+  a.scale_log2 = c.scale * 1.4426950408889634f;
+  a.budget = budget;
+  a.lse = lse_pad;
+  a.Drow = Drow;
+  a.dk = static_cast<__nv_bfloat16*>(dk);
+  a.dv = static_cast<__nv_bfloat16*>(dv);
+  a.dk_acc = dk_acc;
+  a.dv_acc = dv_acc;
+  a.acc_add = acc_add;
+  a.sched = s;
+  if (acc_kv)
+    attn_bwd_bf16_sm100<true><<<grid, bwd::kThreads, bwd::kSmemBytes, st>>>(mq, mk, mv, mdo, mdq,
+                                                                            a);
+  else
+    attn_bwd_bf16_sm100<false><<<grid, bwd::kThreads, bwd::kSmemBytes, st>>>(mq, mk, mv, mdo,
+                                                                             mdq, a);
+  return launched("attn_bwd_bf16_sm100");
+}
+
+lca_status bwd_dq(const Common& c, const void* ws, void* dq, cudaStream_t st) {
+  const float* acc =
+      reinterpret_cast<const float*>(static_cast<const char*>(ws) + 2 * ws_d_bytes(c));
+  const int64_t n8 = static_cast<int64_t>(c.B) * c.S * c.Hq * c.d / 8;
+  dq_finalize<<<static_cast<unsigned>(std::min<int64_t>((n8 + 255) / 256, 148 * 16)), 256, 0,
+                st>>>(acc, static_cast<__nv_bfloat16*>(dq), n8, c.scale);
+  return launched("dq_finalize");
+}
+
+lca_status check_ws(const Common& c, const void* ws, size_t ws_bytes) {
   if (!ws) return fail(LCA_ERR_WORKSPACE, "workspace is NULL");
   if (ws_bytes < ws_bytes_of(c))
     return fail(LCA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes,
                 ws_bytes_of(c));
   if (!aligned16(ws)) return fail(LCA_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+  return LCA_OK;
+}
+
+lca_status run_bwd(const Common& c, const AttnSched& s, const void* q, const void* k,
+                   const void* v, const void* out, const float* lse, const void* dout, void* dq,
+                   void* dk, void* dv, void* ws, size_t ws_bytes, unsigned long long budget,
+                   cudaStream_t st) {
+  lca_status r = check_ws(c, ws, ws_bytes);
+  if (r != LCA_OK) return r;
   const int S_pad = s_pad_of(c);
   float* Drow = static_cast<float*>(ws);
   float* lse_pad = reinterpret_cast<float*>(static_cast<char*>(ws) + ws_d_bytes(c));
@@ -441,44 +571,12 @@ lca_status run_bwd(const Common& c, const AttnSched& s, const void* q, const voi
                 static_cast<long long>(grid64));
   const unsigned grid = static_cast<unsigned>(grid64);
   cudaError_t e;
-  lca_status r;
   if (c.dtype == LCA_BF16) {
-    float* acc = reinterpret_cast<float*>(static_cast<char*>(ws) + 2 * ws_d_bytes(c));
-    const size_t acc_bytes = static_cast<size_t>(rows) * c.d * sizeof(float);
-    e = cudaMemsetAsync(acc, 0, acc_bytes, st);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(dq accumulator)");
-    bwd_rowdot<__nv_bfloat16, 128><<<rd_blocks, 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse,
-        Drow, lse_pad, c.n_seq, c.S, S_pad, c.Hq, c.cu);
-    if ((r = launched("bwd_rowdot")) != LCA_OK) return r;
-    CUtensorMap mq, mk, mv, mdo, mdq;
-    if ((r = make_map(&mq, q, c.B, c.S, c.Hq)) != LCA_OK) return r;
-    if ((r = make_map(&mk, k, c.B, c.S, c.Hkv)) != LCA_OK) return r;
-    if ((r = make_map(&mv, v, c.B, c.S, c.Hkv)) != LCA_OK) return r;
-    if ((r = make_map(&mdo, dout, c.B, c.S, c.Hq)) != LCA_OK) return r;
-    if ((r = make_map_acc(&mdq, acc, c.B, c.S, c.Hq)) != LCA_OK) return r;
-    if ((r = check_bwd_regs()) != LCA_OK) return r;
-    if ((r = ensure_smem(attn_bwd_bf16_sm100, bwd::kSmemBytes, 3)) != LCA_OK) return r;
-    bwd::Args a;
-    a.B = c.n_seq;
-    a.Hq = c.Hq;
-    a.Hkv = c.Hkv;
-    a.S = c.S;
-    a.S_pad = S_pad;
-    a.scale = c.scale;
-    a.scale_log2 = c.scale * 1.4426950408889634f;
-    a.budget = budget;
-    a.lse = lse_pad;
-    a.Drow = Drow;
-    a.dk = static_cast<__nv_bfloat16*>(dk);
-    a.dv = static_cast<__nv_bfloat16*>(dv);
-    a.sched = s;
-    attn_bwd_bf16_sm100<<<grid, bwd::kThreads, bwd::kSmemBytes, st>>>(mq, mk, mv, mdo, mdq, a);
-    if ((r = launched("attn_bwd_bf16_sm100")) != LCA_OK) return r;
-    const int64_t n8 = rows * c.d / 8;
-    dq_finalize<<<static_cast<unsigned>(std::min<int64_t>((n8 + 255) / 256, 148 * 16)), 256, 0,
-                  st>>>(acc, static_cast<__nv_bfloat16*>(dq), n8, c.scale);
-    return launched("dq_finalize");
+    if ((r = bwd_prep(c, out, lse, dout, ws, st)) != LCA_OK) return r;
+    if ((r = bwd_main(c, s, q, k, v, dout, ws, dk, dv, nullptr, nullptr, 0, budget, st)) !=
+        LCA_OK)
+      return r;
+    return bwd_dq(c, ws, dq, st);
   }
   // fp32
   e = cudaMemsetAsync(dq, 0, static_cast<size_t>(rows) * c.d * sizeof(float), st);
@@ -713,11 +811,23 @@ lca_status check_ffn(const lca_ffn_shape* sh, int64_t* block) {
   return LCA_OK;
 }
 
+// Band heights of the feedforward tile raster (row tiles).  Products whose B
+// (weight) operand is the large one and is swept column by column take the
+// whole block of rows as one band, so every weight column is read from DRAM
+// once per block while the block's A rows stay in L2; products whose B fits
+// in L2 whole (W_down for the down product, the block's x for the weight
+// gradients) go row tile by row tile, so B stays resident and A is read once.
+constexpr int kFfnBandWide = 1 << 20;
+constexpr int kFfnBandNarrow = 1;
+
 template <int kEpi, bool kAmn, bool kBmn, bool kSplit>
 lca_status launch_ffn_gemm(const CUtensorMap& ma0, const CUtensorMap& ma1, const CUtensorMap& mb0,
-                           const CUtensorMap& mb1, const ffn::Args& a, int slot,
+                           const CUtensorMap& mb1, const ffn::Args& a0, int slot,
                            cudaStream_t st) {
   auto kernel = ffn_gemm_sm100<kEpi, kAmn, kBmn, kSplit>;
+  if (a0.group_m < 1) return fail(LCA_ERR_INVALID_ARG, "internal: feedforward band height < 1");
+  ffn::Args a = a0;
+  if (a.group_m > a.n_tm) a.group_m = a.n_tm;  // one band at most (keeps t / (gm * n_tn) small)
   lca_status r = ensure_smem(kernel, ffn::kSmemBytes, slot);
   if (r != LCA_OK) return r;
   int sms = 0;
@@ -726,6 +836,279 @@ lca_status launch_ffn_gemm(const CUtensorMap& ma0, const CUtensorMap& ma1, const
   const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
   kernel<<<grid, ffn::kThreads, ffn::kSmemBytes, st>>>(ma0, ma1, mb0, mb1, a);
   return launched("ffn_gemm_sm100");
+}
+
+// ---------------------------------------------------------------- feedforward blocks
+// The products of one block of token rows [r0, r0 + rows) of the
+// feedforward, over tensor maps made once per call (x, dout and the
+// outputs span all T rows; the intermediates span one block).
+struct FfnFwdPlan {
+  CUtensorMap mx, mg, mu, md, mh;
+  int64_t h, f;
+  void* out;
+  void* H;
+};
+
+lca_status ffn_fwd_plan(const void* x, const void* w_gate, const void* w_up, const void* w_down,
+                        int64_t T, int64_t h, int64_t f, int64_t block, void* out, void* H,
+                        FfnFwdPlan* p) {
+  lca_status r;
+  if ((r = make_map_2d(&p->mx, x, T, h)) != LCA_OK) return r;
+  if ((r = make_map_2d(&p->mg, w_gate, f, h)) != LCA_OK) return r;
+  if ((r = make_map_2d(&p->mu, w_up, f, h)) != LCA_OK) return r;
+  if ((r = make_map_2d(&p->md, w_down, h, f)) != LCA_OK) return r;
+  if ((r = make_map_2d(&p->mh, H, block, f)) != LCA_OK) return r;
+  p->h = h;
+  p->f = f;
+  p->out = out;
+  p->H = H;
+  return LCA_OK;
+}
+
+lca_status ffn_fwd_rows(const FfnFwdPlan& p, int64_t r0, int rows, cudaStream_t st) {
+  const int64_t h = p.h, f = p.f;
+  lca_status r;
+  ffn::Args g1{};
+  g1.M = rows;
+  g1.K = static_cast<int>(h);
+  g1.n_tm = (rows + ffn::kBM - 1) / ffn::kBM;
+  g1.n_tn = static_cast<int>(f / 128);
+  g1.a_off = static_cast<int>(r0);
+  g1.ldo = static_cast<int>(f);
+  g1.budget = kDefaultBudget;
+  g1.group_m = kFfnBandWide;
+  g1.out = static_cast<__nv_bfloat16*>(p.H);
+  if ((r = launch_ffn_gemm<ffn::EPI_SWIGLU, false, false, false>(p.mx, p.mx, p.mg, p.mu, g1, 7,
+                                                                 st)) != LCA_OK)
+    return r;
+  ffn::Args g2{};
+  g2.M = rows;
+  g2.K = static_cast<int>(f);
+  g2.n_tm = g1.n_tm;
+  g2.n_tn = static_cast<int>(h / ffn::kBN);
+  g2.a_off = 0;
+  g2.ldo = static_cast<int>(h);
+  g2.budget = kDefaultBudget;
+  g2.group_m = kFfnBandNarrow;
+  g2.out = static_cast<__nv_bfloat16*>(p.out) + r0 * h;
+  return launch_ffn_gemm<ffn::EPI_STORE, false, false, false>(p.mh, p.mh, p.md, p.md, g2, 8, st);
+}
+
+struct FfnBwdPlan {
+  // K-major views (boxes of 128 rows) and MN-major views (boxes of 64 rows)
+  CUtensorMap x_k, x_mn, do_k, do_mn, wg_k, wu_k, wg_mn, wu_mn, wd_mn, dg_k, du_k, dgu_mn, h_mn;
+  int64_t h, f;
+  __nv_bfloat16 *dH, *dGU, *H;
+  float *dw_gate, *dw_up, *dw_down;
+};
+
+// ws: dH [block, f] | [dG | dU] [block, 2f] | H [block, f], bf16
+lca_status ffn_bwd_plan(const void* x, const void* w_gate, const void* w_up, const void* w_down,
+                        const void* dout, int64_t T, int64_t h, int64_t f, int64_t block,
+                        float* dw_gate, float* dw_up, float* dw_down, void* workspace,
+                        FfnBwdPlan* p) {
+  auto* ws = static_cast<__nv_bfloat16*>(workspace);
+  p->dH = ws;
+  p->dGU = ws + block * f;
+  p->H = ws + 3 * block * f;
+  p->h = h;
+  p->f = f;
+  p->dw_gate = dw_gate;
+  p->dw_up = dw_up;
+  p->dw_down = dw_down;
+  lca_status r;
+  if ((r = make_map_2d(&p->x_k, x, T, h)) != LCA_OK) return r;
+  if ((r = make_map_2d(&p->x_mn, x, T, h, 64)) != LCA_OK) return r;
+  if ((r = make_map_2d(&p->do_k, dout, T, h)) != LCA_OK) return r;
+  if ((r = make_map_2d(&p->do_mn, dout, T, h, 64)) != LCA_OK) return r;
+  if ((r = make_map_2d(&p->wg_k, w_gate, f, h)) != LCA_OK) return r;
+  if ((r = make_map_2d(&p->wu_k, w_up, f, h)) != LCA_OK) return r;
+  if ((r = make_map_2d(&p->wg_mn, w_gate, f, h, 64)) != LCA_OK) return r;
+  if ((r = make_map_2d(&p->wu_mn, w_up, f, h, 64)) != LCA_OK) return r;
+  if ((r = make_map_2d(&p->wd_mn, w_down, h, f, 64)) != LCA_OK) return r;
+  if ((r = make_map_2d(&p->dg_k, p->dGU, block, f, 128, 2 * f)) != LCA_OK) return r;
+  if ((r = make_map_2d(&p->du_k, p->dGU + f, block, f, 128, 2 * f)) != LCA_OK) return r;
+  if ((r = make_map_2d(&p->dgu_mn, p->dGU, block, 2 * f, 64)) != LCA_OK) return r;
+  return make_map_2d(&p->h_mn, p->H, block, f, 64);
+}
+
+// dx_rows: where row r0 of dx goes (the plan's dx + r0 * h for a whole-T
+// dx; a block-sized buffer for a caller that consumes dx block by block).
+lca_status ffn_bwd_rows(const FfnBwdPlan& p, int64_t r0, int rows, void* dx_rows,
+                        cudaStream_t st) {
+  const int64_t h = p.h, f = p.f;
+  const int n_tm = (rows + ffn::kBM - 1) / ffn::kBM;
+  const int k_rows = (rows + ffn::kBK - 1) / ffn::kBK * ffn::kBK;  // whole K steps
+  lca_status r;
+  ffn::Args g{};
+  g.budget = kDefaultBudget;
+  // dH = dout W_down
+  g.M = rows, g.K = static_cast<int>(h), g.n_tm = n_tm, g.n_tn = static_cast<int>(f / ffn::kBN);
+  g.group_m = kFfnBandWide;
+  g.a_off = static_cast<int>(r0), g.b_off = 0, g.ldo = static_cast<int>(f), g.out = p.dH;
+  if ((r = launch_ffn_gemm<ffn::EPI_STORE, false, true, false>(p.do_k, p.do_k, p.wd_mn, p.wd_mn,
+                                                               g, 9, st)) != LCA_OK)
+    return r;
+  // G, U recomputed; dG, dU, H written
+  g = ffn::Args{};
+  g.budget = kDefaultBudget;
+  g.M = rows, g.K = static_cast<int>(h), g.n_tm = n_tm, g.n_tn = static_cast<int>(f / 128);
+  g.group_m = kFfnBandWide;
+  g.a_off = static_cast<int>(r0), g.b_off = 0, g.ldo = static_cast<int>(2 * f);
+  g.ldo3 = static_cast<int>(f), g.ld_in = static_cast<int>(f), g.in = p.dH;
+  g.out = p.dGU, g.out2 = p.dGU + f, g.out3 = p.H;
+  if ((r = launch_ffn_gemm<ffn::EPI_SWIGLU_BWD, false, false, false>(p.x_k, p.x_k, p.wg_k, p.wu_k,
+                                                                     g, 10, st)) != LCA_OK)
+    return r;
+  // dX = dG W_gate + dU W_up
+  g = ffn::Args{};
+  g.budget = kDefaultBudget;
+  g.M = rows, g.K = static_cast<int>(2 * f), g.n_tm = n_tm, g.n_tn = static_cast<int>(h / ffn::kBN);
+  g.group_m = kFfnBandNarrow;
+  g.a_off = 0, g.b_off = 0, g.ldo = static_cast<int>(h);
+  g.out = static_cast<__nv_bfloat16*>(dx_rows);
+  if ((r = launch_ffn_gemm<ffn::EPI_STORE, false, true, true>(p.dg_k, p.du_k, p.wg_mn, p.wu_mn, g,
+                                                              11, st)) != LCA_OK)
+    return r;
+  // [dW_gate; dW_up] += [dG | dU]^T x: one product, rows split at f
+  g = ffn::Args{};
+  g.budget = kDefaultBudget;
+  g.M = static_cast<int>(2 * f), g.K = k_rows, g.n_tm = static_cast<int>(2 * f / ffn::kBM);
+  g.group_m = kFfnBandNarrow;
+  g.n_tn = static_cast<int>(h / ffn::kBN);
+  g.a_off = 0, g.b_off = static_cast<int>(r0), g.ldo = static_cast<int>(h);
+  g.m_split = static_cast<int>(f), g.out32 = p.dw_gate, g.out32b = p.dw_up;
+  if ((r = launch_ffn_gemm<ffn::EPI_ACC32, true, true, false>(p.dgu_mn, p.dgu_mn, p.x_mn, p.x_mn,
+                                                              g, 12, st)) != LCA_OK)
+    return r;
+  // dW_down += dout^T H
+  g.M = static_cast<int>(h), g.m_split = static_cast<int>(h), g.out32b = nullptr;
+  g.group_m = kFfnBandWide;
+  g.n_tm = static_cast<int>(h / ffn::kBM);
+  g.n_tn = static_cast<int>(f / ffn::kBN);
+  g.a_off = static_cast<int>(r0), g.b_off = 0, g.ldo = static_cast<int>(f), g.out32 = p.dw_down;
+  return launch_ffn_gemm<ffn::EPI_ACC32, true, true, false>(p.do_mn, p.do_mn, p.h_mn, p.h_mn, g,
+                                                            12, st);
+}
+
+// ---------------------------------------------------------------- blocks
+// A query block of Sq rows at position q_pos0 against a key/value block of
+// Sk keys at position k_pos0 (a sequence-parallel ring step).
+lca_status check_block(const lca_block_shape* sh, Common* c) {
+  if (!sh) return fail(LCA_ERR_INVALID_ARG, "shape is NULL");
+  const lca_shape one{sh->B, sh->Hq, sh->Hkv, sh->Sq, sh->d, sh->dtype, sh->scale};
+  lca_status r = check_shape(&one, c);
+  if (r != LCA_OK) return r;
+  if (sh->Sk <= 0) return fail(LCA_ERR_INVALID_ARG, "dimensions must be positive");
+  if (sh->Sk > (1ll << 26)) return fail(LCA_ERR_INVALID_ARG, "dimension too large");
+  if (sh->B * sh->Sk > (1ll << 31) - 1)
+    return fail(LCA_ERR_INVALID_ARG, "B*Sk must fit in 31 bits");
+  if (c->dtype != LCA_BF16)
+    return fail(LCA_ERR_UNSUPPORTED, "block calls run on the bf16 tensor-core path only");
+  c->S_kv = static_cast<int>(sh->Sk);
+  return LCA_OK;
+}
+
+enum { REL_NONE = 0, REL_FULL = 1, REL_CAUSAL = 2 };
+
+// Which keys of the block the queries see: all (REL_FULL), none (REL_NONE)
+// or a causal band whose diagonal key tile for query tile Q is Q + *diag.
+lca_status block_relation(const Common& c, int causal, int64_t q_pos0, int64_t k_pos0, int* rel,
+                          int* diag) {
+  if (q_pos0 < 0 || k_pos0 < 0 || q_pos0 > (1ll << 40) || k_pos0 > (1ll << 40))
+    return fail(LCA_ERR_INVALID_ARG, "block positions must lie in [0, 2^40]");
+  *diag = 0;
+  if (!causal || k_pos0 + c.S_kv - 1 <= q_pos0) {
+    *rel = REL_FULL;
+  } else if (k_pos0 > q_pos0 + c.S - 1) {
+    *rel = REL_NONE;
+  } else {
+    if ((q_pos0 - k_pos0) % c.tile)
+      return fail(LCA_ERR_INVALID_ARG,
+                  "causal blocks that overlap on the diagonal must start a multiple of %d "
+                  "positions apart",
+                  c.tile);
+    *rel = REL_CAUSAL;
+    *diag = static_cast<int>((q_pos0 - k_pos0) / c.tile);
+  }
+  return LCA_OK;
+}
+
+// The schedule of one block: one chunk spanning the key block, in order.
+// REL_NONE becomes a causal band with its diagonal before every key tile
+// (no query sees a key), which the kernels turn into empty results.
+void make_block_sched(const Common& c, int rel, int diag, AttnSched* s) {
+  std::memset(s, 0, sizeof *s);
+  s->S = c.S;
+  s->tile = c.tile;
+  s->n_tiles = (c.S + c.tile - 1) / c.tile;
+  s->S_kv = c.S_kv;
+  s->n_kv_tiles = (c.S_kv + c.tile - 1) / c.tile;
+  s->causal = rel != REL_FULL;
+  s->diag = rel == REL_NONE ? -(s->n_tiles + 1) : diag;
+  s->kv_chunk = c.S_kv;
+  s->n_chunks = 1;
+  s->order = LCA_ORDER_INORDER;
+  s->q_block = c.S;
+}
+
+// ---------------------------------------------------------------- blockwise transformer
+// One sweep of the Blockwise Transformer over the query blocks: per block,
+// the attention of its rows over the keys they see, then the feedforward of
+// those rows.
+struct BptPlan {
+  Common attn;     // shape of a full query block (rows == q_block)
+  int64_t S, h, f, qb;
+  int causal;
+};
+
+lca_status check_bpt(const lca_bpt_shape* sh, int backward, BptPlan* p) {
+  if (!sh) return fail(LCA_ERR_INVALID_ARG, "shape is NULL");
+  if (sh->S <= 0 || sh->Hq <= 0 || sh->Hkv <= 0 || sh->d <= 0 || sh->f <= 0)
+    return fail(LCA_ERR_INVALID_ARG, "dimensions must be positive");
+  const int64_t qb = sh->q_block ? sh->q_block : LCA_FFN_BLOCK_DEFAULT;
+  if (qb <= 0 || qb % 128) return fail(LCA_ERR_INVALID_ARG, "q_block must be a positive multiple of 128");
+  const lca_block_shape bs{1, sh->Hq, sh->Hkv, qb < sh->S ? qb : sh->S, sh->S, sh->d, LCA_BF16,
+                           sh->scale};
+  lca_status r = check_block(&bs, &p->attn);
+  if (r != LCA_OK) return r;
+  const lca_ffn_shape fs{sh->S, sh->Hq * sh->d, sh->f};
+  int64_t blk = qb;
+  if ((r = check_ffn(&fs, &blk)) != LCA_OK) return r;
+  if (backward && sh->f % ffn::kBN)
+    return fail(LCA_ERR_UNSUPPORTED, "feedforward backward needs f %% 256 == 0");
+  p->S = sh->S;
+  p->h = sh->Hq * sh->d;
+  p->f = sh->f;
+  p->qb = qb;
+  return LCA_OK;
+}
+
+// Attention shape and schedule of the query block [r0, r0 + rows): its
+// rows against keys [0, r0 + rows) (causal) or all keys.
+void bpt_block(const BptPlan& p, int causal, int64_t r0, int rows, Common* c, AttnSched* s) {
+  *c = p.attn;
+  c->S = rows;
+  c->S_seq = rows;
+  c->S_kv = static_cast<int>(causal ? r0 + rows : p.S);
+  int rel, diag;
+  block_relation(*c, causal, r0, 0, &rel, &diag);  // r0 is a multiple of the tile
+  make_block_sched(*c, rel, diag, s);
+}
+
+size_t bpt_fwd_ws(const BptPlan& p) {
+  return align256(static_cast<size_t>(p.attn.Hq) * p.qb * 4) +
+         static_cast<size_t>(p.qb) * p.f * 2;  // lse of a block | H of a block
+}
+
+size_t bpt_bwd_ws(const BptPlan& p) {
+  Common c = p.attn;  // a full block
+  const size_t kv = static_cast<size_t>(p.S) * p.attn.Hkv * p.attn.d * 4;
+  return 4 * static_cast<size_t>(p.qb) * p.f * 2           // feedforward backward
+         + align256(static_cast<size_t>(p.qb) * p.h * 2)    // d(attention out) of a block
+         + align256(ws_bytes_of(c))                          // attention backward of a block
+         + align256(static_cast<size_t>(p.attn.Hq) * p.qb * 4)  // lse of a block
+         + 2 * align256(kv);                                 // dk, dv accumulators
 }
 
 }  // namespace
@@ -905,40 +1288,14 @@ lca_status lca_ffn_fwd(const lca_ffn_shape* shape, const void* x, const void* w_
   if (ws_bytes < need)
     return fail(LCA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, need);
   if (!aligned16(workspace)) return fail(LCA_ERR_INVALID_ARG, "workspace not 16-byte aligned");
-  const int64_t T = shape->T, h = shape->h, f = shape->f;
-  CUtensorMap mx, mg, mu, md, mh;
-  if ((r = make_map_2d(&mx, x, T, h)) != LCA_OK) return r;
-  if ((r = make_map_2d(&mg, w_gate, f, h)) != LCA_OK) return r;
-  if ((r = make_map_2d(&mu, w_up, f, h)) != LCA_OK) return r;
-  if ((r = make_map_2d(&md, w_down, h, f)) != LCA_OK) return r;
-  if ((r = make_map_2d(&mh, workspace, block, f)) != LCA_OK) return r;
+  FfnFwdPlan p;
+  if ((r = ffn_fwd_plan(x, w_gate, w_up, w_down, shape->T, shape->h, shape->f, block, out,
+                        workspace, &p)) != LCA_OK)
+    return r;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  for (int64_t r0 = 0; r0 < T; r0 += block) {
-    const int rows = static_cast<int>(T - r0 < block ? T - r0 : block);
-    ffn::Args g1{};
-    g1.M = rows;
-    g1.K = static_cast<int>(h);
-    g1.n_tm = (rows + ffn::kBM - 1) / ffn::kBM;
-    g1.n_tn = static_cast<int>(f / 128);
-    g1.a_off = static_cast<int>(r0);
-    g1.ldo = static_cast<int>(f);
-    g1.budget = kDefaultBudget;
-    g1.out = static_cast<__nv_bfloat16*>(workspace);
-    if ((r = launch_ffn_gemm<ffn::EPI_SWIGLU, false, false, false>(mx, mx, mg, mu, g1, 7, st)) !=
-        LCA_OK)
-      return r;
-    ffn::Args g2{};
-    g2.M = rows;
-    g2.K = static_cast<int>(f);
-    g2.n_tm = g1.n_tm;
-    g2.n_tn = static_cast<int>(h / ffn::kBN);
-    g2.a_off = 0;
-    g2.ldo = static_cast<int>(h);
-    g2.budget = kDefaultBudget;
-    g2.out = static_cast<__nv_bfloat16*>(out) + r0 * h;
-    if ((r = launch_ffn_gemm<ffn::EPI_STORE, false, false, false>(mh, mh, md, md, g2, 8, st)) !=
-        LCA_OK)
-      return r;
+  for (int64_t r0 = 0; r0 < shape->T; r0 += block) {
+    const int rows = static_cast<int>(shape->T - r0 < block ? shape->T - r0 : block);
+    if ((r = ffn_fwd_rows(p, r0, rows, st)) != LCA_OK) return r;
   }
   return LCA_OK;
 }
@@ -964,80 +1321,19 @@ lca_status lca_ffn_bwd(const lca_ffn_shape* shape, const void* x, const void* w_
   if ((r = check_ptrs({x, w_gate, w_up, w_down, dout, dx, dw_gate, dw_up, dw_down})) != LCA_OK)
     return r;
   if (!workspace) return fail(LCA_ERR_WORKSPACE, "workspace is NULL");
-  const int64_t T = shape->T, h = shape->h, f = shape->f;
-  const size_t one = static_cast<size_t>(block) * static_cast<size_t>(f) * 2;
+  const size_t one = static_cast<size_t>(block) * static_cast<size_t>(shape->f) * 2;
   if (ws_bytes < 4 * one)
     return fail(LCA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, 4 * one);
   if (!aligned16(workspace)) return fail(LCA_ERR_INVALID_ARG, "workspace not 16-byte aligned");
-  auto* ws = static_cast<__nv_bfloat16*>(workspace);
-  // dH [block, f] | [dG | dU] [block, 2f] | H [block, f]
-  __nv_bfloat16* dH = ws;
-  __nv_bfloat16* dGU = ws + block * f;
-  __nv_bfloat16* H = ws + 3 * block * f;
-  // K-major views (boxes of 128 rows) and MN-major views (boxes of 64 rows)
-  CUtensorMap x_k, x_mn, do_k, do_mn, wg_k, wu_k, wg_mn, wu_mn, wd_mn, dg_k, du_k, dgu_mn, h_mn;
-  if ((r = make_map_2d(&x_k, x, T, h)) != LCA_OK) return r;
-  if ((r = make_map_2d(&x_mn, x, T, h, 64)) != LCA_OK) return r;
-  if ((r = make_map_2d(&do_k, dout, T, h)) != LCA_OK) return r;
-  if ((r = make_map_2d(&do_mn, dout, T, h, 64)) != LCA_OK) return r;
-  if ((r = make_map_2d(&wg_k, w_gate, f, h)) != LCA_OK) return r;
-  if ((r = make_map_2d(&wu_k, w_up, f, h)) != LCA_OK) return r;
-  if ((r = make_map_2d(&wg_mn, w_gate, f, h, 64)) != LCA_OK) return r;
-  if ((r = make_map_2d(&wu_mn, w_up, f, h, 64)) != LCA_OK) return r;
-  if ((r = make_map_2d(&wd_mn, w_down, h, f, 64)) != LCA_OK) return r;
-  if ((r = make_map_2d(&dg_k, dGU, block, f, 128, 2 * f)) != LCA_OK) return r;
-  if ((r = make_map_2d(&du_k, dGU + f, block, f, 128, 2 * f)) != LCA_OK) return r;
-  if ((r = make_map_2d(&dgu_mn, dGU, block, 2 * f, 64)) != LCA_OK) return r;
-  if ((r = make_map_2d(&h_mn, H, block, f, 64)) != LCA_OK) return r;
+  FfnBwdPlan p;
+  if ((r = ffn_bwd_plan(x, w_gate, w_up, w_down, dout, shape->T, shape->h, shape->f, block,
+                        dw_gate, dw_up, dw_down, workspace, &p)) != LCA_OK)
+    return r;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  for (int64_t r0 = 0; r0 < T; r0 += block) {
-    const int rows = static_cast<int>(T - r0 < block ? T - r0 : block);
-    const int n_tm = (rows + ffn::kBM - 1) / ffn::kBM;
-    const int k_rows = (rows + ffn::kBK - 1) / ffn::kBK * ffn::kBK;  // whole K steps
-    ffn::Args g{};
-    g.budget = kDefaultBudget;
-    // dH = dout W_down
-    g.M = rows, g.K = static_cast<int>(h), g.n_tm = n_tm, g.n_tn = static_cast<int>(f / ffn::kBN);
-    g.a_off = static_cast<int>(r0), g.b_off = 0, g.ldo = static_cast<int>(f), g.out = dH;
-    if ((r = launch_ffn_gemm<ffn::EPI_STORE, false, true, false>(do_k, do_k, wd_mn, wd_mn, g, 9,
-                                                                 st)) != LCA_OK)
-      return r;
-    // G, U recomputed; dG, dU, H written
-    g = ffn::Args{};
-    g.budget = kDefaultBudget;
-    g.M = rows, g.K = static_cast<int>(h), g.n_tm = n_tm, g.n_tn = static_cast<int>(f / 128);
-    g.a_off = static_cast<int>(r0), g.b_off = 0, g.ldo = static_cast<int>(2 * f);
-    g.ldo3 = static_cast<int>(f), g.ld_in = static_cast<int>(f), g.in = dH;
-    g.out = dGU, g.out2 = dGU + f, g.out3 = H;
-    if ((r = launch_ffn_gemm<ffn::EPI_SWIGLU_BWD, false, false, false>(x_k, x_k, wg_k, wu_k, g,
-                                                                       10, st)) != LCA_OK)
-      return r;
-    // dX = dG W_gate + dU W_up
-    g = ffn::Args{};
-    g.budget = kDefaultBudget;
-    g.M = rows, g.K = static_cast<int>(2 * f), g.n_tm = n_tm, g.n_tn = static_cast<int>(h / ffn::kBN);
-    g.a_off = 0, g.b_off = 0, g.ldo = static_cast<int>(h);
-    g.out = static_cast<__nv_bfloat16*>(dx) + r0 * h;
-    if ((r = launch_ffn_gemm<ffn::EPI_STORE, false, true, true>(dg_k, du_k, wg_mn, wu_mn, g, 11,
-                                                                st)) != LCA_OK)
-      return r;
-    // [dW_gate; dW_up] += [dG | dU]^T x: one product, rows split at f
-    g = ffn::Args{};
-    g.budget = kDefaultBudget;
-    g.M = static_cast<int>(2 * f), g.K = k_rows, g.n_tm = static_cast<int>(2 * f / ffn::kBM);
-    g.n_tn = static_cast<int>(h / ffn::kBN);
-    g.a_off = 0, g.b_off = static_cast<int>(r0), g.ldo = static_cast<int>(h);
-    g.m_split = static_cast<int>(f), g.out32 = dw_gate, g.out32b = dw_up;
-    if ((r = launch_ffn_gemm<ffn::EPI_ACC32, true, true, false>(dgu_mn, dgu_mn, x_mn, x_mn, g, 12,
-                                                                st)) != LCA_OK)
-      return r;
-    // dW_down += dout^T H
-    g.M = static_cast<int>(h), g.m_split = static_cast<int>(h), g.out32b = nullptr;
-    g.n_tm = static_cast<int>(h / ffn::kBM);
-    g.n_tn = static_cast<int>(f / ffn::kBN);
-    g.a_off = static_cast<int>(r0), g.b_off = 0, g.ldo = static_cast<int>(f), g.out32 = dw_down;
-    if ((r = launch_ffn_gemm<ffn::EPI_ACC32, true, true, false>(do_mn, do_mn, h_mn, h_mn, g, 12,
-                                                                st)) != LCA_OK)
+  for (int64_t r0 = 0; r0 < shape->T; r0 += block) {
+    const int rows = static_cast<int>(shape->T - r0 < block ? shape->T - r0 : block);
+    if ((r = ffn_bwd_rows(p, r0, rows, static_cast<__nv_bfloat16*>(dx) + r0 * shape->h, st)) !=
+        LCA_OK)
       return r;
   }
   return LCA_OK;
@@ -1058,6 +1354,226 @@ lca_status lca_lse_merge(int64_t rows, int64_t d, const float* o_a, const float*
   return launched("lse_merge_kernel");
 }
 
+lca_status lca_attn_fwd_block(const lca_block_shape* shape, const void* q, const void* k,
+                              const void* v, int causal, int64_t q_pos0, int64_t k_pos0,
+                              int accumulate, float* o_acc, float* lse_acc, void* out,
+                              void* stream) {
+  Common c;
+  lca_status r = check_block(shape, &c);
+  if (r != LCA_OK) return r;
+  if ((r = check_ptrs({q, k, v, lse_acc})) != LCA_OK) return r;
+  if (!o_acc && !out) return fail(LCA_ERR_INVALID_ARG, "o_acc and out are both NULL");
+  if (accumulate && !o_acc)
+    return fail(LCA_ERR_INVALID_ARG, "accumulating needs the running o_acc");
+  if ((o_acc && !aligned16(o_acc)) || (out && !aligned16(out)))
+    return fail(LCA_ERR_INVALID_ARG, "o_acc / out not 16-byte aligned");
+  int rel, diag;
+  if ((r = block_relation(c, causal, q_pos0, k_pos0, &rel, &diag)) != LCA_OK) return r;
+  if (rel == REL_NONE && accumulate && !out) return LCA_OK;  // nothing visible to add
+  AttnSched s;
+  make_block_sched(c, rel, diag, &s);
+  FwdBlock fb;
+  fb.block = true;
+  fb.o_acc = o_acc;
+  fb.accumulate = accumulate ? 1 : 0;
+  return run_fwd(c, s, q, k, v, out, lse_acc, kDefaultBudget, static_cast<cudaStream_t>(stream),
+                 fb);
+}
+
+size_t lca_attn_bwd_block_workspace_size(const lca_block_shape* shape) {
+  Common c;
+  const std::string keep = t_last_error;
+  const bool ok = check_block(shape, &c) == LCA_OK;
+  t_last_error = keep;
+  return ok ? ws_bytes_of(c) : 0;
+}
+
+lca_status lca_attn_bwd_block_prep(const lca_block_shape* shape, const void* out,
+                                   const float* lse, const void* dout, void* workspace,
+                                   size_t ws_bytes, void* stream) {
+  Common c;
+  lca_status r = check_block(shape, &c);
+  if (r != LCA_OK) return r;
+  if ((r = check_ptrs({out, lse, dout})) != LCA_OK) return r;
+  if ((r = check_ws(c, workspace, ws_bytes)) != LCA_OK) return r;
+  return bwd_prep(c, out, lse, dout, workspace, static_cast<cudaStream_t>(stream));
+}
+
+lca_status lca_attn_bwd_block(const lca_block_shape* shape, const void* q, const void* k,
+                              const void* v, const void* dout, int causal, int64_t q_pos0,
+                              int64_t k_pos0, void* workspace, size_t ws_bytes, float* dk_acc,
+                              float* dv_acc, int accumulate_kv, void* dk, void* dv,
+                              void* stream) {
+  Common c;
+  lca_status r = check_block(shape, &c);
+  if (r != LCA_OK) return r;
+  if ((r = check_ptrs({q, k, v, dout})) != LCA_OK) return r;
+  if ((r = check_ws(c, workspace, ws_bytes)) != LCA_OK) return r;
+  const bool acc = dk_acc || dv_acc;
+  if (acc == (dk || dv))
+    return fail(LCA_ERR_INVALID_ARG, "pass either dk_acc and dv_acc or dk and dv");
+  if ((r = acc ? check_ptrs({dk_acc, dv_acc}) : check_ptrs({dk, dv})) != LCA_OK) return r;
+  int rel, diag;
+  if ((r = block_relation(c, causal, q_pos0, k_pos0, &rel, &diag)) != LCA_OK) return r;
+  // no query sees a key: nothing to add (overwriting still writes zeros)
+  if (rel == REL_NONE && acc && accumulate_kv) return LCA_OK;
+  AttnSched s;
+  make_block_sched(c, rel, diag, &s);
+  return bwd_main(c, s, q, k, v, dout, workspace, dk, dv, dk_acc, dv_acc, accumulate_kv ? 1 : 0,
+                  kDefaultBudget, static_cast<cudaStream_t>(stream));
+}
+
+lca_status lca_attn_bwd_block_dq(const lca_block_shape* shape, const void* workspace,
+                                 size_t ws_bytes, void* dq, void* stream) {
+  Common c;
+  lca_status r = check_block(shape, &c);
+  if (r != LCA_OK) return r;
+  if ((r = check_ptrs({dq})) != LCA_OK) return r;
+  if ((r = check_ws(c, workspace, ws_bytes)) != LCA_OK) return r;
+  return bwd_dq(c, workspace, dq, static_cast<cudaStream_t>(stream));
+}
+
+lca_status lca_cast_f32_bf16(int64_t n, const float* src, void* dst, void* stream) {
+  if (n <= 0) return fail(LCA_ERR_INVALID_ARG, "n must be positive");
+  lca_status r = check_ptrs({src, dst});
+  if (r != LCA_OK) return r;
+  const int64_t n8 = n / 8;
+  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((n8 + 255) / 256, 148 * 16));
+  cast_f32_bf16<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      src, static_cast<__nv_bfloat16*>(dst), n);
+  return launched("cast_f32_bf16");
+}
+
+lca_status lca_accumulate_f32(int64_t n, const float* src, float* dst, void* stream) {
+  if (n <= 0) return fail(LCA_ERR_INVALID_ARG, "n must be positive");
+  lca_status r = check_ptrs({src, dst});
+  if (r != LCA_OK) return r;
+  const int64_t n4 = n / 4;
+  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((n4 + 255) / 256, 148 * 16));
+  accumulate_f32<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      src, dst, n);
+  return launched("accumulate_f32");
+}
+
+size_t lca_bpt_fwd_workspace_size(const lca_bpt_shape* shape) {
+  BptPlan p;
+  const std::string keep = t_last_error;
+  const bool ok = check_bpt(shape, 0, &p) == LCA_OK;
+  t_last_error = keep;
+  return ok ? bpt_fwd_ws(p) : 0;
+}
+
+lca_status lca_bpt_fwd(const lca_bpt_shape* shape, const void* q, const void* k, const void* v,
+                       int causal, const void* w_gate, const void* w_up, const void* w_down,
+                       void* attn_out, float* lse, void* out, void* workspace, size_t ws_bytes,
+                       void* stream) {
+  BptPlan p;
+  lca_status r = check_bpt(shape, 0, &p);
+  if (r != LCA_OK) return r;
+  if ((r = check_ptrs({q, k, v, w_gate, w_up, w_down, attn_out, lse, out})) != LCA_OK) return r;
+  if (!workspace) return fail(LCA_ERR_WORKSPACE, "workspace is NULL");
+  if (ws_bytes < bpt_fwd_ws(p))
+    return fail(LCA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, bpt_fwd_ws(p));
+  if (!aligned16(workspace)) return fail(LCA_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* lse_blk = static_cast<float*>(workspace);
+  void* H = static_cast<char*>(workspace) + align256(static_cast<size_t>(p.attn.Hq) * p.qb * 4);
+  FfnFwdPlan fp;
+  if ((r = ffn_fwd_plan(attn_out, w_gate, w_up, w_down, p.S, p.h, p.f, p.qb, out, H, &fp)) !=
+      LCA_OK)
+    return r;
+  const size_t row_q = static_cast<size_t>(p.attn.Hq) * p.attn.d;  // elements per query row
+  for (int64_t r0 = 0; r0 < p.S; r0 += p.qb) {
+    const int rows = static_cast<int>(p.S - r0 < p.qb ? p.S - r0 : p.qb);
+    Common c;
+    AttnSched s;
+    bpt_block(p, causal, r0, rows, &c, &s);
+    FwdBlock fb;
+    fb.block = true;
+    if ((r = run_fwd(c, s, static_cast<const __nv_bfloat16*>(q) + r0 * row_q, k, v,
+                     static_cast<__nv_bfloat16*>(attn_out) + r0 * row_q, lse_blk, kDefaultBudget,
+                     st, fb)) != LCA_OK)
+      return r;
+    const cudaError_t e = cudaMemcpy2DAsync(lse + r0, p.S * sizeof(float), lse_blk,
+                                            rows * sizeof(float), rows * sizeof(float),
+                                            p.attn.Hq, cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy2DAsync(lse of a block)");
+    if ((r = ffn_fwd_rows(fp, r0, rows, st)) != LCA_OK) return r;
+  }
+  return LCA_OK;
+}
+
+size_t lca_bpt_bwd_workspace_size(const lca_bpt_shape* shape) {
+  BptPlan p;
+  const std::string keep = t_last_error;
+  const bool ok = check_bpt(shape, 1, &p) == LCA_OK;
+  t_last_error = keep;
+  return ok ? bpt_bwd_ws(p) : 0;
+}
+
+lca_status lca_bpt_bwd(const lca_bpt_shape* shape, const void* q, const void* k, const void* v,
+                       int causal, const void* w_gate, const void* w_up, const void* w_down,
+                       const void* attn_out, const float* lse, const void* dout, void* dq,
+                       void* dk, void* dv, float* dw_gate, float* dw_up, float* dw_down,
+                       void* workspace, size_t ws_bytes, void* stream) {
+  BptPlan p;
+  lca_status r = check_bpt(shape, 1, &p);
+  if (r != LCA_OK) return r;
+  if ((r = check_ptrs({q, k, v, w_gate, w_up, w_down, attn_out, lse, dout, dq, dk, dv, dw_gate,
+                       dw_up, dw_down})) != LCA_OK)
+    return r;
+  if (!workspace) return fail(LCA_ERR_WORKSPACE, "workspace is NULL");
+  if (ws_bytes < bpt_bwd_ws(p))
+    return fail(LCA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, bpt_bwd_ws(p));
+  if (!aligned16(workspace)) return fail(LCA_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(workspace);
+  void* ffn_ws = w;
+  w += 4 * static_cast<size_t>(p.qb) * p.f * 2;
+  auto* dx_blk = reinterpret_cast<__nv_bfloat16*>(w);
+  w += align256(static_cast<size_t>(p.qb) * p.h * 2);
+  void* attn_ws = w;
+  w += align256(ws_bytes_of(p.attn));
+  float* lse_blk = reinterpret_cast<float*>(w);
+  w += align256(static_cast<size_t>(p.attn.Hq) * p.qb * 4);
+  const size_t kv_elems = static_cast<size_t>(p.S) * p.attn.Hkv * p.attn.d;
+  float* dk_acc = reinterpret_cast<float*>(w);
+  w += align256(kv_elems * 4);
+  float* dv_acc = reinterpret_cast<float*>(w);
+  cudaError_t e = cudaMemsetAsync(dk_acc, 0, kv_elems * 4, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(dv_acc, 0, kv_elems * 4, st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(dk/dv accumulators)");
+  FfnBwdPlan fp;
+  if ((r = ffn_bwd_plan(attn_out, w_gate, w_up, w_down, dout, p.S, p.h, p.f, p.qb, dw_gate,
+                        dw_up, dw_down, ffn_ws, &fp)) != LCA_OK)
+    return r;
+  const size_t row_q = static_cast<size_t>(p.attn.Hq) * p.attn.d;
+  for (int64_t r0 = 0; r0 < p.S; r0 += p.qb) {
+    const int rows = static_cast<int>(p.S - r0 < p.qb ? p.S - r0 : p.qb);
+    // feedforward backward of the block: its weight gradients, and the
+    // gradient of its input rows (the attention output) into dx_blk
+    if ((r = ffn_bwd_rows(fp, r0, rows, dx_blk, st)) != LCA_OK) return r;
+    // attention backward of the block's query rows with that gradient
+    Common c;
+    AttnSched s;
+    bpt_block(p, causal, r0, rows, &c, &s);
+    e = cudaMemcpy2DAsync(lse_blk, rows * sizeof(float), lse + r0, p.S * sizeof(float),
+                          rows * sizeof(float), p.attn.Hq, cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy2DAsync(lse of a block)");
+    const auto* o_rows = static_cast<const __nv_bfloat16*>(attn_out) + r0 * row_q;
+    if ((r = bwd_prep(c, o_rows, lse_blk, dx_blk, attn_ws, st)) != LCA_OK) return r;
+    if ((r = bwd_main(c, s, static_cast<const __nv_bfloat16*>(q) + r0 * row_q, k, v, dx_blk,
+                      attn_ws, nullptr, nullptr, dk_acc, dv_acc, 1, kDefaultBudget, st)) !=
+        LCA_OK)
+      return r;
+    if ((r = bwd_dq(c, attn_ws, static_cast<__nv_bfloat16*>(dq) + r0 * row_q, st)) != LCA_OK)
+      return r;
+  }
+  if ((r = lca_cast_f32_bf16(static_cast<int64_t>(kv_elems), dk_acc, dk, stream)) != LCA_OK)
+    return r;
+  return lca_cast_f32_bf16(static_cast<int64_t>(kv_elems), dv_acc, dv, stream);
+}
+
 lca_status lca_check(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
@@ -1067,7 +1583,13 @@ lca_status lca_check(void* stream) {
   if (h[0]) {
     const int z[2] = {0, 0};
     cudaMemcpyToSymbol(g_err, z, sizeof z);
-    if (h[0] & kErrTimeout) return fail(LCA_ERR_TIMEOUT, "a kernel wait ran out (site %d)", h[1]);
+    if (h[0] & kErrTimeout)
+      return fail(LCA_ERR_TIMEOUT, "a kernel wait ran out (site %d)%s", h[1],
+                  (h[0] & kErrDrain) ? "; a CTA then gave up waiting for its work in flight"
+                                     : "");
+    if (h[0] & kErrDrain)
+      return fail(LCA_ERR_TIMEOUT,
+                  "a CTA gave up waiting for its own copies or MMAs in flight (site %d)", h[1]);
     if (h[0] & kErrSeqOffsets)
       return fail(LCA_ERR_INVALID_ARG,
                   "cu_seqlens out of order or range, or a sequence longer than max_seqlen "

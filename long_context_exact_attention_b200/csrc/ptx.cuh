@@ -14,11 +14,12 @@ namespace lca {
 
 // Device error word: [0] = error bits (1 = a wait timed out, 2 = a kernel
 // could not align its shared-memory layout, 4 = packed sequence offsets out
-// of order or out of range), [1] = site id of the first error.  Read and
+// of order or out of range, 8 = an unwinding CTA gave up waiting for its own
+// copies or MMAs in flight), [1] = site id of the first error.  Read and
 // cleared by lca_check().  The library is one translation unit, so the
 // definition lives here.
 __device__ int g_err[2];
-constexpr int kErrTimeout = 1, kErrSmemAlign = 2, kErrSeqOffsets = 4;
+constexpr int kErrTimeout = 1, kErrSmemAlign = 2, kErrSeqOffsets = 4, kErrDrain = 8;
 
 __device__ __forceinline__ void record_error(int bit, int site) {
   atomicOr(&g_err[0], bit);
@@ -78,15 +79,20 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Wa
   }
 }
 
-// Bounded wait used while unwinding after an abort: ignores the abort flag
-// (the point is to let in-flight copies / MMAs land) and gives up silently
-// after a fixed budget of 2^31 clocks, whatever budget the caller chose for
-// ordinary waits.
-__device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity, unsigned long long) {
+// Bounded wait used while unwinding after an abort, and before TMEM is
+// freed: ignores the abort flag (the point is to let in-flight copies / MMAs
+// land) and gives up after a fixed budget of 2^31 clocks, whatever budget
+// the caller chose for ordinary waits.  Giving up is recorded as its own
+// error bit (kErrDrain) with `site`, so lca_check() reports that the CTA may
+// have exited with work still in flight.
+__device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity, int site) {
   const unsigned long long budget = 1ull << 31;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (static_cast<unsigned long long>(clock64() - t0) > budget) return;
+    if (static_cast<unsigned long long>(clock64() - t0) > budget) {
+      record_error(kErrDrain, site);
+      return;
+    }
   }
 }
 

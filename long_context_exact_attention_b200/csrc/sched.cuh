@@ -13,6 +13,15 @@
 // counted from its first token.  When a sequence's length is not a multiple
 // of the tile its last tile is partial.
 //
+// Blocks.  A sequence-parallel caller attends a block of queries to a block
+// of keys that starts elsewhere on the position axis (Ring Attention with
+// Blockwise Transformers, Summary: each host keeps its query block and sees
+// the key/value blocks of the others in turn).  Then the key block has its
+// own length S_kv and the causal diagonal is shifted: key tile T is on the
+// diagonal of query tile Q when T == Q + diag (diag = (query position -
+// key position of the blocks' first rows) / tile), visible in full before
+// it and invisible after it.  Ordinary calls have S_kv == S and diag == 0.
+//
 // Chunk order (Ring Attention with Blockwise Transformers, Summary: a query
 // block meets the key/value blocks in the order the ring delivers them, and
 // the result does not depend on it).  Keys are split into chunks of
@@ -33,6 +42,9 @@ namespace lca {
 struct AttnSched {
   int S;                   // longest sequence in tokens (every sequence when not packed)
   int n_tiles;             // ceil(S / tile)
+  int S_kv;                // keys of a dense sequence (== S except for block calls)
+  int n_kv_tiles;          // ceil(S_kv / tile)
+  int diag;                // causal: key tile Q + diag is the diagonal of query tile Q
   int tile;                // tokens per tile
   int causal;
   int s2;                  // 1: S2-Attn walk
@@ -58,11 +70,14 @@ __host__ __device__ inline int token_tile(const AttnSched& s, int t, bool shifte
 
 // Where sequence b lives in the tensors: tensor coordinates (batch index bm,
 // first token tokb), its first row on the flattened token axis of all batch
-// entries (row0 = bm * S_tensor + tokb) and its length.  S_tensor is the
-// token extent of one batch entry of the tensors (the packed length for
-// packed sequences).
+// entries (row0 = bm * S_tensor + tokb) and its length; the same for its
+// keys (kv_row0, kv_len), which differ only for block calls.  S_tensor is
+// the token extent of one batch entry of the query tensors (the packed
+// length for packed sequences); a dense key tensor holds S_kv tokens per
+// batch entry.
 struct SeqView {
   int bm, tokb, row0, len, n_tiles;
+  int kv_row0, kv_len, kv_n_tiles;
 };
 
 // False when packed offsets are out of order or out of range (the caller
@@ -74,6 +89,9 @@ __host__ __device__ inline bool seq_view(const AttnSched& s, int b, int S_tensor
     v->row0 = b * S_tensor;
     v->len = s.S;
     v->n_tiles = s.n_tiles;
+    v->kv_row0 = b * s.S_kv;
+    v->kv_len = s.S_kv;
+    v->kv_n_tiles = s.n_kv_tiles;
     return true;
   }
   const int c0 = s.cu_seqlens[b], c1 = s.cu_seqlens[b + 1];
@@ -83,11 +101,14 @@ __host__ __device__ inline bool seq_view(const AttnSched& s, int b, int S_tensor
   v->row0 = c0;
   v->len = c1 - c0;
   v->n_tiles = (v->len + s.tile - 1) / s.tile;
+  v->kv_row0 = v->row0;
+  v->kv_len = v->len;
+  v->kv_n_tiles = v->n_tiles;
   return true;
 }
 
 // Walk of the key/value position tiles for query position tile qt of a
-// sequence of `len` tokens.
+// sequence whose keys number `len`.
 struct KvWalk {
   const AttnSched* s;
   int qt, len, n_chunks, key_end;
@@ -107,7 +128,8 @@ struct KvWalk {
       n_chunks = (len + s->kv_chunk - 1) / s->kv_chunk;
       // keys past the query tile's last row are invisible under the mask
       key_end = len;
-      if (s->causal && (qt + 1) * s->tile < key_end) key_end = (qt + 1) * s->tile;
+      if (s->causal && (qt + 1 + s->diag) * s->tile < key_end)
+        key_end = (qt + 1 + s->diag) * s->tile;
       qb = qt * s->tile / s->q_block;
     }
   }
@@ -196,7 +218,7 @@ struct TileWalk {
       t = c * tpc;
       t_end = t + tpc;
       if (t_end > n_tiles) t_end = n_tiles;
-      if (s->causal && t_end > qt + 1) t_end = qt + 1;
+      if (s->causal && t_end > qt + 1 + s->diag) t_end = qt + 1 + s->diag;
     }
     tile = t++;
     return true;
@@ -204,8 +226,8 @@ struct TileWalk {
 };
 
 // Query position tiles whose walk contains key position tile kt, for a
-// sequence of n_tiles tiles (the backward pass loops over queries for a
-// fixed key tile).
+// sequence of n_tiles query tiles (the backward pass loops over queries for
+// a fixed key tile).
 struct QWalk {
   int t, t_end;
   __host__ __device__ void init(const AttnSched* s, int kt, int n_tiles) {
@@ -214,7 +236,7 @@ struct QWalk {
       t = s->causal ? kt : g0;
       t_end = g0 + s->group_tiles;
     } else {
-      t = s->causal ? kt : 0;
+      t = (s->causal && kt - s->diag > 0) ? kt - s->diag : 0;
       t_end = n_tiles;
     }
   }

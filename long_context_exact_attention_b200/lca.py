@@ -25,8 +25,12 @@ SYMBOLS = ["lca_attn_fwd", "lca_attn_bwd_workspace_size", "lca_attn_bwd",
            "lca_attn_fwd_varlen", "lca_attn_bwd_varlen_workspace_size", "lca_attn_bwd_varlen",
            "lca_ffn_workspace_size", "lca_ffn_fwd", "lca_ffn_bwd_workspace_size", "lca_ffn_bwd",
            "lca_s2attn_fwd", "lca_s2attn_fwd_ws", "lca_s2attn_fwd_workspace_size",
-           "lca_s2attn_bwd", "lca_s2attn_bwd_workspace_size", "lca_lse_merge", "lca_check",
-           "lca_status_string", "lca_last_error", "lca_version"]
+           "lca_s2attn_bwd", "lca_s2attn_bwd_workspace_size", "lca_lse_merge",
+           "lca_attn_fwd_block", "lca_attn_bwd_block_workspace_size", "lca_attn_bwd_block_prep",
+           "lca_attn_bwd_block", "lca_attn_bwd_block_dq", "lca_cast_f32_bf16",
+           "lca_accumulate_f32", "lca_bpt_fwd_workspace_size", "lca_bpt_fwd",
+           "lca_bpt_bwd_workspace_size", "lca_bpt_bwd", "lca_check", "lca_status_string",
+           "lca_last_error", "lca_version"]
 
 
 class LcaError(RuntimeError):
@@ -38,6 +42,18 @@ class LcaError(RuntimeError):
 class Shape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int64), ("Hq", ctypes.c_int64), ("Hkv", ctypes.c_int64),
                 ("S", ctypes.c_int64), ("d", ctypes.c_int64), ("dtype", ctypes.c_int32),
+                ("scale", ctypes.c_float)]
+
+
+class BlockShape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int64), ("Hq", ctypes.c_int64), ("Hkv", ctypes.c_int64),
+                ("Sq", ctypes.c_int64), ("Sk", ctypes.c_int64), ("d", ctypes.c_int64),
+                ("dtype", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
+class BptShape(ctypes.Structure):
+    _fields_ = [("S", ctypes.c_int64), ("Hq", ctypes.c_int64), ("Hkv", ctypes.c_int64),
+                ("d", ctypes.c_int64), ("f", ctypes.c_int64), ("q_block", ctypes.c_int64),
                 ("scale", ctypes.c_float)]
 
 
@@ -83,6 +99,23 @@ def lib() -> ctypes.CDLL:
         L.lca_s2attn_bwd.argtypes = [SP, P, P, P, P, P, P, I32, I64, I64, P, P, P, P,
                                      ctypes.c_size_t, P]
         L.lca_lse_merge.argtypes = [I64, I64, P, P, P, P, P, P, P]
+        BP = ctypes.POINTER(BlockShape)
+        L.lca_attn_fwd_block.argtypes = [BP, P, P, P, I32, I64, I64, I32, P, P, P, P]
+        L.lca_attn_bwd_block_workspace_size.argtypes = [BP]
+        L.lca_attn_bwd_block_workspace_size.restype = ctypes.c_size_t
+        L.lca_attn_bwd_block_prep.argtypes = [BP, P, P, P, P, ctypes.c_size_t, P]
+        L.lca_attn_bwd_block.argtypes = [BP, P, P, P, P, I32, I64, I64, P, ctypes.c_size_t, P,
+                                         P, I32, P, P, P]
+        L.lca_attn_bwd_block_dq.argtypes = [BP, P, ctypes.c_size_t, P, P]
+        L.lca_cast_f32_bf16.argtypes = [I64, P, P, P]
+        L.lca_accumulate_f32.argtypes = [I64, P, P, P]
+        TP = ctypes.POINTER(BptShape)
+        for fn in ("lca_bpt_fwd_workspace_size", "lca_bpt_bwd_workspace_size"):
+            getattr(L, fn).argtypes = [TP]
+            getattr(L, fn).restype = ctypes.c_size_t
+        L.lca_bpt_fwd.argtypes = [TP, P, P, P, I32, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+        L.lca_bpt_bwd.argtypes = [TP, P, P, P, I32, P, P, P, P, P, P, P, P, P, P, P, P, P,
+                                  ctypes.c_size_t, P]
         FP = ctypes.POINTER(FfnShape)
         L.lca_ffn_workspace_size.argtypes = [FP, I64]
         L.lca_ffn_workspace_size.restype = ctypes.c_size_t
@@ -96,7 +129,9 @@ def lib() -> ctypes.CDLL:
         for fn in ("lca_attn_fwd", "lca_attn_bwd", "lca_attn_bwd_noalloc", "lca_s2attn_fwd",
                    "lca_s2attn_fwd_ws",
                    "lca_s2attn_bwd", "lca_attn_fwd_varlen", "lca_attn_bwd_varlen", "lca_ffn_fwd", "lca_ffn_bwd",
-                   "lca_lse_merge", "lca_check"):
+                   "lca_lse_merge", "lca_attn_fwd_block", "lca_attn_bwd_block_prep",
+                   "lca_attn_bwd_block", "lca_attn_bwd_block_dq", "lca_cast_f32_bf16",
+                   "lca_accumulate_f32", "lca_bpt_fwd", "lca_bpt_bwd", "lca_check"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -395,6 +430,168 @@ def lse_merge(o_a, lse_a, o_b, lse_b, o_out=None, lse_out=None, stream=None):
     _raise(lib().lca_lse_merge(rows, d, _ptr(o_a), _ptr(lse_a), _ptr(o_b), _ptr(lse_b),
                                _ptr(o_out), _ptr(lse_out), _stream(stream)))
     return o_out, lse_out
+
+
+# ---------------------------------------------------------------- blocks
+
+def _block_shape(q, k, scale) -> BlockShape:
+    """q [B,Sq,Hq,d] (bf16), k/v [B,Sk,Hkv,d]."""
+    if not (q.is_cuda and k.is_cuda):
+        raise ValueError("lca needs CUDA tensors")
+    if q.dim() != 4 or k.dim() != 4 or k.shape[0] != q.shape[0] or k.shape[3] != q.shape[3]:
+        raise ValueError("q is [B,Sq,Hq,d], k/v are [B,Sk,Hkv,d]")
+    if q.dtype != torch.bfloat16:
+        raise ValueError("block calls take bf16 tensors")
+    B, Sq, Hq, d = q.shape
+    return BlockShape(B, Hq, k.shape[2], Sq, k.shape[1], d, LCA_BF16, float(scale or 0.0))
+
+
+def attn_fwd_block(q, k, v, q_pos0: int, k_pos0: int, causal: bool = True,
+                   accumulate: bool = False, o_acc=None, lse_acc=None, out=None, scale=None,
+                   stream=None):
+    """One ring step of the forward (lca_attn_fwd_block): attend the query
+    block (rows at positions q_pos0...) to the key/value block (keys at
+    k_pos0...) and fold the result into the running float32 (o_acc, lse_acc)
+    (or start it when accumulate is False).  out, when given, receives the
+    merged output as bf16.  Returns (o_acc, lse_acc, out)."""
+    sh = _block_shape(q, k, scale)
+    _check_tensors(torch.bfloat16, q, k, v)
+    B, Sq, Hq, d = q.shape
+    if o_acc is None:
+        o_acc = torch.empty((B, Sq, Hq, d), device=q.device, dtype=torch.float32)
+    if lse_acc is None:
+        lse_acc = torch.empty((B, Hq, Sq), device=q.device, dtype=torch.float32)
+    _check_tensors(torch.float32, o_acc, lse_acc)
+    _raise(lib().lca_attn_fwd_block(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), int(causal),
+                                    int(q_pos0), int(k_pos0), int(bool(accumulate)), _ptr(o_acc),
+                                    _ptr(lse_acc), _ptr(out), _stream(stream)))
+    return o_acc, lse_acc, out
+
+
+def bwd_block_workspace_size(q, k) -> int:
+    sh = _block_shape(q, k, None)
+    return int(lib().lca_attn_bwd_block_workspace_size(ctypes.byref(sh)))
+
+
+def attn_bwd_block_prep(q, out, lse, dout, workspace=None, scale=None, stream=None):
+    """Start a query block's backward (lca_attn_bwd_block_prep) from its
+    final out and lse.  Returns the workspace (allocated when not given)."""
+    sh = _block_shape(q, q, scale)
+    _check_tensors(torch.bfloat16, out, dout)
+    if workspace is None:
+        workspace = torch.empty(bwd_block_workspace_size(q, q), device=q.device,
+                                dtype=torch.uint8)
+    _raise(lib().lca_attn_bwd_block_prep(ctypes.byref(sh), _ptr(out), _ptr(lse), _ptr(dout),
+                                         _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(),
+                                         _stream(stream)))
+    return workspace
+
+
+def attn_bwd_block(q, k, v, dout, q_pos0: int, k_pos0: int, workspace, causal: bool = True,
+                   dk_acc=None, dv_acc=None, accumulate_kv: bool = True, dk=None, dv=None,
+                   scale=None, stream=None):
+    """One ring step of the backward (lca_attn_bwd_block): dQ into the
+    workspace, dK/dV into the float32 accumulators dk_acc/dv_acc (added when
+    accumulate_kv, else overwritten) or, when those are None, into bf16
+    dk/dv (overwritten).  Returns (dk_acc, dv_acc) or (dk, dv)."""
+    sh = _block_shape(q, k, scale)
+    _check_tensors(torch.bfloat16, q, k, v, dout)
+    if dk_acc is None and dk is None:
+        dk, dv = torch.empty_like(k), torch.empty_like(v)
+    _raise(lib().lca_attn_bwd_block(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(dout),
+                                    int(causal), int(q_pos0), int(k_pos0), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _ptr(dk_acc),
+                                    _ptr(dv_acc), int(bool(accumulate_kv)), _ptr(dk), _ptr(dv),
+                                    _stream(stream)))
+    return (dk_acc, dv_acc) if dk_acc is not None else (dk, dv)
+
+
+def attn_bwd_block_dq(q, workspace, dq=None, scale=None, stream=None):
+    """Finish a query block's backward (lca_attn_bwd_block_dq).  Returns dq."""
+    sh = _block_shape(q, q, scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    _raise(lib().lca_attn_bwd_block_dq(ctypes.byref(sh), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(), _ptr(dq),
+                                       _stream(stream)))
+    return dq
+
+
+def cast_bf16(src, dst=None, stream=None):
+    """dst = bf16(src) for a contiguous float32 CUDA tensor (lca_cast_f32_bf16)."""
+    _check_tensors(torch.float32, src)
+    dst = torch.empty(src.shape, device=src.device, dtype=torch.bfloat16) if dst is None else dst
+    _check_tensors(torch.bfloat16, dst)
+    _raise(lib().lca_cast_f32_bf16(src.numel(), _ptr(src), _ptr(dst), _stream(stream)))
+    return dst
+
+
+def accumulate(src, dst, stream=None):
+    """dst += src for contiguous float32 CUDA tensors (lca_accumulate_f32)."""
+    _check_tensors(torch.float32, src, dst)
+    if src.numel() != dst.numel():
+        raise ValueError("accumulate: sizes differ")
+    _raise(lib().lca_accumulate_f32(src.numel(), _ptr(src), _ptr(dst), _stream(stream)))
+    return dst
+
+
+# ---------------------------------------------------------------- blockwise transformer
+
+def _bpt_shape(q, k, w_gate, q_block, scale) -> BptShape:
+    """q [S, Hq, d], k/v [S, Hkv, d] (one sequence), w_gate [f, Hq*d]."""
+    if q.dim() != 3 or k.dim() != 3 or k.shape[0] != q.shape[0] or k.shape[2] != q.shape[2]:
+        raise ValueError("q is [S,Hq,d], k/v are [S,Hkv,d]")
+    S, Hq, d = q.shape
+    if w_gate.dim() != 2 or w_gate.shape[1] != Hq * d:
+        raise ValueError("w_gate is [f, Hq*d]")
+    return BptShape(S, Hq, k.shape[1], d, w_gate.shape[0], int(q_block), float(scale or 0.0))
+
+
+def bpt_fwd(q, k, v, w_gate, w_up, w_down, causal: bool = True, q_block: int = 0, scale=None,
+            attn_out=None, lse=None, out=None, workspace=None, stream=None):
+    """Blockwise Transformer sweep (lca_bpt_fwd): per block of q_block query
+    rows, attention over the keys they see, then the gated-SiLU feedforward
+    of those rows.  Returns (attn_out [S,Hq,d], lse [Hq,S], out [S,Hq*d])."""
+    _check_tensors(torch.bfloat16, q, k, v, w_gate, w_up, w_down)
+    sh = _bpt_shape(q, k, w_gate, q_block, scale)
+    S, Hq, d = q.shape
+    attn_out = torch.empty_like(q) if attn_out is None else attn_out
+    lse = torch.empty((Hq, S), device=q.device, dtype=torch.float32) if lse is None else lse
+    out = torch.empty((S, Hq * d), device=q.device, dtype=torch.bfloat16) if out is None else out
+    if workspace is None:
+        n = int(lib().lca_bpt_fwd_workspace_size(ctypes.byref(sh)))
+        workspace = torch.empty(max(n, 16), device=q.device, dtype=torch.uint8)
+    _raise(lib().lca_bpt_fwd(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), int(causal),
+                             _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(attn_out), _ptr(lse),
+                             _ptr(out), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream(stream)))
+    return attn_out, lse, out
+
+
+def bpt_bwd(q, k, v, w_gate, w_up, w_down, attn_out, lse, dout, causal: bool = True,
+            q_block: int = 0, scale=None, dq=None, dk=None, dv=None, dw_gate=None, dw_up=None,
+            dw_down=None, workspace=None, stream=None):
+    """Gradients of the sweep (lca_bpt_bwd).  dw_* are float32 and the
+    gradients are added to them (new zero tensors when not given).  Returns
+    (dq, dk, dv, dw_gate, dw_up, dw_down)."""
+    _check_tensors(torch.bfloat16, q, k, v, w_gate, w_up, w_down, attn_out, dout)
+    sh = _bpt_shape(q, k, w_gate, q_block, scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    z = lambda t: torch.zeros(t.shape, device=t.device, dtype=torch.float32)
+    dw_gate = z(w_gate) if dw_gate is None else dw_gate
+    dw_up = z(w_up) if dw_up is None else dw_up
+    dw_down = z(w_down) if dw_down is None else dw_down
+    if workspace is None:
+        n = int(lib().lca_bpt_bwd_workspace_size(ctypes.byref(sh)))
+        workspace = torch.empty(max(n, 16), device=q.device, dtype=torch.uint8)
+    _raise(lib().lca_bpt_bwd(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), int(causal),
+                             _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(attn_out), _ptr(lse),
+                             _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dw_gate),
+                             _ptr(dw_up), _ptr(dw_down), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream(stream)))
+    return dq, dk, dv, dw_gate, dw_up, dw_down
 
 
 def check(stream=None):

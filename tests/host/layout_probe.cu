@@ -1,7 +1,7 @@
 // Host-side probe of index logic the kernels share with the host: the
 // feedforward tile raster (ffn_sm100.cuh) and the packed-sequence view
 // (sched.cuh).  Built and run by tests/test_layout_host.py.
-//   layout_probe tiles n_tm n_tn        -> "t tm tn" per tile
+//   layout_probe tiles n_tm n_tn group_m -> "t tm tn" per tile
 //   layout_probe seq S_max tile S_tensor cu0 cu1 ...  -> "b ok tokb len n_tiles"
 //   layout_probe s2 S half H first_shifted -> "h p token" per head and position
 #include <cstdio>
@@ -18,10 +18,10 @@
 int main(int argc, char** argv) {
   if (argc < 2) return 2;
   if (!strcmp(argv[1], "tiles")) {
-    const int n_tm = atoi(argv[2]), n_tn = atoi(argv[3]);
+    const int n_tm = atoi(argv[2]), n_tn = atoi(argv[3]), group_m = atoi(argv[4]);
     for (int t = 0; t < n_tm * n_tn; ++t) {
       int tm, tn;
-      lca::ffn::tile_coords(t, n_tm, n_tn, tm, tn);
+      lca::ffn::tile_coords(t, n_tm, n_tn, group_m, tm, tn);
       printf("%d %d %d\n", t, tm, tn);
     }
     return 0;

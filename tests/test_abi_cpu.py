@@ -219,3 +219,74 @@ def test_python_binding_refuses_cpu_tensors():
     q = torch.zeros(1, 128, 1, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         lca.attn_fwd(q, q, q)
+
+
+# ---------------------------------------------------------------- blocks
+
+def bshape(**kw):
+    base = dict(B=1, Hq=4, Hkv=2, Sq=256, Sk=256, d=128, dtype=lca.LCA_BF16, scale=0.0)
+    base.update(kw)
+    return lca.BlockShape(base["B"], base["Hq"], base["Hkv"], base["Sq"], base["Sk"], base["d"],
+                          base["dtype"], base["scale"])
+
+
+def fwd_block(sh, causal=1, q_pos0=0, k_pos0=0, accumulate=0, o_acc=FAKE, lse=FAKE, out=FAKE):
+    return lca.lib().lca_attn_fwd_block(ctypes.byref(sh), FAKE, FAKE, FAKE, causal, q_pos0,
+                                        k_pos0, accumulate, o_acc, lse, out, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Sk=0), 1), (dict(Sq=0), 1), (dict(dtype=lca.LCA_FP32, d=64), 2), (dict(d=64), 2),
+    (dict(Hq=3, Hkv=2), 1),
+])
+def test_block_shapes_rejected(kw, code):
+    assert fwd_block(bshape(**kw)) == code
+
+
+def test_block_positions_and_outputs_rejected():
+    sh = bshape()
+    assert fwd_block(sh, q_pos0=-1) == 1
+    # the diagonal crosses the blocks 100 positions apart: not a whole tile
+    assert fwd_block(sh, q_pos0=100, k_pos0=0) == 1
+    assert b"multiple of 128" in lca.lib().lca_last_error()
+    assert fwd_block(sh, o_acc=None, out=None) == 1
+    assert fwd_block(sh, accumulate=1, o_acc=None) == 1
+    assert fwd_block(sh, lse=None) == 1
+
+
+def test_bwd_block_needs_exactly_one_output_pair():
+    sh = bshape()
+    n = lca.lib().lca_attn_bwd_block_workspace_size(ctypes.byref(sh))
+    assert n > 0
+    call = lambda dka, dva, dk, dv: lca.lib().lca_attn_bwd_block(
+        ctypes.byref(sh), FAKE, FAKE, FAKE, FAKE, 1, 0, 0, FAKE, n, dka, dva, 1, dk, dv, None)
+    assert call(None, None, None, None) == 1
+    assert call(FAKE, FAKE, FAKE, FAKE) == 1
+    assert lca.lib().lca_attn_bwd_block(ctypes.byref(sh), FAKE, FAKE, FAKE, FAKE, 1, 0, 0, FAKE,
+                                        n - 16, FAKE, FAKE, 1, None, None, None) == 5
+
+
+def test_finishing_ops_rejected():
+    L = lca.lib()
+    assert L.lca_cast_f32_bf16(0, FAKE, FAKE, None) == 1
+    assert L.lca_cast_f32_bf16(8, FAKE, MISALIGNED, None) == 1
+    assert L.lca_accumulate_f32(-1, FAKE, FAKE, None) == 1
+    assert L.lca_accumulate_f32(8, None, FAKE, None) == 1
+
+
+def test_bpt_arguments_rejected():
+    L = lca.lib()
+    def mk(**kw):
+        base = dict(S=1024, Hq=4, Hkv=2, d=128, f=768, q_block=256, scale=0.0)
+        base.update(kw)
+        return lca.BptShape(*(base[n] for n in ("S", "Hq", "Hkv", "d", "f", "q_block", "scale")))
+
+    ok = mk()
+    assert L.lca_bpt_fwd_workspace_size(ctypes.byref(ok)) > 0
+    assert L.lca_bpt_bwd_workspace_size(ctypes.byref(ok)) > 0
+    assert L.lca_bpt_fwd_workspace_size(ctypes.byref(mk(q_block=100))) == 0
+    assert L.lca_bpt_fwd_workspace_size(ctypes.byref(mk(Hq=3, Hkv=3))) == 0   # h % 256
+    assert L.lca_bpt_bwd_workspace_size(ctypes.byref(mk(f=640))) == 0         # f % 256
+    args = [FAKE] * 3 + [1] + [FAKE] * 6
+    assert L.lca_bpt_fwd(ctypes.byref(mk(q_block=100)), *args, FAKE, 1 << 30, None) == 1
+    assert L.lca_bpt_fwd(ctypes.byref(ok), *args, None, 0, None) == 5

@@ -28,22 +28,56 @@ def sample_rows(S, chunk, n_random, seed):
     return np.array(sorted(rows))
 
 
-def check_rows(x, out, lse, w, heads, rows):
-    """Exact oracle rows vs GPU rows for the given heads."""
-    outs, refs = [], []
+_KV_CACHE = {}
+
+
+def _kv_host(x, g):
+    """Host float64 copies of key/value head g (kept for the heads that
+    share it; one entry at a time bounds host memory)."""
+    key = (id(x["k"]), g)
+    if key not in _KV_CACHE:
+        _KV_CACHE.clear()
+        _KV_CACHE[key] = (host(x["k"][:, :, g:g + 1]), host(x["v"][:, :, g:g + 1]))
+    return _KV_CACHE[key]
+
+
+def oracle_rows(x, w, h, rows, row_chunk=256):
+    """The oracle's exact (out, lse) of the given query rows of head h, in
+    chunks of rows to bound host memory at long sequence lengths."""
+    g = h // (w.Hq // w.Hkv)
+    kh, vh = _kv_host(x, g)
+    outs, lses = [], []
+    for i in range(0, len(rows), row_chunk):
+        # q stays on the device (the oracle gathers just the sampled rows)
+        ro, rl = oracle.attention_rows(x["q"][:, :, h:h + 1], kh, vh, w.causal, 0, 0,
+                                       rows[i:i + row_chunk])
+        outs.append(ro)
+        lses.append(rl)
+    return np.concatenate(outs), np.concatenate(lses)
+
+
+def check_rows(x, outs_lses, w, heads, rows):
+    """Exact oracle rows vs GPU rows for the given heads; outs_lses is a list
+    of (out, lse) results of the same inputs (e.g. two chunk orders), each
+    compared with the same oracle rows."""
+    idx = torch.as_tensor(rows, device=outs_lses[0][0].device)
+    got = [[] for _ in outs_lses]
+    refs = []
     for h in heads:
-        g = h // (w.Hq // w.Hkv)
-        ro, rl = oracle.attention_rows(x["q"][:, :, h:h + 1], x["k"][:, :, g:g + 1],
-                                       x["v"][:, :, g:g + 1], w.causal, 0, 0, rows)
-        idx = torch.as_tensor(rows, device=out.device)
-        go = host(out[0, idx, h])
-        gl = host(lse[0, h, idx])
-        assert max_abs(go, ro) <= BF16_OUT_ABS, (h, max_abs(go, ro))
-        assert max_abs(gl, rl) <= BF16_LSE_ABS, (h, max_abs(gl, rl))
-        outs.append(go)
+        ro, rl = oracle_rows(x, w, h, rows)
         refs.append(ro)
-    r = rel_fro(np.stack(outs), np.stack(refs))
-    assert r <= BF16_OUT_REL, r
+        for i, (out, lse) in enumerate(outs_lses):
+            go = host(out[0, idx, h])
+            gl = host(lse[0, h, idx])
+            assert max_abs(go, ro) <= BF16_OUT_ABS, (i, h, max_abs(go, ro))
+            assert max_abs(gl, rl) <= BF16_LSE_ABS, (i, h, max_abs(gl, rl))
+            # the stricter per-head relative bound (the absolute one is loose
+            # once |O| is small at long sequence lengths)
+            assert rel_fro(go, ro) <= BF16_OUT_REL, (i, h, rel_fro(go, ro))
+            got[i].append(go)
+    for g_ in got:
+        r = rel_fro(np.stack(g_), np.stack(refs))
+        assert r <= BF16_OUT_REL, r
 
 
 def test_llama2_7b_s32k_ring_fwd_bwd():
@@ -65,7 +99,7 @@ def test_llama2_7b_s32k_ring_fwd_bwd():
         assert_grads_close([host(dq[:, :, sl]), host(dk[:, :, sl]), host(dv[:, :, sl])], rg)
     # sampled rows in every head
     rows = sample_rows(w.S, w.kv_chunk, 8, 1)
-    check_rows(x, out, lse, w, range(w.Hq), rows)
+    check_rows(x, [(out, lse)], w, range(w.Hq), rows)
 
 
 def test_longlora_s2_s8k_fwd_bwd():
@@ -93,26 +127,31 @@ def test_llama3_8b_gqa_s128k_fwd_bwd_permuted():
     # order-permuted run matches the in-order run (float32 rounding only)
     assert max_abs(host(lse_p), host(lse)) <= 1e-4
     assert (out_p.float() - out.float()).abs().max().item() <= 4e-3
-    rows = sample_rows(w.S, w.kv_chunk, 32, 3)
-    check_rows(x, out, lse, w, (0, 7, 20, 31), rows)
-    check_rows(x, out_p, lse_p, w, (3, 28), rows)
+    # 256 exact rows (first and last of every chunk, the rest drawn with the
+    # workload's seed) in every one of the 32 query heads, for both orders
+    rows = sample_rows(w.S, w.kv_chunk, 256 - 2 * n, 3)
+    check_rows(x, [(out, lse), (out_p, lse_p)], w, range(w.Hq), rows)
 
     dq, dk, dv = lca.attn_bwd(x["q"], x["k"], x["v"], out, lse, x["dout"], causal=True)
     torch.cuda.synchronize()
     lca.check()
     rep = w.Hq // w.Hkv
-    for g in (0, 5):
-        # dQ on sampled rows, exact per row
+    idx = torch.as_tensor(rows, device="cuda")
+    for g in range(w.Hkv):
+        # dQ on the sampled rows of the four query heads of every key/value
+        # head, exact per row
         dq_r, _, _ = oracle.attention_backward_rows(x["q"], x["k"], x["v"], x["dout"], True, 0,
                                                     g, rows)
-        got = host(dq[0, torch.as_tensor(rows, device="cuda"), g * rep:(g + 1) * rep])
-        assert rel_fro(got, dq_r) <= GRAD_REL, rel_fro(got, dq_r)
-    # dK/dV exact for keys in the last 1024 positions (only rows >= j contribute)
+        got = host(dq[0, idx, g * rep:(g + 1) * rep])
+        assert rel_fro(got, dq_r) <= GRAD_REL, (g, rel_fro(got, dq_r))
+    # dK/dV exact for keys in the last 1024 positions (only rows >= j
+    # contribute), for the first and the last key/value head
     tail = np.arange(w.S - 1024, w.S)
-    _, dk_t, dv_t = oracle.attention_backward_rows(x["q"], x["k"], x["v"], x["dout"], True, 0,
-                                                   7, tail)
-    assert rel_fro(host(dk[0, -1024:, 7]), dk_t[-1024:]) <= GRAD_REL
-    assert rel_fro(host(dv[0, -1024:, 7]), dv_t[-1024:]) <= GRAD_REL
+    for g in (0, w.Hkv - 1):
+        _, dk_t, dv_t = oracle.attention_backward_rows(x["q"], x["k"], x["v"], x["dout"], True,
+                                                       0, g, tail)
+        assert rel_fro(host(dk[0, -1024:, g]), dk_t[-1024:]) <= GRAD_REL, g
+        assert rel_fro(host(dv[0, -1024:, g]), dv_t[-1024:]) <= GRAD_REL, g
     # global identities over all positions: sum_j dK_j = 0, sum_j dV_j = sum_i dO_i
     dk64 = dk.double()
     ratio = (dk64.sum(1).abs() / dk64.abs().sum(1)).max().item()
@@ -142,7 +181,7 @@ def test_llama2_13b_s1m_forward_sampled_blocks():
         r0 = b * blk
         rows += [r0, r0 + blk - 1] + (r0 + rng.integers(0, blk, 62)).tolist()
     rows = np.array(sorted(set(rows)))
-    check_rows(x, out, lse, w, (0, 13, 26, 39), rows)
+    check_rows(x, [(out, lse)], w, range(w.Hq), rows)  # all 40 heads
 
 
 def test_longlora_s2_s100k_sampled_rows():

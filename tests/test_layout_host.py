@@ -1,6 +1,6 @@
 """Host-side checks of index logic compiled for the CPU: the feedforward
-kernel's tile raster visits every output tile exactly once, in bands of 16
-row tiles walked column by column; and the packed-sequence view accepts
+kernel's tile raster visits every output tile exactly once, in bands of a
+given number of row tiles walked column by column; and the packed-sequence view accepts
 exactly the in-order, in-range offsets no longer than the longest sequence
 (the kernels skip anything else and report it); and the S2 roll's position
 -> token map is the oracle's, a permutation of each head's tokens."""
@@ -31,13 +31,13 @@ def probe():
     return run
 
 
+@pytest.mark.parametrize("band", [1, 16, 32, 64])
 @pytest.mark.parametrize("n_tm,n_tn", [(1, 1), (64, 86), (64, 16), (86, 16), (17, 3), (33, 43),
-                                       (16, 1), (5, 7)])
-def test_tile_raster_is_a_bijection_in_bands(probe, n_tm, n_tn):
-    rows = probe("tiles", n_tm, n_tn)
+                                       (16, 1), (5, 7), (172, 16)])
+def test_tile_raster_is_a_bijection_in_bands(probe, n_tm, n_tn, band):
+    rows = probe("tiles", n_tm, n_tn, band)
     coords = [(tm, tn) for _, tm, tn in rows]
     assert sorted(coords) == [(m, n) for m in range(n_tm) for n in range(n_tn)]
-    band = 16
     for t, tm, tn in rows:
         b = t // (band * n_tn)
         assert b * band <= tm < min((b + 1) * band, n_tm)   # its own band of row tiles
@@ -81,7 +81,7 @@ def test_random_tile_rasters(probe):
     import random
     rng = random.Random(7)
     for _ in range(20):
-        n_tm, n_tn = rng.randint(1, 60), rng.randint(1, 50)
-        rows = probe("tiles", n_tm, n_tn)
+        n_tm, n_tn, band = rng.randint(1, 60), rng.randint(1, 50), rng.randint(1, 70)
+        rows = probe("tiles", n_tm, n_tn, band)
         assert sorted((tm, tn) for _, tm, tn in rows) == \
             [(m, n) for m in range(n_tm) for n in range(n_tn)]

@@ -3,14 +3,16 @@ device memory (for example a plugin whose host framework owns every device
 allocation, or a latency-critical caller that cannot take cudaMalloc's cost).
 It takes its scratch from a fixed array inside the library instead of a
 caller workspace.  These tests call it through the C ABI and check it against
-lca_attn_bwd, on two calls in a row (the second call finds the first call's
-leftovers in the shared scratch).  The file is named to run last."""
+lca_attn_bwd and against the fp64 oracle's gradients, on two calls in a row
+(the second call finds the first call's leftovers in the shared scratch).
+The file is named to run last."""
 
 import ctypes
 
 import pytest
 import torch
 
+import oracle
 from long_context_exact_attention_b200 import lca
 from long_context_exact_attention_b200.inputs import WORKLOADS, make_inputs, shrink
 
@@ -53,15 +55,18 @@ def test_noalloc_matches_workspace_backward(name, kw, causal):
     ref = lca.attn_bwd(x["q"], x["k"], x["v"], out, lse, x["dout"], causal=causal)
     torch.cuda.synchronize()
     ref = [host(t) for t in ref]
+    want = oracle.attention_backward(x["q"], x["k"], x["v"], x["dout"], causal)
     for _ in range(2):
         grads = [torch.full_like(t, float("nan")) for t in (x["q"], x["k"], x["v"])]
         _call_noalloc(x, out, lse, causal, grads)
         torch.cuda.synchronize()
         lca.check()
-        for g, r in zip(grads, ref):
+        for g, r, o in zip(grads, ref, want):
             g = host(g)
             assert torch.isfinite(torch.from_numpy(g)).all()
             if w.dtype == "fp32":
                 assert max_abs(g, r) <= F32_ABS
+                assert max_abs(g, o) <= F32_ABS
             else:
                 assert rel_fro(g, r) <= GRAD_REL
+                assert rel_fro(g, o) <= GRAD_REL
