@@ -28,6 +28,11 @@ there is).
 --workload llama2_7b_ffn_s32k measures the blockwise feedforward instead
 (lca_ffn_fwd + lca_ffn_bwd over 32768 tokens of the Llama-2-7B feedforward
 in blocks of 8192): its own line, metric "blockwise feedforward TFLOP/s".
+
+--workload ring_<attention workload> (e.g. ring_llama3_8b_gqa_s256k) runs
+ring attention across the N ranks instead of replicas: one sequence split
+zig-zag over the ranks, every step one ring forward + backward with NCCL
+transfers; strong scaling, value = the whole problem's FLOPs / step time.
 """
 
 from __future__ import annotations
@@ -606,11 +611,149 @@ def attn_summary(w, t, pk):
     return d
 
 
+def main_ring(args, w):
+    """Sequence-parallel ring attention over the ranks (strong scaling: one
+    sequence of w.S tokens split over N ranks, zig-zag)."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    flops_step = w.fwd_flops() + w.bwd_flops()
+    cfg = {"workload": "ring_" + w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "S": w.S, "d": w.d,
+           "causal": w.causal, "parallelism": f"ring x{world} (zig-zag, sequence split)"}
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        vals, info = [], None
+        for _ in range(args.warmup):
+            oracle_sample(w, seconds_target=2.0, max_rows=512)
+        for _ in range(args.steps):
+            info = oracle_sample(w, seconds_target=5.0, max_rows=4096)
+            vals.append(info[0])
+        tf, R, dt, cores, reps = info
+        val = statistics.median(vals)
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": f"fp64 oracle fwd+bwd of the last {R} query rows of "
+                                       f"the {w.Hq // w.Hkv} query heads of key/value head 0"},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from long_context_exact_attention_b200 import lca, ring
+    from long_context_exact_attention_b200.inputs import make_tensor
+
+    if world > 1:
+        dist.init_process_group("nccl", init_method="env://",
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.Stream(dev)
+    # this rank's zig-zag block: chunks r and 2N-1-r of 2N
+    c = w.S // (2 * world)
+    a, b = ring.zigzag_chunks(rank, world)
+    blk = {n: torch.cat([make_tensor(w, n, dev, (a * c, (a + 1) * c)),
+                         make_tensor(w, n, dev, (b * c, (b + 1) * c))], dim=1).contiguous()
+           for n in ("q", "k", "v", "dout")}
+    torch.cuda.synchronize()
+
+    def step(S=None, st=None):
+        S = S or blk
+        with torch.cuda.stream(st or stream):
+            o, l = ring.ring_attn_fwd(S["q"], S["k"], S["v"], causal=w.causal)
+            g = ring.ring_attn_bwd(S["q"], S["k"], S["v"], o, l, S["dout"], causal=w.causal)
+            S["out"], S["lse"] = o, l
+            S["dq"], S["dk"], S["dv"] = g
+
+    for _ in range(args.warmup):
+        step()
+    stream.synchronize()
+    lca.check(stream)
+    cvd = os.environ.get("CUDA_VISIBLE_DEVICES")
+    clocks = ClockSampler(cvd.split(",")[local] if cvd else str(local))
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    start.record(stream)
+    for _ in range(args.steps):
+        step()
+    stop.record(stream)
+    stop.synchronize()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    lca.check(stream)
+    total_ms = max_over_ranks(start.elapsed_time(stop), dev)
+    value = flops_step * args.steps / (total_ms * 1e-3) / 1e12
+
+    e2e = None
+    if not args.no_e2e:
+        in_names, out_names = ["q", "k", "v", "dout"], ["out", "lse", "dq", "dk", "dv"]
+        host_in = [blk[n].cpu().pin_memory() for n in in_names]
+        host_out = [torch.empty_like(blk[n], device="cpu").pin_memory() for n in out_names]
+        sets = [blk, {n: torch.empty_like(t) for n, t in blk.items()}]
+        compute = lambda S, st: step(S, st)
+        pipelined_e2e(torch, dev, sets, in_names, out_names, host_in, host_out, compute, 2)
+        n_e2e = max(3, min(args.steps, 4))
+        if world > 1:
+            dist.barrier()
+        e_ms = max_over_ranks(pipelined_e2e(torch, dev, sets, in_names, out_names, host_in,
+                                            host_out, compute, n_e2e), dev)
+        e2e = {"value": flops_step * n_e2e / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in host_in),
+               "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in host_out),
+               "per": "rank 0's block (every rank moves its own)", "ms_per_step": e_ms / n_e2e}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    pk, pk_kind = peaks()
+    burst = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "impl": "lca", "config": cfg,
+        "frac_of_peak": {"measured_burst": value / world / burst,
+                         "nominal_2250": value / world / NOMINAL_BF16_TFLOPS},
+        "roofline": {"bound": "tensor", "kernel": "ring step (block forward and backward "
+                     "kernels)", "achieved": value / world, "peak": burst, "unit": "TFLOP/s",
+                     "frac": value / world / burst,
+                     "peak_kind": f"{pk_kind} burst bf16", "traffic": None,
+                     "timing": "CUDA events around whole ring steps (kernels and transfers), "
+                               "per GPU"},
+        "clocks": clk,
+        "gpu_launches": args.steps * ring.launches_per_step(world, w.causal),
+        "e2e": e2e,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        tf, R, dt, cores, reps = oracle_sample(w)
+        line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cores,
+                                "kind": "oracle",
+                                "sample": f"fp64 oracle fwd+bwd of the last {R} query rows of "
+                                          f"the {w.Hq // w.Hkv} query heads of key/value head 0"
+                                          f", {reps} runs, {dt:.2f} s each"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     from long_context_exact_attention_b200.inputs import FFN_WORKLOADS, WORKLOADS
     if args.workload in FFN_WORKLOADS:
         main_ffn(args, FFN_WORKLOADS[args.workload])
+        return
+    if args.workload.startswith("ring_"):
+        main_ring(args, WORKLOADS[args.workload[len("ring_"):]])
         return
     w = WORKLOADS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -111,6 +111,10 @@ WORKLOADS = {
         Workload("longlora_s2_s100k", B=1, Hq=32, Hkv=32, S=100000, d=128,
                  dtype="bf16", causal=True, seed=5, std=0.5, group=25000,
                  shift_heads=16),
+        # the Llama-3-8B layer at 256K tokens: the sequence-parallel (ring)
+        # workload, split over the ranks
+        Workload("llama3_8b_gqa_s256k", B=1, Hq=32, Hkv=8, S=262144, d=128,
+                 dtype="bf16", causal=True, seed=7, std=0.5),
         # a quarter of the 32K layer's heads: the case ncu captures in full
         # (inputs 4 x 64 MiB, still larger than L2 together)
         Workload("llama2_7b_s32k_h8", B=1, Hq=8, Hkv=8, S=32768, d=128,

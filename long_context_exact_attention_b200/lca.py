@@ -14,7 +14,10 @@ from typing import Optional, Sequence
 
 import torch
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblca.so")
+# The in-tree build; the LCA_LIBRARY environment variable names another
+# build of the same library to load instead.
+LIB_PATH = os.environ.get("LCA_LIBRARY") or os.path.join(
+    os.path.dirname(os.path.abspath(__file__)), "liblca.so")
 
 LCA_BF16, LCA_FP32 = 0, 1
 ORDERS = {"inorder": 0, "ring": 1, "custom": 2}

@@ -263,12 +263,31 @@ def _drive(gen, transport):
             reply = None
 
 
+class _NoTransport:
+    """A ring of one rank exchanges nothing."""
+    rank, world = 0, 1
+
+    def exchange(self, send, recv):
+        raise RuntimeError("a ring of one rank has nothing to exchange")
+
+    def wait(self, handle):
+        pass
+
+
+def _transport(group):
+    import torch.distributed as dist
+    if group is None and not (dist.is_available() and dist.is_initialized()):
+        return _NoTransport()
+    return DistTransport(group)
+
+
 def ring_attn_fwd(q, k, v, causal: bool = True, group=None, scale=None, ops=None):
     """Ring attention forward on this rank.  q [B, 2c, Hq, d], k/v
     [B, 2c, Hkv, d]: this rank's zig-zag block (``shard``) of the sequence;
     c must be a multiple of 128 when causal.  Every rank of `group` calls
-    it together.  Returns (out, lse) of this rank's block."""
-    t = DistTransport(group)
+    it together (without a process group: a ring of one rank).  Returns
+    (out, lse) of this rank's block."""
+    t = _transport(group)
     return _drive(_fwd_rank(t.rank, t.world, q, k, v, causal, scale, ops or KernelOps), t)
 
 
@@ -277,9 +296,20 @@ def ring_attn_bwd(q, k, v, out, lse, dout, causal: bool = True, group=None, scal
     """Ring attention backward on this rank (zig-zag blocks, as
     ``ring_attn_fwd``; out and lse are its results).  Returns (dq, dk, dv)
     of this rank's block."""
-    t = DistTransport(group)
+    t = _transport(group)
     return _drive(_bwd_rank(t.rank, t.world, q, k, v, out, lse, dout, causal, scale,
                             ops or KernelOps), t)
+
+
+def launches_per_step(world: int, causal: bool = True) -> int:
+    """This library's kernel launches of one ring forward + backward on one
+    rank (block forwards and a cast; per query chunk a row-dot and a dq
+    finalize; block backwards, the accumulator additions of the later steps
+    and a cast)."""
+    pairs = [step_pairs(0, world, s, causal) for s in range(world)]
+    n_blocks = sum(len(p) for p in pairs)
+    adds = sum(2 * len({kj for _, kj, _, _ in p}) for p in pairs[1:])
+    return (n_blocks + 1) + (2 + n_blocks + adds + 2 + 1)
 
 
 def _emulate(gens):
