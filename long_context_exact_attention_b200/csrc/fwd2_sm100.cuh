@@ -80,7 +80,7 @@ constexpr uint32_t kIdescO = idesc_bf16_f32(256, 128, false, true);   // P V (V 
 // kBlock: a block call (merging epilogue), as attn_fwd_bf16_sm100.  Only the
 // tile walk (chunks of whole tiles) runs here.
 template <bool kBlock>
-__global__ void __cluster_dims__(2, 1, 1) __maxnreg__(200)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(fwd2::kThreads, 1)
     attn_fwd_bf16_sm100_pair(const __grid_constant__ CUtensorMap tmQ,
                              const __grid_constant__ CUtensorMap tmK,   // box of 64 keys
                              const __grid_constant__ CUtensorMap tmV,   // box of 128 keys

@@ -123,13 +123,14 @@ __device__ __forceinline__ bool walk_next(TileWalk& w, int& t, int&, int&) { ret
 // Epilogue of a block call for one query row (one thread): fold this
 // block's partial (TMEM O, running m and l in log2 units) into the running
 // float32 (o_acc, lse) and/or write the merged row as bf16.  Every lane of
-// the warp calls it (the TMEM loads are warp-collective).
+// the warp calls it (the TMEM loads are warp-collective).  Four columns at a
+// time: a wider body makes the softmax loop of the block instantiation
+// spill under the 168-register limit.
 __device__ __forceinline__ void fwd_block_epilogue(const fwd::Args& a, uint32_t tO, int cnt,
-                                                float m_run, float l_run, bool row_in,
-                                                size_t trow, int h, size_t li) {
+                                                   float m_run, float l_run, bool row_in,
+                                                   size_t trow, int h, size_t li) {
   using namespace fwd;
   const float L2E = 1.4426950408889634f;
-  // log2-domain lse of this block's partial and of the running result
   const float lb = (cnt >= 1 && l_run > 0.f) ? m_run + lg2_approx(l_run) : -INFINITY;
   const float lold = (a.accumulate && row_in) ? a.lse[li] * L2E : -INFINITY;
   const float mx = fmaxf(lb, lold);
@@ -139,8 +140,7 @@ __device__ __forceinline__ void fwd_block_epilogue(const fwd::Args& a, uint32_t 
     w_old = (lold == -INFINITY) ? 0.f : ex2_approx(lold - ln);
     w_b = (lb == -INFINITY) ? 0.f : ex2_approx(m_run - ln);
   }
-  float* arow = a.o_acc ? a.o_acc + (trow * a.Hq + h) * kD : nullptr;
-  __nv_bfloat16* orow = a.out ? a.out + (trow * a.Hq + h) * kD : nullptr;
+  const size_t e0 = (trow * a.Hq + h) * kD;
 #pragma unroll 1
   for (int q4 = 0; q4 < 4; ++q4) {
     float o[32];
@@ -151,37 +151,22 @@ __device__ __forceinline__ void fwd_block_epilogue(const fwd::Args& a, uint32_t 
 #pragma unroll
       for (int i = 0; i < 32; ++i) o[i] = 0.f;
     }
-    if (row_in) {
-#pragma unroll
-      for (int i = 0; i < 32; ++i) o[i] *= w_b;
-      if (a.accumulate && w_old != 0.f) {
-        const float4* src = reinterpret_cast<const float4*>(arow + q4 * 32);
-#pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          const float4 x = src[v];
-          o[4 * v + 0] = fmaf(w_old, x.x, o[4 * v + 0]);
-          o[4 * v + 1] = fmaf(w_old, x.y, o[4 * v + 1]);
-          o[4 * v + 2] = fmaf(w_old, x.z, o[4 * v + 2]);
-          o[4 * v + 3] = fmaf(w_old, x.w, o[4 * v + 3]);
-        }
+    if (!row_in) continue;
+#pragma unroll 2
+    for (int v = 0; v < 8; ++v) {
+      const size_t e = e0 + q4 * 32 + 4 * v;
+      float4 y = make_float4(o[4 * v] * w_b, o[4 * v + 1] * w_b, o[4 * v + 2] * w_b,
+                             o[4 * v + 3] * w_b);
+      if (w_old != 0.f) {
+        const float4 x = *reinterpret_cast<const float4*>(a.o_acc + e);
+        y.x = fmaf(w_old, x.x, y.x);
+        y.y = fmaf(w_old, x.y, y.y);
+        y.z = fmaf(w_old, x.z, y.z);
+        y.w = fmaf(w_old, x.w, y.w);
       }
-      if (arow) {
-        float4* dst = reinterpret_cast<float4*>(arow + q4 * 32);
-#pragma unroll
-        for (int v = 0; v < 8; ++v)
-          dst[v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
-      }
-      if (orow) {
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          uint4 pk;
-          pk.x = pack_bf16x2(o[v * 8 + 0], o[v * 8 + 1]);
-          pk.y = pack_bf16x2(o[v * 8 + 2], o[v * 8 + 3]);
-          pk.z = pack_bf16x2(o[v * 8 + 4], o[v * 8 + 5]);
-          pk.w = pack_bf16x2(o[v * 8 + 6], o[v * 8 + 7]);
-          *reinterpret_cast<uint4*>(orow + q4 * 32 + v * 8) = pk;
-        }
-      }
+      if (a.o_acc) *reinterpret_cast<float4*>(a.o_acc + e) = y;
+      if (a.out) *reinterpret_cast<uint2*>(a.out + e) = make_uint2(pack_bf16x2(y.x, y.y),
+                                                                   pack_bf16x2(y.z, y.w));
     }
   }
   if (row_in) a.lse[li] = ln * 0.69314718055994531f;
@@ -190,12 +175,11 @@ __device__ __forceinline__ void fwd_block_epilogue(const fwd::Args& a, uint32_t 
 // kRanged: some chunk boundary falls inside a tile, so visits carry key
 // ranges (KvWalk).  Otherwise the cheaper tile walk runs and only a ragged
 // last tile needs a key mask.  kBlock: a block call (merging epilogue).
-// Register cap: 200 per thread (10 warps x 200 fit the register file at one
-// CTA per SM, which shared memory fixes anyway).  The ranged and block
-// instantiations need a few registers more than the plain one's 168, which
-// the default cap for 320 threads did not give them (they spilled).
+// 320 threads: the register file is handed out in groups of four warps, so
+// a CTA of ten warps is charged for twelve and may use at most 168
+// registers per thread (more fails to launch).
 template <bool kRanged, bool kBlock>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(fwd::kThreads, 1)
     attn_fwd_bf16_sm100(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV,
@@ -311,7 +295,9 @@ __global__ void __maxnreg__(200)
   } else if (warp == 1) {
     // =================================================== MMA issuer
     if (lane == 0) {
-      const uint32_t qts[2] = {static_cast<uint32_t>(qt0), static_cast<uint32_t>(qt0 + 1)};
+      // query tiles moved onto the key tiles' diagonal (block calls)
+      const int qd0 = qt0 + (kBlock ? sc.diag : 0);
+      const uint32_t qts[2] = {static_cast<uint32_t>(qd0), static_cast<uint32_t>(qd0 + 1)};
       bool ok = wait_bar(bar(B_Q), 0, wc, 201);
       Walk w;
       walk_init(w, &sc, qt_last, sv);
@@ -330,8 +316,7 @@ __global__ void __maxnreg__(200)
         tc_commit(bar(B_SFULL + tq));
       };
       auto act = [&](int tq, int T_) {
-        return (tq == 0 || has1) &&
-               tile_vis(causal, kBlock ? sc.diag : 0, static_cast<int>(qts[tq]), T_) != VIS_NONE;
+        return (tq == 0 || has1) && tile_vis(causal, 0, static_cast<int>(qts[tq]), T_) != VIS_NONE;
       };
       bool have = ok && walk_next(w, T, lo, hi);
       if (have) {
@@ -384,7 +369,9 @@ __global__ void __maxnreg__(200)
     const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + lane_addr + tq * 128;
     const uint32_t tO = tmem + lane_addr + 256 + tq * 128;
-    const int qt = qt0 + tq;
+    // this warpgroup's query tile, moved onto the key tiles' diagonal for
+    // block calls (the tile itself is recovered for the epilogue)
+    const int qt_d = qt0 + tq + (kBlock ? sc.diag : 0);
     const float c = a.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
     int cnt = 0;
@@ -394,7 +381,7 @@ __global__ void __maxnreg__(200)
       walk_init(w, &sc, qt_last, sv);
       int t, lo = 0, hi = kTile;
       while (ok && walk_next(w, t, lo, hi)) {
-        const int vis = tile_vis(causal, kBlock ? sc.diag : 0, qt, t);
+        const int vis = tile_vis(causal, 0, qt_d, t);
         if (vis == VIS_NONE) continue;
         ok = __all_sync(0xffffffffu, wait_bar(bar(B_SFULL + tq), cnt & 1, wc, 301));
         if (!ok) break;
@@ -421,20 +408,12 @@ __global__ void __maxnreg__(200)
           // for every row that is stored when queries and keys are one
           // sequence; a block call's key block can end inside the diagonal
           // tile before the query rows do)
-          if constexpr (kBlock) {
-            int lim = r + 1;
-            if (t == w.n_tiles - 1) {
-              const int kv_valid = ld_shared_volatile_s32(seq_smem + 16) - t * kTile;
-              lim = kv_valid < lim ? kv_valid : lim;
-            }
+          // (a key block that ends inside a tile is one chunk of a length
+          // that is not a whole number of tiles, so it takes the ranged walk,
+          // which masks by key range; here every key tile is whole)
 #pragma unroll
-            for (int i = 0; i < 128; ++i)
-              if (i >= lim) s[i] = -INFINITY;
-          } else {
-#pragma unroll
-            for (int i = 0; i < 128; ++i)
-              if (i > r) s[i] = -INFINITY;
-          }
+          for (int i = 0; i < 128; ++i)
+            if (i > r) s[i] = -INFINITY;
         } else if (t == w.n_tiles - 1) {
           // last key tile of a ragged sequence: rows past its end (S2-Attn
           // sequences are whole tiles, so nothing is masked there)
@@ -515,6 +494,7 @@ __global__ void __maxnreg__(200)
       } else {
         ok = __all_sync(0xffffffffu, ok && cnt >= 1);
       }
+      const int qt = qt_d - (kBlock ? sc.diag : 0);
       const int tok = token_tile(sc, qt, shifted) * kTile + r;
       // Every lane takes part in the TMEM loads (warp-collective); rows past
       // the end of the sequence (ragged last tile) only skip their stores.
