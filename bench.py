@@ -588,8 +588,7 @@ class AttnRun:
         med = lambda a, b: statistics.median(e[a].elapsed_time(e[b]) for e in evs)
         total = max_over_ranks(start.elapsed_time(stop), self.dev)
         return {"total_ms": total, "fwd_ms": med(0, 1), "bwd_ms": med(1, 4),
-                "bwd_main_ms": med(2, 3), "bwd_prep_ms": med(1, 2), "bwd_dq_ms": med(3, 4),
-                "clocks": clk}
+                "bwd_main_ms": med(2, 3), "clocks": clk}
 
 
 def attn_summary(w, t, pk):
@@ -601,8 +600,9 @@ def attn_summary(w, t, pk):
     d = {"fwd_tflops": tf(ff, t["fwd_ms"]), "fwd_ms": t["fwd_ms"]}
     if w.backward:
         d.update(bwd_tflops=tf(fb, t["bwd_ms"]), bwd_ms=t["bwd_ms"],
-                 bwd_main_tflops=tf(fb, t["bwd_main_ms"]), bwd_main_ms=t["bwd_main_ms"],
                  fwd_bwd_tflops=tf(ff + fb, t["fwd_ms"] + t["bwd_ms"]))
+        if run_phased(w):  # the main kernel has events of its own
+            d.update(bwd_main_tflops=tf(fb, t["bwd_main_ms"]), bwd_main_ms=t["bwd_main_ms"])
     for key in ("fwd_tflops", "bwd_main_tflops"):
         if d.get(key):
             d[key.replace("_tflops", "_frac")] = {

@@ -9,6 +9,10 @@ library's backward entry point.  Every step runs in the CUDA library.
     out = attention(q, k, v, causal=True, kv_chunk=4096, order="ring")
     out.float().sum().backward()
 
+Sequence parallel (every rank of the process group calls with its own block):
+``ring_attention`` over zig-zag blocks (ring.shard), ``ulysses_attention``
+over contiguous shards.
+
 Errors inside a kernel (a wait that ran out, invalid packed offsets) are
 recorded in the library's device error word, not raised by these calls,
 because reading it synchronises the stream.  Call ``lca.check()`` at a point
@@ -21,7 +25,7 @@ from __future__ import annotations
 
 import torch
 
-from . import lca
+from . import lca, ring, ulysses
 
 
 class _Attention(torch.autograd.Function):
@@ -58,6 +62,40 @@ class _S2Attention(torch.autograd.Function):
         return dq, dk, dv, None, None, None, None
 
 
+class _RingAttention(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, q, k, v, causal, group, scale):
+        out, lse = ring.ring_attn_fwd(q, k, v, causal=causal, group=group, scale=scale)
+        ctx.save_for_backward(q, k, v, out, lse)
+        ctx.args = (causal, group, scale)
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, out, lse = ctx.saved_tensors
+        causal, group, scale = ctx.args
+        dq, dk, dv = ring.ring_attn_bwd(q, k, v, out, lse, dout.contiguous(), causal=causal,
+                                        group=group, scale=scale)
+        return dq, dk, dv, None, None, None
+
+
+class _UlyssesAttention(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, q, k, v, causal, group, scale):
+        out, lse_h = ulysses.ulysses_attn_fwd(q, k, v, causal=causal, group=group, scale=scale)
+        ctx.save_for_backward(q, k, v, out, lse_h)
+        ctx.args = (causal, group, scale)
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, out, lse_h = ctx.saved_tensors
+        causal, group, scale = ctx.args
+        dq, dk, dv = ulysses.ulysses_attn_bwd(q, k, v, out, lse_h, dout.contiguous(),
+                                              causal=causal, group=group, scale=scale)
+        return dq, dk, dv, None, None, None
+
+
 class _Feedforward(torch.autograd.Function):
     @staticmethod
     def forward(ctx, x, w_gate, w_up, w_down, block_tokens):
@@ -90,3 +128,17 @@ def feedforward(x, w_gate, w_up, w_down, block_tokens: int = 0):
     gradients are accumulated in float32 by the library and returned in the
     weights' dtype."""
     return _Feedforward.apply(x, w_gate, w_up, w_down, block_tokens)
+
+
+def ring_attention(q, k, v, causal: bool = True, group=None, scale=None):
+    """Ring attention with autograd on this rank: q [B,2c,Hq,d], k/v
+    [B,2c,Hkv,d] are the rank's zig-zag block (ring.shard); the output is
+    the block's rows.  Every rank of `group` calls it together (without a
+    process group it is one rank holding the whole sequence)."""
+    return _RingAttention.apply(q, k, v, causal, group, scale)
+
+
+def ulysses_attention(q, k, v, causal: bool = True, group=None, scale=None):
+    """Ulysses sequence parallelism with autograd on this rank: q
+    [B,S/W,Hq,d], k/v [B,S/W,Hkv,d] are the rank's contiguous shard."""
+    return _UlyssesAttention.apply(q, k, v, causal, group, scale)

@@ -14,7 +14,6 @@
 #include "aux_kernels.cuh"
 #include "bwd_sm100.cuh"
 #include "ffn_sm100.cuh"
-#include "fwd2_sm100.cuh"
 #include "fwd_sm100.cuh"
 #include "ptx.cuh"
 #include "sched.cuh"
@@ -223,14 +222,13 @@ EncodeTiledFn encode_fn() {
 // axis of all B*S rows); box = 64 head dims x 1 head x 128 tokens.  Rows
 // past the last token load as zeros; a ragged tile otherwise reads the
 // following batch entry's rows, which the kernels mask.
-lca_status make_map(CUtensorMap* m, const void* ptr, int64_t B, int64_t S, int64_t heads,
-                    uint32_t box_tokens = 128) {
+lca_status make_map(CUtensorMap* m, const void* ptr, int64_t B, int64_t S, int64_t heads) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(LCA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(heads),
                               static_cast<cuuint64_t>(B * S)};
   const cuuint64_t strides[2] = {128 * 2, static_cast<cuuint64_t>(heads) * 128 * 2};
-  const cuuint32_t box[3] = {64, 1, box_tokens};
+  const cuuint32_t box[3] = {64, 1, 128};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -351,9 +349,6 @@ unsigned long long budget_of(const lca_opts* o) {
 }
 
 // ---------------------------------------------------------------- forward
-// The forward on CTA pairs (fwd2_sm100.cuh) for the paths it covers.
-constexpr bool kUsePairForward = false;
-
 // Block calls pass o_acc (may be null when out is given) and `accumulate`;
 // `block` selects the merging epilogue.
 struct FwdBlock {
@@ -380,46 +375,6 @@ lca_status run_fwd(const Common& c, const AttnSched& s, const void* q, const voi
     if ((r = make_map(&mv, v, c.B, c.S_kv, c.Hkv)) != LCA_OK) return r;
     // chunk boundaries inside a tile need the ranged walk
     const bool ranged = !s.s2 && s.kv_chunk % c.tile != 0;
-    // CTA pairs (M = 256 products) for the tile walk over dense sequences;
-    // packed sequences, ranged chunks, S2 groups of other than a multiple of
-    // four tiles and block calls whose key block ends inside a tile take the
-    // single-CTA kernel
-    const bool pair = kUsePairForward && !ranged && !c.cu &&
-                      (!s.s2 || s.group_tiles % 4 == 0) &&
-                      (!fb.block || c.S_kv % c.tile == 0);
-    if (pair) {
-      CUtensorMap mk64;
-      if ((r = make_map(&mk64, k, c.B, c.S_kv, c.Hkv, 64)) != LCA_OK) return r;
-      fwd::Args a;
-      a.B = c.n_seq;
-      a.Hq = c.Hq;
-      a.Hkv = c.Hkv;
-      a.S = c.S;
-      a.scale_log2 = c.scale * 1.4426950408889634f;
-      a.budget = budget;
-      a.out = static_cast<__nv_bfloat16*>(out);
-      a.lse = lse;
-      a.o_acc = fb.o_acc;
-      a.accumulate = fb.accumulate;
-      a.sched = s;
-      const int64_t n_quads = (s.n_tiles + 3) / 4;
-      const int64_t grid_pair = 2 * n_quads * c.n_seq * c.Hq;
-      if (grid_pair > 0x7fffffffll)
-        return fail(LCA_ERR_INVALID_ARG, "%lld query tiles exceed one launch",
-                    static_cast<long long>(grid_pair));
-      if (fb.block) {
-        if ((r = ensure_smem(attn_fwd_bf16_sm100_pair<true>, fwd2::kSmemBytes, 17)) != LCA_OK)
-          return r;
-        attn_fwd_bf16_sm100_pair<true><<<static_cast<unsigned>(grid_pair), fwd2::kThreads,
-                                         fwd2::kSmemBytes, st>>>(mq, mk64, mv, a);
-      } else {
-        if ((r = ensure_smem(attn_fwd_bf16_sm100_pair<false>, fwd2::kSmemBytes, 16)) != LCA_OK)
-          return r;
-        attn_fwd_bf16_sm100_pair<false><<<static_cast<unsigned>(grid_pair), fwd2::kThreads,
-                                          fwd2::kSmemBytes, st>>>(mq, mk64, mv, a);
-      }
-      return launched("attn_fwd_bf16_sm100_pair");
-    }
     if (fb.block) {
       if (ranged) {
         if ((r = ensure_smem(attn_fwd_bf16_sm100<true, true>, fwd::kSmemBytes, 14)) != LCA_OK)
@@ -702,6 +657,7 @@ Common packed_of(const Common& c, const S2Plan& p, const int* cu) {
   Common q = c;
   q.n_seq = p.n_seq;
   q.S = c.B * c.S;
+  q.S_kv = q.S;  // the rolled keys share the packed token axis
   q.B = 1;
   q.S_seq = static_cast<int>(p.group);
   q.cu = cu;

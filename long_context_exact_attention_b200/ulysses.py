@@ -79,6 +79,10 @@ class DistAllToAll:
         import torch.distributed as dist
         self.dist = dist
         self.group = group
+        if group is None and not (dist.is_available() and dist.is_initialized()):
+            # no process group: one rank holding the whole sequence
+            self.rank, self.world, self.nccl = 0, 1, False
+            return
         self.rank = dist.get_rank(group)
         self.world = dist.get_world_size(group)
         self.nccl = dist.get_backend(group) == "nccl"

@@ -64,3 +64,22 @@ def test_feedforward_autograd_matches_direct_calls():
     assert torch.equal(out.detach(), ref) and torch.equal(xs[0].grad, dx)
     for t, g32 in zip(xs[1:], (dwg, dwu, dwd)):
         assert torch.equal(t.grad, g32.to(torch.bfloat16))
+
+
+def test_ring_attention_autograd_one_rank_matches_attention():
+    """Without a process group the ring is one rank holding the whole
+    sequence as its zig-zag block (chunks 0 and 1): the same results as the
+    dense wrapper, up to the float32 order of the block merges."""
+    from long_context_exact_attention_b200.autograd import ring_attention
+    w = shrink(WORKLOADS["llama3_8b_gqa_s128k"], S=512, B=1, Hq=4, Hkv=2, seed=23)
+    x = device_inputs(w)
+    q, k, v = leaf(x["q"]), leaf(x["k"]), leaf(x["v"])
+    out = ring_attention(q, k, v, causal=True)
+    out.backward(x["dout"])
+    q2, k2, v2 = leaf(x["q"]), leaf(x["k"]), leaf(x["v"])
+    ref = attention(q2, k2, v2, causal=True)
+    ref.backward(x["dout"])
+    torch.cuda.synchronize()
+    assert (out.detach().float() - ref.detach().float()).abs().max() < 2e-2
+    for a, b in ((q.grad, q2.grad), (k.grad, k2.grad), (v.grad, v2.grad)):
+        assert ((a.float() - b.float()).norm() / b.float().norm()).item() < 2e-2
