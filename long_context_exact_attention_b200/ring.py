@@ -189,9 +189,11 @@ def _bwd_rank(rank: int, world: int, q, k, v, out, lse, dout, causal: bool, scal
                     ops.accumulate(part[kj], acc[kj])
                     ops.accumulate(part[2 + kj], acc[2 + kj])
         # hand the block's accumulators on; after the last step this sends
-        # every block home (rank r then holds its own block's gradients)
-        h_acc = yield Exchange(acc, acc_nxt)
-        acc, acc_nxt = acc_nxt, acc
+        # every block home (rank r then holds its own block's gradients).
+        # A ring of one rank holds its own block throughout.
+        if world > 1:
+            h_acc = yield Exchange(acc, acc_nxt)
+            acc, acc_nxt = acc_nxt, acc
         if step + 1 < world:
             yield Wait(h_kv)
             kv, kv_nxt = kv_nxt, kv

@@ -221,3 +221,16 @@ def test_single_process_emulation_matches_the_definition(world):
     assert torch.equal(dk, want_dk.view(1, -1, 1, 1).expand(B, S, k.shape[2], d))
     assert torch.equal(ring.unshard(lses, dim=2),
                        want_cnt.view(1, 1, -1).expand(B, Hq, S))
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_one_rank_ring_without_a_process_group(causal):
+    """No process group: the driver runs a ring of one rank, which holds its
+    own key/value block throughout and sends nothing (its backward must not
+    try to hand the block's accumulators on)."""
+    assert not (dist.is_available() and dist.is_initialized())
+    calls = {}
+    _check_rank(1, 0, causal, 3, calls)
+    want = [(0, 0), (1, 0), (1, 1)] if causal else [(a, b) for a in range(2) for b in range(2)]
+    for kind in ("fwd", "bwd"):
+        assert sorted((gq, gk) for kd, gq, gk in calls[0] if kd == kind) == want, kind
