@@ -90,16 +90,16 @@ def source_sha(files=None):
     return h.hexdigest()[:16]
 
 
-def traffic_record(kernel):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current sources of that kernel (the files the record lists);
-    else None."""
+def traffic_record(kernel, workload):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu
+    summaries, if they were taken on the current sources of that kernel (the
+    files the record lists); else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
-    rec = d.get(kernel)
+    rec = d.get(f"{kernel}@{workload}")
     if not rec or rec.get("source_sha") != source_sha(rec.get("sources")):
         return None
     return rec
@@ -427,7 +427,7 @@ def main_ffn(args, w):
     sustained = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     fwd_t, bwd_t = statistics.median(fwd_ms), statistics.median(bwd_ms)
     ach = bwd_flops / (bwd_t * 1e-3) / 1e12
-    tr = traffic_record("ffn_gemm_sm100_bwd")
+    tr = traffic_record("ffn_gemm_sm100_bwd", w.name)
     in_bytes = sum(t.numel() * t.element_size() for t in list(x.values()) + [dout])
     cfg["l2"] = (f"inputs larger than L2 (x and weights {in_bytes / 2**20:.0f} MiB together, "
                  "L2 126 MB); no flush")
@@ -873,7 +873,7 @@ def main():
         kname = "attn_fwd_bf16_sm100"
         ach = summary["fwd_tflops"]
         timing = "CUDA events around lca_attn_fwd, median over timed steps"
-    tr = traffic_record(kname)
+    tr = traffic_record(kname, w.name)
     roof = {"bound": "tensor", "kernel": kname, "achieved": ach, "peak": burst,
             "unit": "TFLOP/s", "frac": ach / burst,
             "peak_kind": f"{pk_kind} burst bf16 (the kernel is timed per launch)",
