@@ -120,6 +120,11 @@ WORKLOADS = {
         Workload("llama2_7b_s32k_h8", B=1, Hq=8, Hkv=8, S=32768, d=128,
                  dtype="bf16", causal=True, seed=1, std=0.5, rope=True,
                  kv_chunk=4096, order="ring"),
+        # a quarter of the 128K GQA layer's heads (8 query, 2 key/value),
+        # the same sequence and chunking: the case ncu captures in full for
+        # that layer (inputs 2 x 256 + 2 x 64 MiB)
+        Workload("llama3_8b_gqa_s128k_h8", B=1, Hq=8, Hkv=2, S=131072, d=128,
+                 dtype="bf16", causal=True, seed=3, std=0.5, kv_chunk=8192),
     ]
 }
 
