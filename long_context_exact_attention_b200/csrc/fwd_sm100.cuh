@@ -57,6 +57,7 @@ constexpr int kD = 128;
 constexpr uint32_t kHalf = kTile * 64 * 2;  // 16 KB
 constexpr uint32_t kTileB = 2 * kHalf;      // 32 KB
 constexpr int kThreads = 320;
+constexpr int kHeadBand = 4;  // heads whose CTAs are ordered together (work order)
 
 constexpr uint32_t kOffQ = 0;                      // 2 query tiles
 constexpr uint32_t kOffK = kOffQ + 2 * kTileB;     // 2 stages
@@ -203,13 +204,25 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work item: a pair of query tiles.  Head-major order (the CTAs in
-  // flight share one or two heads' K/V in L2), longest causal pairs first
-  // within a head.
+  // ---- work item: a pair of query tiles.  Heads in bands of kHeadBand;
+  // inside a band the longest causal pairs of all its heads come first
+  // (with S2-Attn, the pairs at the same place in every group), so the grid
+  // ends on short pairs, while the CTAs in flight still share a few heads'
+  // K/V in L2.  (One head per band would start the last head's longest
+  // pair only once the heads before it are done, and end the grid on it.)
   const AttnSched& sc = a.sched;
   const int n_pairs = (sc.n_tiles + 1) >> 1;
-  const int pr = n_pairs - 1 - static_cast<int>(blockIdx.x) % n_pairs;
-  const int bh = static_cast<int>(blockIdx.x) / n_pairs;
+  const int pg_s2 = sc.s2 ? sc.group_tiles >> 1 : 0;  // pairs per S2 group
+  const int pg = (pg_s2 > 0 && !(sc.group_tiles & 1) && n_pairs % pg_s2 == 0) ? pg_s2 : n_pairs;
+  const int n_groups = n_pairs / pg;
+  const int n_bh = a.B * a.Hq;
+  const int band_cta = kHeadBand * n_pairs;
+  const int band = static_cast<int>(blockIdx.x) / band_cta;
+  const int in_band = static_cast<int>(blockIdx.x) - band * band_cta;
+  const int band_heads = min(kHeadBand, n_bh - band * kHeadBand);
+  const int slot = in_band / band_heads;  // (length class, group), longest class first
+  const int pr = (slot % n_groups) * pg + (pg - 1 - slot / n_groups);
+  const int bh = band * kHeadBand + in_band % band_heads;
   const int h = bh % a.Hq;
   const int b = bh / a.Hq;
   const int g = h / (a.Hq / a.Hkv);
