@@ -336,10 +336,10 @@ def main_ffn(args, w):
     from long_context_exact_attention_b200 import lca
     from long_context_exact_attention_b200.inputs import make_ffn_inputs
 
+    torch.cuda.set_device(local)  # before the process group, so NCCL binds this GPU
     if world > 1:
         dist.init_process_group("nccl", init_method="env://",
                                 timeout=__import__("datetime").timedelta(seconds=120))
-    torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     stream = torch.cuda.Stream(dev)
     x = make_ffn_inputs(w, dev)
@@ -648,10 +648,10 @@ def main_ring(args, w):
     from long_context_exact_attention_b200 import lca, ring
     from long_context_exact_attention_b200.inputs import make_tensor
 
+    torch.cuda.set_device(local)  # before the process group, so NCCL binds this GPU
     if world > 1:
         dist.init_process_group("nccl", init_method="env://",
                                 timeout=__import__("datetime").timedelta(seconds=120))
-    torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     stream = torch.cuda.Stream(dev)
     # this rank's zig-zag block: chunks r and 2N-1-r of 2N
@@ -793,10 +793,10 @@ def main():
     import torch
     import torch.distributed as dist
 
+    torch.cuda.set_device(local)  # before the process group, so NCCL binds this GPU
     if world > 1:
         dist.init_process_group("nccl", init_method="env://",
                                 timeout=__import__("datetime").timedelta(seconds=120))
-    torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     stream = torch.cuda.Stream(dev)
     run = AttnRun(w, dev, stream)
