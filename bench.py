@@ -33,6 +33,9 @@ in blocks of 8192): its own line, metric "blockwise feedforward TFLOP/s".
 ring attention across the N ranks instead of replicas: one sequence split
 zig-zag over the ranks, every step one ring forward + backward with NCCL
 transfers; strong scaling, value = the whole problem's FLOPs / step time.
+--workload ulysses_<attention workload> does the same with Ulysses
+(contiguous blocks, all-to-all between the sequence split and a head split;
+N must divide the key/value heads).
 """
 
 from __future__ import annotations
@@ -611,15 +614,19 @@ def attn_summary(w, t, pk):
     return d
 
 
-def main_ring(args, w):
-    """Sequence-parallel ring attention over the ranks (strong scaling: one
-    sequence of w.S tokens split over N ranks, zig-zag)."""
+def main_seqpar(args, w, method):
+    """Sequence-parallel attention over the ranks (strong scaling: one
+    sequence of w.S tokens split over N ranks): ring attention (zig-zag
+    blocks, key/value blocks rotating) or Ulysses (contiguous blocks, heads
+    exchanged by all-to-all)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     flops_step = w.fwd_flops() + w.bwd_flops()
-    cfg = {"workload": "ring_" + w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "S": w.S, "d": w.d,
-           "causal": w.causal, "parallelism": f"ring x{world} (zig-zag, sequence split)"}
+    label = ("ring x%d (zig-zag, sequence split)" if method == "ring"
+             else "ulysses x%d (sequence split, heads exchanged by all-to-all)") % world
+    cfg = {"workload": f"{method}_{w.name}", "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "S": w.S,
+           "d": w.d, "causal": w.causal, "parallelism": label}
     if args.impl == "reference":
         if rank != 0:
             return
@@ -645,7 +652,7 @@ def main_ring(args, w):
 
     import torch
     import torch.distributed as dist
-    from long_context_exact_attention_b200 import lca, ring
+    from long_context_exact_attention_b200 import lca, ring, ulysses
     from long_context_exact_attention_b200.inputs import make_tensor
 
     torch.cuda.set_device(local)  # before the process group, so NCCL binds this GPU
@@ -654,19 +661,29 @@ def main_ring(args, w):
                                 timeout=__import__("datetime").timedelta(seconds=120))
     dev = torch.device("cuda", local)
     stream = torch.cuda.Stream(dev)
-    # this rank's zig-zag block: chunks r and 2N-1-r of 2N
-    c = w.S // (2 * world)
-    a, b = ring.zigzag_chunks(rank, world)
-    blk = {n: torch.cat([make_tensor(w, n, dev, (a * c, (a + 1) * c)),
-                         make_tensor(w, n, dev, (b * c, (b + 1) * c))], dim=1).contiguous()
-           for n in ("q", "k", "v", "dout")}
+    if method == "ring":
+        # this rank's zig-zag block: chunks r and 2N-1-r of 2N
+        c = w.S // (2 * world)
+        a, b = ring.zigzag_chunks(rank, world)
+        blk = {n: torch.cat([make_tensor(w, n, dev, (a * c, (a + 1) * c)),
+                             make_tensor(w, n, dev, (b * c, (b + 1) * c))], dim=1).contiguous()
+               for n in ("q", "k", "v", "dout")}
+        fwd, bwd = ring.ring_attn_fwd, ring.ring_attn_bwd
+        launches = ring.launches_per_step(world, w.causal)
+    else:
+        # this rank's contiguous block of S / N tokens
+        c = w.S // world
+        blk = {n: make_tensor(w, n, dev, (rank * c, (rank + 1) * c)).contiguous()
+               for n in ("q", "k", "v", "dout")}
+        fwd, bwd = ulysses.ulysses_attn_fwd, ulysses.ulysses_attn_bwd
+        launches = ulysses.launches_per_step(world)
     torch.cuda.synchronize()
 
     def step(S=None, st=None):
         S = S or blk
         with torch.cuda.stream(st or stream):
-            o, l = ring.ring_attn_fwd(S["q"], S["k"], S["v"], causal=w.causal)
-            g = ring.ring_attn_bwd(S["q"], S["k"], S["v"], o, l, S["dout"], causal=w.causal)
+            o, l = fwd(S["q"], S["k"], S["v"], causal=w.causal)
+            g = bwd(S["q"], S["k"], S["v"], o, l, S["dout"], causal=w.causal)
             S["out"], S["lse"] = o, l
             S["dq"], S["dk"], S["dv"] = g
 
@@ -726,14 +743,16 @@ def main_ring(args, w):
         "data": "synthetic", "impl": "lca", "config": cfg,
         "frac_of_peak": {"measured_burst": value / world / burst,
                          "nominal_2250": value / world / NOMINAL_BF16_TFLOPS},
-        "roofline": {"bound": "tensor", "kernel": "ring step (block forward and backward "
-                     "kernels)", "achieved": value / world, "peak": burst, "unit": "TFLOP/s",
+        "roofline": {"bound": "tensor", "kernel": ("ring step (block forward and backward "
+                     "kernels)" if method == "ring" else "Ulysses step (attention forward and "
+                     "backward over the rank's heads)"), "achieved": value / world, "peak": burst,
+                     "unit": "TFLOP/s",
                      "frac": value / world / burst,
                      "peak_kind": f"{pk_kind} burst bf16", "traffic": None,
-                     "timing": "CUDA events around whole ring steps (kernels and transfers), "
-                               "per GPU"},
+                     "timing": f"CUDA events around whole {method} steps (kernels and "
+                               "transfers), per GPU"},
         "clocks": clk,
-        "gpu_launches": args.steps * ring.launches_per_step(world, w.causal),
+        "gpu_launches": args.steps * launches,
         "e2e": e2e,
     }
     if not args.no_cpu_baseline and world == 1:
@@ -752,9 +771,10 @@ def main():
     if args.workload in FFN_WORKLOADS:
         main_ffn(args, FFN_WORKLOADS[args.workload])
         return
-    if args.workload.startswith("ring_"):
-        main_ring(args, WORKLOADS[args.workload[len("ring_"):]])
-        return
+    for method in ("ring", "ulysses"):
+        if args.workload.startswith(method + "_"):
+            main_seqpar(args, WORKLOADS[args.workload[len(method) + 1:]], method)
+            return
     w = WORKLOADS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -136,6 +136,14 @@ def ulysses_attn_bwd(q, k, v, out, lse_h, dout, causal: bool = True, group=None,
     return tuple(heads_from_front(a2a(seq_to_front(t, W))) for t in (dqh, dkh, dvh))
 
 
+def launches_per_step(world: int) -> int:
+    """This library's kernel launches of one Ulysses forward + backward on
+    one rank: the forward over the rank's heads, then the backward's row-dot,
+    main kernel and dq finalize (the re-layouts around the all-to-alls are
+    tensor copies, the all-to-alls the process group's)."""
+    return 1 + 3
+
+
 # ---------------------------------------------------------------- one-device stand-in
 
 def emulate_all_to_all(slabs: List[torch.Tensor]) -> List[torch.Tensor]:
