@@ -2,7 +2,7 @@
 //
 // One CTA per (pair of query tiles of 128 rows, query head, batch).  Roles:
 //   warp 0      TMA producer: both Q tiles once, then K and V tiles through
-//               2-stage rings
+//               3- and 2-stage rings
 //   warp 1      TMEM owner; lane 0 issues every tcgen05.mma
 //   warps 2..5  softmax warpgroup of query tile 0, one row per thread
 //   warps 6..9  softmax warpgroup of query tile 1
@@ -39,7 +39,7 @@
 //
 // TMEM columns: S/P tile 0 [0,128) | S/P tile 1 [128,256) | O tile 0
 // [256,384) | O tile 1 [384,512).
-// Shared memory (1024-aligned, 128-byte swizzle): Q0 | Q1 | K x2 | V x2.
+// Shared memory (1024-aligned, 128-byte swizzle): Q0 | Q1 | K x3 | V x2.
 // Each 128x128 bf16 tile is two 16 KB halves (head dims 0-63, 64-127).
 #pragma once
 
@@ -60,24 +60,35 @@ constexpr int kThreads = 320;
 constexpr int kHeadBand = 4;  // heads whose CTAs are ordered together (work order)
 
 constexpr uint32_t kOffQ = 0;                      // 2 query tiles
-constexpr uint32_t kOffK = kOffQ + 2 * kTileB;     // 2 stages
-constexpr uint32_t kOffV = kOffK + 2 * kTileB;     // 2 stages
-constexpr uint32_t kOffBar = kOffV + 2 * kTileB;   // barriers (8 B each)
+// Ring depths: K is read by the next S product of both query tiles right
+// behind the PV that frees V, so it gets the deeper ring (225 KB of shared
+// memory in all).
+constexpr int kKStages = 3;
+constexpr int kVStages = 2;
+constexpr uint32_t kOffK = kOffQ + 2 * kTileB;             // kKStages stages
+constexpr uint32_t kOffV = kOffK + kKStages * kTileB;      // kVStages stages
+constexpr uint32_t kOffBar = kOffV + kVStages * kTileB;    // barriers (8 B each)
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + alignment slack
 
 // barrier indices
 enum {
   B_Q = 0,
-  B_KFULL = 1,   // +stage
-  B_KEMPTY = 3,  // +stage
-  B_VFULL = 5,   // +stage
-  B_VEMPTY = 7,  // +stage
-  B_SFULL = 9,   // +query tile
-  B_PFULL = 11,  // +query tile, 128 arrivals
-  B_OREADY = 13, // +query tile
-  B_DRAIN = 15,
-  NUM_BARS = 16
+  B_KFULL = 1,                       // +stage
+  B_KEMPTY = B_KFULL + kKStages,     // +stage
+  B_VFULL = B_KEMPTY + kKStages,     // +stage
+  B_VEMPTY = B_VFULL + kVStages,     // +stage
+  B_SFULL = B_VEMPTY + kVStages,     // +query tile
+  B_PFULL = B_SFULL + 2,             // +query tile, 128 arrivals
+  B_OREADY = B_PFULL + 2,            // +query tile
+  B_DRAIN = B_OREADY + 2,
+  NUM_BARS
 };
+static_assert(8 * NUM_BARS + 40 <= 256, "barrier area");
+// ring slot and phase of key/value tile j
+__device__ __forceinline__ int kslot(int j) { return j % kKStages; }
+__device__ __forceinline__ uint32_t kphase(int j) { return (j / kKStages) & 1; }
+__device__ __forceinline__ int vslot(int j) { return j % kVStages; }
+__device__ __forceinline__ uint32_t vphase(int j) { return (j / kVStages) & 1; }
 
 constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false, false);   // Q K^T
 constexpr uint32_t kIdescO = idesc_bf16_f32(128, 128, false, true);    // P V (V MN-major)
@@ -277,32 +288,33 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       Walk w;
       walk_init(w, &sc, qt_last, sv);
       int t, lo = 0, hi = kTile, j = 0;
-      int k_issued0 = 0, k_issued1 = 0, v_issued0 = 0, v_issued1 = 0;
+      int k_issued = 0, v_issued = 0;  // tiles whose K / V copy was issued
       bool ok = true;
       while (ok && walk_next(w, t, lo, hi)) {
-        const int st = j & 1;
         const int tok = sv.kv_row0 + token_tile(sc, t, shifted) * kTile;
-        if (j >= 2) ok = wait_bar(bar(B_KEMPTY + st), ((j - 2) >> 1) & 1, wc, 101);
+        const int ks = kslot(j), vs = vslot(j);
+        if (j >= kKStages) ok = wait_bar(bar(B_KEMPTY + ks), kphase(j - kKStages), wc, 101);
         if (!ok) break;
-        mbar_expect_tx(bar(B_KFULL + st), kTileB);
-        tma_load_3d(sK + st * kTileB, &tmK, bar(B_KFULL + st), 0, g, tok);
-        tma_load_3d(sK + st * kTileB + kHalf, &tmK, bar(B_KFULL + st), 64, g, tok);
-        if (st) ++k_issued1; else ++k_issued0;
-        if (j >= 2) ok = wait_bar(bar(B_VEMPTY + st), ((j - 2) >> 1) & 1, wc, 102);
+        mbar_expect_tx(bar(B_KFULL + ks), kTileB);
+        tma_load_3d(sK + ks * kTileB, &tmK, bar(B_KFULL + ks), 0, g, tok);
+        tma_load_3d(sK + ks * kTileB + kHalf, &tmK, bar(B_KFULL + ks), 64, g, tok);
+        ++k_issued;
+        if (j >= kVStages) ok = wait_bar(bar(B_VEMPTY + vs), vphase(j - kVStages), wc, 102);
         if (!ok) break;
-        mbar_expect_tx(bar(B_VFULL + st), kTileB);
-        tma_load_3d(sV + st * kTileB, &tmV, bar(B_VFULL + st), 0, g, tok);
-        tma_load_3d(sV + st * kTileB + kHalf, &tmV, bar(B_VFULL + st), 64, g, tok);
-        if (st) ++v_issued1; else ++v_issued0;
+        mbar_expect_tx(bar(B_VFULL + vs), kTileB);
+        tma_load_3d(sV + vs * kTileB, &tmV, bar(B_VFULL + vs), 0, g, tok);
+        tma_load_3d(sV + vs * kTileB + kHalf, &tmV, bar(B_VFULL + vs), 64, g, tok);
+        ++v_issued;
         ++j;
       }
       if (!ok) {
-        // Unwind: let the copies already issued land before the CTA exits.
+        // Unwind: let the copies already issued land before the CTA exits
+        // (the last copy into each slot completes that slot's last phase).
         drain_bar(bar(B_Q), 0, 161);
-        if (k_issued0) drain_bar(bar(B_KFULL), (k_issued0 - 1) & 1, 162);
-        if (k_issued1) drain_bar(bar(B_KFULL + 1), (k_issued1 - 1) & 1, 163);
-        if (v_issued0) drain_bar(bar(B_VFULL), (v_issued0 - 1) & 1, 164);
-        if (v_issued1) drain_bar(bar(B_VFULL + 1), (v_issued1 - 1) & 1, 165);
+        for (int x = k_issued - 1; x >= 0 && x >= k_issued - kKStages; --x)
+          drain_bar(bar(B_KFULL + kslot(x)), kphase(x), 162);
+        for (int x = v_issued - 1; x >= 0 && x >= v_issued - kVStages; --x)
+          drain_bar(bar(B_VFULL + vslot(x)), vphase(x), 164);
       }
     }
   } else if (warp == 1) {
@@ -318,7 +330,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       int pv_cnt[2] = {0, 0};
       // S_t for key tile j into the S/P columns of query tile t
       auto issue_s = [&](int tq, int j) {
-        const uint32_t kbase = sK + (j & 1) * kTileB;
+        const uint32_t kbase = sK + kslot(j) * kTileB;
         const uint32_t qbase = sQ + tq * kTileB;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
@@ -344,14 +356,14 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       int j = 0;
       while (ok && have) {
         const bool has_next = walk_next(w, Tn, lo, hi);
-        ok = wait_bar(bar(B_VFULL + (j & 1)), (j >> 1) & 1, wc, 203);
-        if (ok && has_next) ok = wait_bar(bar(B_KFULL + ((j + 1) & 1)), ((j + 1) >> 1) & 1, wc, 204);
+        ok = wait_bar(bar(B_VFULL + vslot(j)), vphase(j), wc, 203);
+        if (ok && has_next) ok = wait_bar(bar(B_KFULL + kslot(j + 1)), kphase(j + 1), wc, 204);
         for (int tq = 0; tq < 2 && ok; ++tq) {
           if (act(tq, T)) {
             ok = wait_bar(bar(B_PFULL + tq), pv_cnt[tq] & 1, wc, 205);
             if (!ok) break;
             tc_fence_after();
-            const uint32_t vbase = sV + (j & 1) * kTileB;
+            const uint32_t vbase = sV + vslot(j) * kTileB;
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
               mma_bf16_ts(tmem + 256 + tq * 128, tmem + tq * 128 + k * 8,
@@ -364,8 +376,8 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
           if (has_next && act(tq, Tn)) issue_s(tq, j + 1);
         }
         if (!ok) break;
-        tc_commit(bar(B_VEMPTY + (j & 1)));
-        if (has_next) tc_commit(bar(B_KEMPTY + ((j + 1) & 1)));
+        tc_commit(bar(B_VEMPTY + vslot(j)));
+        if (has_next) tc_commit(bar(B_KEMPTY + kslot(j + 1)));
         have = has_next;
         T = Tn;
         ++j;
