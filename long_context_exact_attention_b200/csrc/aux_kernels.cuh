@@ -67,17 +67,32 @@ __global__ void bwd_rowdot(const T* __restrict__ out, const T* __restrict__ dout
     const T* o = out + ((r0 + s) * H + h) * D;
     const T* g = dout + ((r0 + s) * H + h) * D;
     float acc = 0.f;
+    if constexpr (sizeof(T) == 2 && D == 128) {
+      // one 8-byte word (four bf16) of each row per lane: the warp reads
+      // both 256-byte rows with one load each
+      const uint2 ow = reinterpret_cast<const uint2*>(o)[lane];
+      const uint2 gw = reinterpret_cast<const uint2*>(g)[lane];
+      const uint32_t ov[2] = {ow.x, ow.y}, gv[2] = {gw.x, gw.y};
 #pragma unroll
-    for (int c = lane; c < D; c += 32) {
-      float ov, gv;
-      if constexpr (sizeof(T) == 2) {
-        ov = __bfloat162float(o[c]);
-        gv = __bfloat162float(g[c]);
-      } else {
-        ov = o[c];
-        gv = g[c];
+      for (int k = 0; k < 2; ++k) {
+        // bf16 -> float: the bf16 bits are the high half of the float's
+        acc = fmaf(__uint_as_float(ov[k] << 16), __uint_as_float(gv[k] << 16), acc);
+        acc = fmaf(__uint_as_float(ov[k] & 0xffff0000u), __uint_as_float(gv[k] & 0xffff0000u),
+                   acc);
       }
-      acc = fmaf(ov, gv, acc);
+    } else {
+#pragma unroll
+      for (int c = lane; c < D; c += 32) {
+        float ov, gv;
+        if constexpr (sizeof(T) == 2) {
+          ov = __bfloat162float(o[c]);
+          gv = __bfloat162float(g[c]);
+        } else {
+          ov = o[c];
+          gv = g[c];
+        }
+        acc = fmaf(ov, gv, acc);
+      }
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
