@@ -117,6 +117,50 @@ static int gpu_checks(void) {
   CHECK(max_o <= 2e-2, "output off the running mean by %g", max_o);
   CHECK(max_l <= 1e-3, "lse off ln(i+1) by %g", max_l);
   printf("max |out - mean| %g, max |lse - ln(i+1)| %g\n", max_o, max_l);
+
+  /* The same attention as two ring steps through the block entry points:
+   * keys [0, 128) then keys [128, 300) (a ragged block whose diagonal
+   * starts one tile in), folded into a running float32 (O, lse). */
+  float *oacc, *lacc;
+  void* dout2;
+  if (cudaMalloc((void**)&oacc, n * 4) || cudaMalloc((void**)&lacc, (size_t)H * S * 4) ||
+      cudaMalloc(&dout2, n * 2)) {
+    fprintf(stderr, "cudaMalloc failed\n");
+    return 1;
+  }
+  const size_t row = (size_t)H * D; /* elements per token */
+  lca_block_shape b1 = {1, H, H, S, 128, D, LCA_BF16, 0.0f};
+  lca_block_shape b2 = {1, H, H, S, S - 128, D, LCA_BF16, 0.0f};
+  CHECK(lca_attn_fwd_block(&b1, dq, dk, dv, 1, 0, 0, 0, oacc, lacc, NULL, NULL) == LCA_OK,
+        "first block: %s", lca_last_error());
+  CHECK(lca_attn_fwd_block(&b2, dq, (uint16_t*)dk + 128 * row, (uint16_t*)dv + 128 * row, 1, 0,
+                           128, 1, oacc, lacc, dout2, NULL) == LCA_OK,
+        "second block: %s", lca_last_error());
+  CHECK(lca_check(NULL) == LCA_OK, "lca_check: %s", lca_last_error());
+  cudaMemcpy(ho, dout2, n * 2, cudaMemcpyDeviceToHost);
+  cudaMemcpy(hl, lacc, (size_t)H * S * 4, cudaMemcpyDeviceToHost);
+  max_o = 0.0;
+  max_l = 0.0;
+  for (int h = 0; h < H; ++h) {
+    for (int c = 0; c < D; ++c) {
+      double run = 0.0;
+      for (int i = 0; i < S; ++i) {
+        run += from_bf16(hv[((size_t)i * H + h) * D + c]);
+        const double got = from_bf16(ho[((size_t)i * H + h) * D + c]);
+        if (fabs(got - run / (i + 1)) > max_o) max_o = fabs(got - run / (i + 1));
+      }
+    }
+    for (int i = 0; i < S; ++i) {
+      const double e = fabs(hl[(size_t)h * S + i] - log((double)(i + 1)));
+      if (e > max_l) max_l = e;
+    }
+  }
+  CHECK(max_o <= 2e-2, "block output off the running mean by %g", max_o);
+  CHECK(max_l <= 1e-3, "block lse off ln(i+1) by %g", max_l);
+  printf("blocks: max |out - mean| %g, max |lse - ln(i+1)| %g\n", max_o, max_l);
+  cudaFree(oacc);
+  cudaFree(lacc);
+  cudaFree(dout2);
   cudaFree(dq);
   cudaFree(dk);
   cudaFree(dv);

@@ -1,4 +1,5 @@
-"""The C ABI from plain C: tests/host/abi_c_probe.c is compiled with gcc
+"""The C ABI from plain C (a forward and a two-block ring step checked against
+a closed form on the GPU): tests/host/abi_c_probe.c is compiled with gcc
 against include/lca.h and liblca.so (no Python, no torch in the client).
 The CPU part checks status strings and synchronous argument errors; the GPU
 part runs a causal forward whose answer is a closed form (zero keys: each
