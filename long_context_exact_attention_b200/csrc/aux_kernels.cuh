@@ -19,7 +19,9 @@
 namespace lca {
 
 // One warp per padded row (sequence b, position s < S_pad, head h), h
-// fastest so that neighbouring warps read neighbouring memory.  Sequence b
+// fastest so that neighbouring warps read neighbouring memory.  acc_zero
+// (dense batches only, else null): the float32 dq accumulator, whose row
+// of each visited (b, s, h) is zeroed on the way.  Sequence b
 // occupies tensor rows [b*S, b*S + S) or, packed, [cu[b], cu[b+1]); lse is
 // [B,H,S] or, packed, [H, total].  Writes D and a copy of lse into
 // [B,H,S_pad] arrays; positions past a sequence's end get D = 0 and
@@ -30,7 +32,7 @@ template <typename T, int D>
 __global__ void bwd_rowdot(const T* __restrict__ out, const T* __restrict__ dout,
                            const float* __restrict__ lse, float* __restrict__ Dst,
                            float* __restrict__ lse_pad, int B, int S, int S_pad, int H,
-                           const int* __restrict__ cu_seqlens) {
+                           const int* __restrict__ cu_seqlens, float* __restrict__ acc_zero) {
   const int lane = threadIdx.x & 31;
   const int64_t n = static_cast<int64_t>(B) * S_pad * H;
   const int64_t warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
@@ -66,6 +68,14 @@ __global__ void bwd_rowdot(const T* __restrict__ out, const T* __restrict__ dout
     }
     const T* o = out + ((r0 + s) * H + h) * D;
     const T* g = dout + ((r0 + s) * H + h) * D;
+    if (acc_zero) {
+      // the row's float32 dq accumulator starts at zero (dense batches,
+      // where the rows visited here are every row of the accumulator)
+      float* z = acc_zero + ((r0 + s) * H + h) * D;
+#pragma unroll
+      for (int c = 4 * lane; c < D; c += 128)
+        *reinterpret_cast<float4*>(z + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     float acc = 0.f;
     if constexpr (sizeof(T) == 2 && D == 128) {
       // one 8-byte word (four bf16) of each row per lane: the warp reads

@@ -470,12 +470,16 @@ lca_status bwd_prep(const Common& c, const void* out, const float* lse, const vo
   const int64_t pad_rows = static_cast<int64_t>(c.n_seq) * S_pad * c.Hq;
   const unsigned rd_blocks =
       static_cast<unsigned>(std::min<int64_t>((pad_rows * 32 + 255) / 256, 148 * 64));
-  const cudaError_t e =
-      cudaMemsetAsync(acc, 0, static_cast<size_t>(rows) * c.d * sizeof(float), st);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(dq accumulator)");
+  // A dense batch: the row-dot visits every row of the accumulator and
+  // zeroes it on the way; a packed one may leave rows between sequences.
+  if (c.cu) {
+    const cudaError_t e =
+        cudaMemsetAsync(acc, 0, static_cast<size_t>(rows) * c.d * sizeof(float), st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(dq accumulator)");
+  }
   bwd_rowdot<__nv_bfloat16, 128><<<rd_blocks, 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse, Drow,
-      lse_pad, c.n_seq, c.S, S_pad, c.Hq, c.cu);
+      lse_pad, c.n_seq, c.S, S_pad, c.Hq, c.cu, c.cu ? nullptr : acc);
   return launched("bwd_rowdot");
 }
 
@@ -584,12 +588,13 @@ lca_status run_bwd(const Common& c, const AttnSched& s, const void* q, const voi
   if (c.d == 64)
     bwd_rowdot<float, 64><<<rd_blocks, 256, 0, st>>>(static_cast<const float*>(out),
                                                        static_cast<const float*>(dout), lse, Drow,
-                                                       lse_pad, c.n_seq, c.S, S_pad, c.Hq, c.cu);
+                                                       lse_pad, c.n_seq, c.S, S_pad, c.Hq, c.cu,
+                                                       nullptr);
   else
     bwd_rowdot<float, 128><<<rd_blocks, 256, 0, st>>>(static_cast<const float*>(out),
                                                         static_cast<const float*>(dout), lse,
                                                         Drow, lse_pad, c.n_seq, c.S, S_pad, c.Hq,
-                                                        c.cu);
+                                                        c.cu, nullptr);
   if ((r = launched("bwd_rowdot")) != LCA_OK) return r;
   f32::Args a{};
   a.q = static_cast<const float*>(q);
