@@ -57,11 +57,14 @@ constexpr uint32_t kHalf = kTile * 64 * 2;
 constexpr uint32_t kTileB = 2 * kHalf;
 constexpr int kThreads = 512;
 // Registers per thread at launch (launch bounds 512 x 1 CTA) and the split
-// the warpgroups take with setmaxnreg: 56 + 3 * 152 = 4 * 128.
+// the warpgroups take with setmaxnreg: control 56, the two P/dS warpgroups
+// 160 each, the dQ warpgroup 136 (56 + 2 * 160 + 136 = 4 * 128; the dQ
+// warpgroup spills below 128, the control one below 56).
 constexpr int kRegsLaunch = 128;
 constexpr int kRegsCtl = 56;
-constexpr int kRegsWork = 152;
-static_assert(kRegsCtl + 3 * kRegsWork == 4 * kRegsLaunch, "register split");
+constexpr int kRegsWork = 160;
+constexpr int kRegsDq = 136;
+static_assert(kRegsCtl + 2 * kRegsWork + kRegsDq == 4 * kRegsLaunch, "register split");
 
 constexpr uint32_t kOffK = 0;
 constexpr uint32_t kOffV = kOffK + kTileB;
@@ -450,7 +453,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       }
     }
   } else {
-    regs_inc<kRegsWork>();
+    regs_inc<kRegsDq>();
     // =================================================== dQ warpgroup
     const int wq = warp & 3;
     const int r = wq * 32 + lane;  // head dim (dQ^T) / key row (dV)
